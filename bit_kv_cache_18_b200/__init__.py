@@ -1,0 +1,203 @@
+"""Python binding of libkvq.so, the B200 (sm_100a) quantized paged KV cache.
+
+Argument marshalling only: every step of the write and read paths runs in the
+library's CUDA kernels.  The names mirror include/kvq.h.  Torch is used for
+device memory, dtypes and streams.  There is no fallback: if libkvq.so is
+missing or fails to load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+import threading
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libkvq.so")
+HEADER = os.path.join(os.path.dirname(PKG), "include", "kvq.h")
+
+KVQ_OK = 0
+KVQ_ERR_INVALID = -1
+KVQ_ERR_UNSUPPORTED = -2
+KVQ_ERR_CUDA = -3
+KVQ_ERR_POOL_EXHAUSTED = -4
+KVQ_ERR_OUT_OF_RANGE = -5
+KVQ_ERR_DEVICE_TIMEOUT = -6
+KVQ_ERR_WORKSPACE = -7
+
+KVQ_F16, KVQ_BF16, KVQ_F32 = 0, 1, 2
+
+HEAD_DIM = 128
+BLOCK_SIZE = 16
+SEGMENT_BYTES = 1664
+
+_lock = threading.Lock()
+_lib = None
+
+
+class KvqError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {kvq_error_string(status)} ({status})")
+
+
+class CacheDesc(ctypes.Structure):
+    _fields_ = [("num_blocks", ctypes.c_int32), ("block_size", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("k_bits", ctypes.c_int32), ("v_bits", ctypes.c_int32), ("group", ctypes.c_int32),
+                ("pool", ctypes.c_void_p)]
+
+
+def lib():
+    """Load libkvq.so (raises if it is absent: there is no other path)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"{LIB_PATH} is missing; build it with python -m bit_kv_cache_18_b200.build")
+            L = ctypes.CDLL(LIB_PATH)
+            i32, i64, u64, sz, vp, f32 = (ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64, ctypes.c_size_t,
+                                          ctypes.c_void_p, ctypes.c_float)
+            dp = ctypes.POINTER(CacheDesc)
+            sig = {
+                "kvq_parse_dtype": (ctypes.c_int, [ctypes.c_char_p, vp, vp, vp]),
+                "kvq_cache_bytes": (sz, [dp]),
+                "kvq_block_table": (ctypes.c_int, [i32, i32, vp, i32, i32, u64, vp, vp]),
+                "kvq_slot_mapping": (ctypes.c_int, [vp, i32, vp, vp, i32, i32, vp]),
+                "kvq_quantize_append": (ctypes.c_int, [dp, vp, vp, ctypes.c_int, i32, i64, vp, vp]),
+                "kvq_decode_workspace_bytes": (sz, [dp, i32, i32, i32]),
+                "kvq_decode_workspace_bytes_ex": (sz, [dp, i32, i32, i32, i32]),
+                "kvq_decode_attention": (ctypes.c_int, [dp, vp, ctypes.c_int, i32, i32, vp, i32, vp, i32, f32, vp,
+                                                        ctypes.c_int, vp, sz, vp]),
+                "kvq_decode_attention_ex": (ctypes.c_int, [dp, vp, ctypes.c_int, i32, i32, vp, i32, vp, i32, f32,
+                                                           vp, ctypes.c_int, vp, sz, i32, vp]),
+                "kvq_last_device_status": (ctypes.c_int, [vp]),
+                "kvq_error_string": (ctypes.c_char_p, [ctypes.c_int]),
+            }
+            for name, (res, args) in sig.items():
+                f = getattr(L, name)
+                f.restype, f.argtypes = res, args
+            _lib = L
+    return _lib
+
+
+def header_functions() -> list[str]:
+    """Names of the functions include/kvq.h declares."""
+    with open(HEADER) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kvq_[a-z_]+)\s*\(", text)))
+
+
+def kvq_error_string(status: int) -> str:
+    return lib().kvq_error_string(status).decode()
+
+
+def _check(rc: int, what: str):
+    if rc != KVQ_OK:
+        raise KvqError(rc, what)
+
+
+def _stream_ptr(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t) -> int:
+    import torch
+    return {torch.float16: KVQ_F16, torch.bfloat16: KVQ_BF16, torch.float32: KVQ_F32}[t.dtype]
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+# ---- host-only helpers -------------------------------------------------------
+
+def kvq_parse_dtype(s: str):
+    kb, vb, g = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+    rc = lib().kvq_parse_dtype(s.encode(), ctypes.byref(kb), ctypes.byref(vb), ctypes.byref(g))
+    return rc, (kb.value, vb.value, g.value)
+
+
+def make_desc(num_blocks: int, num_kv_heads: int, pool=None) -> CacheDesc:
+    return CacheDesc(num_blocks, BLOCK_SIZE, num_kv_heads, HEAD_DIM, 4, 2, HEAD_DIM,
+                     pool.data_ptr() if pool is not None else None)
+
+
+def kvq_cache_bytes(desc: CacheDesc) -> int:
+    return lib().kvq_cache_bytes(ctypes.byref(desc))
+
+
+def kvq_block_table(num_blocks, seq_lens, max_blocks_per_seq, shuffle_seed=0, block_size=BLOCK_SIZE):
+    """-> (block_table int32 numpy [batch, max_blocks_per_seq], blocks_used)"""
+    import numpy as np
+    lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    out = np.empty((lens.size, max_blocks_per_seq), dtype=np.int32)
+    used = ctypes.c_int32()
+    _check(lib().kvq_block_table(num_blocks, block_size, lens.ctypes.data, lens.size, max_blocks_per_seq,
+                                 shuffle_seed, out.ctypes.data, ctypes.byref(used)), "kvq_block_table")
+    return out, used.value
+
+
+def kvq_slot_mapping(block_table, positions, seq_ids, block_size=BLOCK_SIZE):
+    import numpy as np
+    bt = np.ascontiguousarray(block_table, dtype=np.int32)
+    pos = np.ascontiguousarray(positions, dtype=np.int32)
+    sid = np.ascontiguousarray(seq_ids, dtype=np.int32)
+    out = np.empty(pos.size, dtype=np.int32)
+    _check(lib().kvq_slot_mapping(bt.ctypes.data, bt.shape[1], pos.ctypes.data, sid.ctypes.data, pos.size,
+                                  block_size, out.ctypes.data), "kvq_slot_mapping")
+    return out
+
+
+# ---- device calls ------------------------------------------------------------
+
+def new_pool(num_blocks: int, num_kv_heads: int, device="cuda"):
+    """A caller-owned pool tensor (uint8) sized by kvq_cache_bytes."""
+    import torch
+    nbytes = kvq_cache_bytes(make_desc(num_blocks, num_kv_heads))
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device)
+
+
+def kvq_quantize_append(pool, num_blocks, num_kv_heads, k, v, slot_mapping, stream=None, token_stride=None):
+    """k, v: [n_tokens, ..., Hkv*128 elements per row] fp16/bf16 device tensors
+    with stride(0) = token_stride; slot_mapping: int32 device [n_tokens]."""
+    desc = make_desc(num_blocks, num_kv_heads, pool)
+    n = int(slot_mapping.numel())
+    ts = k.stride(0) if token_stride is None else token_stride
+    rc = lib().kvq_quantize_append(ctypes.byref(desc), _ptr(k), _ptr(v), _dtype_code(k), n, ts, _ptr(slot_mapping),
+                                   _stream_ptr(stream))
+    _check(rc, "kvq_quantize_append")
+
+
+def kvq_decode_workspace_bytes(num_blocks, num_kv_heads, batch, num_q_heads, max_seq_len, blocks_per_split=0):
+    desc = make_desc(num_blocks, num_kv_heads)
+    return lib().kvq_decode_workspace_bytes_ex(ctypes.byref(desc), batch, num_q_heads, max_seq_len,
+                                               blocks_per_split)
+
+
+def new_workspace(num_blocks, num_kv_heads, batch, num_q_heads, max_seq_len, blocks_per_split=0, device="cuda"):
+    import torch
+    n = kvq_decode_workspace_bytes(num_blocks, num_kv_heads, batch, num_q_heads, max_seq_len, blocks_per_split)
+    if n == 0:
+        raise KvqError(KVQ_ERR_UNSUPPORTED, "kvq_decode_workspace_bytes")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def kvq_decode_attention(pool, num_blocks, num_kv_heads, q, block_table, seq_lens, max_seq_len, out, workspace,
+                         softmax_scale=0.0, blocks_per_split=0, stream=None):
+    """q: [batch, Hq, 128] device; block_table int32 [batch, max_blocks]; seq_lens int32 [batch];
+    out: [batch, Hq, 128] device (fp32/bf16/fp16); workspace from new_workspace()."""
+    desc = make_desc(num_blocks, num_kv_heads, pool)
+    batch, hq, _ = q.shape
+    rc = lib().kvq_decode_attention_ex(ctypes.byref(desc), _ptr(q), _dtype_code(q), batch, hq, _ptr(block_table),
+                                       block_table.shape[1], _ptr(seq_lens), max_seq_len, softmax_scale, _ptr(out),
+                                       _dtype_code(out), _ptr(workspace), workspace.numel(), blocks_per_split,
+                                       _stream_ptr(stream))
+    _check(rc, "kvq_decode_attention")
+
+
+def kvq_last_device_status(stream=None) -> int:
+    return lib().kvq_last_device_status(_stream_ptr(stream))

@@ -1,0 +1,116 @@
+// kvq_internal.cuh -- shared pieces of the sm_100a KV-cache kernels.
+//
+// Format constants of the k4v2_g128 pool (see include/kvq.h for the layout and
+// the pages it follows), the device status word, small PTX wrappers and the
+// launcher entry points that kvq_host.cu calls.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kvq.h"
+
+namespace kvq {
+
+// ---- pool format (k4v2_g128, 16-token blocks) ------------------------------
+constexpr int kHeadDim = 128;
+constexpr int kBlockSize = 16;
+constexpr int kKBits = 4;
+constexpr int kVBits = 2;
+constexpr int kKRowBytes = kHeadDim * kKBits / 8;  // 64
+constexpr int kVRowBytes = kHeadDim * kVBits / 8;  // 32
+constexpr int kOffK = 0;
+constexpr int kOffV = kOffK + kBlockSize * kKRowBytes;  // 1024
+constexpr int kOffSK = kOffV + kBlockSize * kVRowBytes;  // 1536
+constexpr int kOffZK = kOffSK + 2 * kBlockSize;          // 1568
+constexpr int kOffSV = kOffZK + 2 * kBlockSize;          // 1600
+constexpr int kOffZV = kOffSV + 2 * kBlockSize;          // 1632
+constexpr int kSegBytes = kOffZV + 2 * kBlockSize;       // 1664
+static_assert(kSegBytes == 1664, "segment size");
+static_assert(kSegBytes % 128 == 0, "segments stay 128-byte aligned");
+
+// Split-K partial record in the decode workspace: o~[128], m (log2 domain), l.
+constexpr int kPartialFloats = kHeadDim + 4;
+
+// ---- device status word ----------------------------------------------------
+// One int per device (a module-scope __device__ variable in kvq_host.cu whose
+// address the host looks up once per device and passes to every kernel).
+// Kernels record the first error with a compare-and-swap from 0;
+// kvq_last_device_status reads and clears it.
+__device__ __forceinline__ void record_status(int* status, int code) { atomicCAS(status, 0, code); }
+int* device_status_ptr();  // nullptr if the lookup failed
+
+// ---- small helpers -----------------------------------------------------------
+__device__ __forceinline__ float bf16lo_to_f32(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi_to_f32(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ float load_as_f32(const void* p, int dtype, int64_t i) {
+  if (dtype == KVQ_F32) return static_cast<const float*>(p)[i];
+  const uint16_t u = static_cast<const uint16_t*>(p)[i];
+  if (dtype == KVQ_BF16) return __uint_as_float(static_cast<uint32_t>(u) << 16);
+  return __half2float(__ushort_as_half(u));
+}
+
+__device__ __forceinline__ void store_from_f32(void* p, int dtype, int64_t i, float v) {
+  if (dtype == KVQ_F32)
+    static_cast<float*>(p)[i] = v;
+  else if (dtype == KVQ_BF16)
+    static_cast<__nv_bfloat16*>(p)[i] = __float2bfloat16_rn(v);
+  else
+    static_cast<__half*>(p)[i] = __float2half_rn(v);
+}
+
+// ---- launchers (return cudaError_t of the launch) ---------------------------
+struct QuantizeArgs {
+  uint8_t* pool;
+  int32_t num_blocks;
+  int32_t num_kv_heads;
+  const void* k;
+  const void* v;
+  int32_t in_dtype;
+  int32_t n_tokens;
+  int64_t token_stride;
+  const int32_t* slots;
+  int* status;
+};
+cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream);
+
+struct DecodeArgs {
+  const uint8_t* pool;
+  int32_t num_blocks;
+  int32_t num_kv_heads;
+  const void* q;
+  int32_t q_dtype;
+  int32_t batch;
+  int32_t num_q_heads;
+  const int32_t* block_table;
+  int32_t max_blocks_per_seq;
+  const int32_t* seq_lens;
+  int32_t max_seq_len;
+  float scale_log2;  // softmax scale times log2(e)
+  void* out;
+  int32_t out_dtype;
+  int32_t* tickets;   // [batch * num_kv_heads]
+  float* partials;    // [batch, num_q_heads, nsplit, kPartialFloats]
+  int32_t blocks_per_split;
+  int32_t nsplit;
+  int* status;
+};
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+
+// Split-K plan of a decode call on the current device.
+struct DecodePlan {
+  int32_t blocks_per_split;
+  int32_t nsplit;
+  size_t ticket_bytes;   // rounded up to 256
+  size_t partial_bytes;
+  size_t total_bytes;
+};
+int plan_decode(int32_t batch, int32_t num_kv_heads, int32_t num_q_heads, int32_t max_seq_len,
+                int32_t blocks_per_split_request, DecodePlan* plan);
+
+int device_sm_count();
+
+}  // namespace kvq

@@ -1,0 +1,192 @@
+/*
+ * kvq.h -- C ABI of the B200 (sm_100a) KVarN-style quantized paged KV cache.
+ *
+ * What the library computes.  The KVarN pages describe a vLLM attention
+ * backend whose cache blocks go through a Hadamard rotation, a variance
+ * normalisation and asymmetric low-bit quantisation (4-bit keys, 2-bit values
+ * by default, preset flag kvarn_k4v2_g128), with the group scales folded into
+ * attention at read time:
+ *   - "Трюк Huawei с KV-кэшем" (beyondheadline.xyz), lede and section
+ *     "Заявка, которая ломает привычный компромисс";
+ *   - "KVarN vs TurboQuant" (dothoosh.com), the four-stage pipeline list and
+ *     the kv_cache_dtype flag paragraph.
+ * The pages give no formula or layout; the library fixes them as follows.
+ *
+ * Write path, per 128-element K or V head vector x of one token:
+ *   r = R x, R = H/sqrt(128), H the natural-order Sylvester Hadamard matrix;
+ *   mu, sigma = mean and population standard deviation of r (sigma = 0 -> 1);
+ *   u = (r - mu)/sigma, lo = min u, hi = max u;
+ *   S = fp16(sigma (hi - lo)/(2^b - 1)), Z = fp16(mu + sigma lo)   [g128]
+ *   c_i = clamp(rne((r_i - Z)/S), 0, 2^b - 1) (all 0 when S == 0), b = 4 for
+ *   keys and 2 for values.  Dequantized vector: x^ = R (S c + Z).
+ *
+ * Read path (decode), for query head j of sequence b, kv head h = j / G,
+ * G = Hq/Hkv, tau = softmax_scale (<= 0 means 1/sqrt(128)):
+ *   o = sum_t softmax_t(tau <q, k^_t>) v^_t over the seq_lens[b] cached
+ *   tokens.  The kernel computes it with the scales folded in: q~ = R q once,
+ *   s_t = tau (S_K,t <q~, c_K,t> + Z_K,t sum(q~)), o~ = sum_t p_t (S_V,t c_V,t
+ *   + Z_V,t), o = R o~ once.
+ *
+ * Pool layout (the ABI; the pages leave it open).  A pool is num_blocks
+ * physical blocks of block_size (16) token slots for each of num_kv_heads
+ * heads.  Segment (p, h) starts at byte (p*num_kv_heads + h) * 1664 and holds
+ *   [0,1024)    K codes, 16 rows of 64 B; element i at byte i/2, low nibble
+ *               for even i
+ *   [1024,1536) V codes, 16 rows of 32 B; element i at byte i/4, bits 2(i%4)
+ *   [1536,1568) S_K[16]  [1568,1600) Z_K[16]
+ *   [1600,1632) S_V[16]  [1632,1664) Z_V[16]          (fp16, little endian)
+ * Slot s of the pool is block s/16, row s%16 (vLLM slot mapping).  That is
+ * 104 bytes per token per kv head against 512 for an fp16 cache (4.92x).
+ *
+ * Conventions.
+ *   - The caller owns every buffer.  Device pointers are CUDA device memory
+ *     of the current device; host pointers are ordinary host memory.  The
+ *     library allocates nothing and keeps no state except cached device
+ *     attributes and one device status word per device (see
+ *     kvq_last_device_status).
+ *   - Calls that take a stream are asynchronous on that stream (a
+ *     cudaStream_t passed as void*, NULL = legacy default stream) and return
+ *     after validating arguments and enqueueing work.
+ *   - Every entry point returns 0 (KVQ_OK) or a negative kvq_status.  No
+ *     exception, abort or device trap ever leaves the library: argument
+ *     errors are caught on the host; out-of-range block ids and slots met on
+ *     the device are skipped and recorded in the device status word.
+ *   - Supported geometry: head_dim 128, group 128, block_size 16, k_bits 4,
+ *     v_bits 2, num_q_heads a multiple of num_kv_heads with G = Hq/Hkv in
+ *     {1, 2, 4, 8}.  Anything else returns KVQ_ERR_UNSUPPORTED.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KVQ_OK = 0,
+  KVQ_ERR_INVALID = -1,        /* null pointer, negative size, bad enum value */
+  KVQ_ERR_UNSUPPORTED = -2,    /* geometry or preset the kernels do not cover */
+  KVQ_ERR_CUDA = -3,           /* a CUDA runtime call failed (launch, query)  */
+  KVQ_ERR_POOL_EXHAUSTED = -4, /* kvq_block_table: not enough physical blocks */
+  KVQ_ERR_OUT_OF_RANGE = -5,   /* block id or slot outside the pool           */
+  KVQ_ERR_DEVICE_TIMEOUT = -6, /* a bounded device-side wait gave up          */
+  KVQ_ERR_WORKSPACE = -7       /* workspace missing, misaligned or too small  */
+} kvq_status;
+
+typedef enum { KVQ_F16 = 0, KVQ_BF16 = 1, KVQ_F32 = 2 } kvq_dtype;
+
+/* One cache pool.  pool is device memory of kvq_cache_bytes(desc) bytes,
+ * 16-byte aligned, owned by the caller; its initial contents do not matter. */
+typedef struct {
+  int32_t num_blocks;   /* physical blocks in the pool (>= 0)             */
+  int32_t block_size;   /* token slots per block: 16                      */
+  int32_t num_kv_heads; /* Hkv >= 1                                       */
+  int32_t head_dim;     /* 128                                            */
+  int32_t k_bits;       /* 4                                              */
+  int32_t v_bits;       /* 2                                              */
+  int32_t group;        /* elements per scale/zero group: 128 (= head_dim) */
+  void* pool;           /* device pointer                                 */
+} kvq_cache_desc;
+
+/* Parse a cache dtype string of the form "kvarn_k<kb>v<vb>_g<g>", the vLLM
+ * flag named on the KVarN pages ("KVarN vs TurboQuant", flag paragraph).
+ * Host only.  Writes the three numbers and returns KVQ_OK for a well-formed
+ * string (KVQ_ERR_UNSUPPORTED if it is well formed but not k4v2_g128),
+ * KVQ_ERR_INVALID otherwise.  Output pointers may not be NULL. */
+int kvq_parse_dtype(const char* s, int32_t* k_bits, int32_t* v_bits, int32_t* group);
+
+/* Bytes of the pool described by desc (num_blocks * num_kv_heads * 1664 for
+ * k4v2_g128), or 0 if desc is NULL or unsupported.  Host only. */
+size_t kvq_cache_bytes(const kvq_cache_desc* desc);
+
+/* Assign physical blocks to sequences, host only (no device work).
+ * Sequence b needs ceil(seq_lens[b]/block_size) blocks, which are taken in
+ * order from a permutation of 0..num_blocks-1: the identity when
+ * shuffle_seed == 0, otherwise a seeded shuffle (SplitMix64-driven
+ * Fisher-Yates), as a fragmented vLLM block manager would hand them out.
+ * block_table_out is [batch * max_blocks_per_seq] host int32, row-major,
+ * unused entries set to -1; *blocks_used_out (may be NULL) gets the total.
+ * Returns KVQ_ERR_POOL_EXHAUSTED if the pool is too small and
+ * KVQ_ERR_INVALID if a sequence needs more than max_blocks_per_seq blocks. */
+int kvq_block_table(int32_t num_blocks, int32_t block_size, const int32_t* seq_lens, int32_t batch,
+                    int32_t max_blocks_per_seq, uint64_t shuffle_seed, int32_t* block_table_out,
+                    int32_t* blocks_used_out);
+
+/* slots_out[i] = block_table[seq_ids[i]][positions[i]/block_size] *
+ * block_size + positions[i] % block_size, host only.  An entry whose block
+ * is -1 gives -1 (the write path then skips that token).  All pointers are
+ * host memory; returns KVQ_ERR_INVALID for a negative position or a position
+ * beyond the table row. */
+int kvq_slot_mapping(const int32_t* block_table, int32_t max_blocks_per_seq,
+                     const int32_t* positions, const int32_t* seq_ids, int32_t n_tokens,
+                     int32_t block_size, int32_t* slots_out);
+
+/* Cache write (the write path above, one kernel launch).
+ * k, v: device, n_tokens rows; row t starts at element t*token_stride and
+ * holds [num_kv_heads, 128] contiguous elements of in_dtype (F16 or BF16);
+ * token_stride >= num_kv_heads*128 and a multiple of 8; k and v 16-byte
+ * aligned.  slot_mapping: device int32 [n_tokens]; a negative slot skips the
+ * token; a slot at or beyond num_blocks*16 is skipped and recorded as
+ * KVQ_ERR_OUT_OF_RANGE in the device status word.  n_tokens == 0 is a no-op.
+ * Tokens with distinct slots may share a block. */
+int kvq_quantize_append(const kvq_cache_desc* desc, const void* k, const void* v,
+                        kvq_dtype in_dtype, int32_t n_tokens, int64_t token_stride,
+                        const int32_t* slot_mapping, void* stream);
+
+/* Workspace bytes kvq_decode_attention needs for this problem on the current
+ * device (split-K partials plus one int32 ticket per (sequence, kv head)),
+ * or 0 for an unsupported geometry.  Host only (reads cached device
+ * attributes). */
+size_t kvq_decode_workspace_bytes(const kvq_cache_desc* desc, int32_t batch, int32_t num_q_heads,
+                                  int32_t max_seq_len);
+
+/* Decode attention over the packed cache (the read path above, one kernel
+ * launch: query rotation, paged split-K scan with scale folding, in-kernel
+ * split combine by atomic ticket, output rotation).
+ * q: device [batch, num_q_heads, 128] of q_dtype (F16, BF16 or F32).
+ * block_table: device int32 [batch, max_blocks_per_seq]; seq_lens: device
+ * int32 [batch], each in [0, max_seq_len]; max_seq_len sizes the split
+ * grid and must be >= every seq_lens[b] (a longer sequence is truncated and
+ * recorded as KVQ_ERR_OUT_OF_RANGE).  out: device [batch, num_q_heads, 128]
+ * of out_dtype (F32, BF16 or F16); a sequence of length 0 gives zeros.
+ * workspace: device, 16-byte aligned, at least kvq_decode_workspace_bytes
+ * bytes, zero-filled by the caller once before its first use; every call
+ * leaves it ready for the next call (tickets reset themselves).  Calls that
+ * share a workspace must be ordered on one stream.  A block id outside the
+ * pool is read as nothing (the token is skipped) and recorded as
+ * KVQ_ERR_OUT_OF_RANGE in the device status word. */
+int kvq_decode_attention(const kvq_cache_desc* desc, const void* q, kvq_dtype q_dtype,
+                         int32_t batch, int32_t num_q_heads, const int32_t* block_table,
+                         int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                         int32_t max_seq_len, float softmax_scale, void* out,
+                         kvq_dtype out_dtype, void* workspace, size_t ws_bytes, void* stream);
+
+/* As kvq_decode_attention / kvq_decode_workspace_bytes, with the split-K
+ * granularity chosen by the caller: blocks_per_split physical blocks (of 16
+ * tokens) per CTA; 0 picks the default.  The workspace size depends on it. */
+size_t kvq_decode_workspace_bytes_ex(const kvq_cache_desc* desc, int32_t batch,
+                                     int32_t num_q_heads, int32_t max_seq_len,
+                                     int32_t blocks_per_split);
+int kvq_decode_attention_ex(const kvq_cache_desc* desc, const void* q, kvq_dtype q_dtype,
+                            int32_t batch, int32_t num_q_heads, const int32_t* block_table,
+                            int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                            int32_t max_seq_len, float softmax_scale, void* out,
+                            kvq_dtype out_dtype, void* workspace, size_t ws_bytes,
+                            int32_t blocks_per_split, void* stream);
+
+/* Synchronise the stream, then read and clear the current device's status
+ * word: KVQ_OK, or the first error that a kernel recorded since the last
+ * read (KVQ_ERR_OUT_OF_RANGE, KVQ_ERR_DEVICE_TIMEOUT).  Returns
+ * KVQ_ERR_CUDA if the synchronisation itself fails. */
+int kvq_last_device_status(void* stream);
+
+/* Static description of a status code; never NULL. */
+const char* kvq_error_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KVQ_H */

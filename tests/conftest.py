@@ -24,3 +24,22 @@ def syn():
     import synth
     synth._load()
     return synth
+
+
+@pytest.fixture(scope="session")
+def kvq():
+    """The C-ABI library's Python binding, built in-tree if missing (nvcc)."""
+    from bit_kv_cache_18_b200 import build
+    import bit_kv_cache_18_b200 as m
+    if not os.path.exists(m.LIB_PATH):
+        build.build()
+    m.lib()
+    return m
+
+
+@pytest.fixture(scope="session")
+def cuda():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return torch.device("cuda:0")

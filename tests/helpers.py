@@ -1,0 +1,92 @@
+"""Parity checking used by the GPU tests.
+
+The rules for comparing a quantized pool written by the CUDA kernel with the
+oracle's (the two compute in different precisions, so exact agreement is
+required only away from rounding boundaries):
+  - codes must be bit-exact, except at near-ties: an element whose oracle
+    quotient (r_i - Z)/S lies within 1e-3 of k + 1/2 may differ by one code;
+    such mismatches may make up at most 1e-4 of all elements;
+  - S and Z must be bit-exact, except in a group whose exact (unrounded)
+    value lies within 1e-3 of an fp16 ulp from a rounding midpoint, where
+    they may differ by one ulp; the codes of such a group are then checked
+    against the codes the oracle computes from the GPU's S and Z.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+import oracle
+
+NEAR_TIE = 1e-3
+MAX_MISMATCH_FRACTION = 1e-4
+ATTN_TOL = 2e-3
+
+
+def to_f64(bits: np.ndarray, dtype: int) -> np.ndarray:
+    if dtype == oracle.F16:
+        return bits.view(np.float16).astype(np.float64)
+    if dtype == oracle.BF16:
+        return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return bits.astype(np.float64)
+
+
+def _near_midpoint(exact: float, a: int, b: int) -> bool:
+    va, vb = oracle.f16_to_f64(a), oracle.f16_to_f64(b)
+    ulp = abs(va - vb)
+    return abs(int(a) - int(b)) == 1 and abs(exact - (va + vb) / 2) <= NEAR_TIE * ulp
+
+
+class QuantReport:
+    def __init__(self):
+        self.vectors = 0
+        self.elements = 0
+        self.code_mismatches = 0
+        self.meta_mismatch_groups = 0
+        self.failures: list[str] = []
+
+    def ok(self) -> bool:
+        return not self.failures and self.code_mismatches <= MAX_MISMATCH_FRACTION * max(self.elements, 1)
+
+    def __repr__(self):
+        return (f"QuantReport(vectors={self.vectors}, code_mismatches={self.code_mismatches}/{self.elements}, "
+                f"meta_1ulp_groups={self.meta_mismatch_groups}, failures={self.failures[:5]})")
+
+
+def check_vector(rep: QuantReport, x: np.ndarray, bits: int, gpu_codes, gpu_S: int, gpu_Z: int, where: str):
+    """One group: GPU codes/metadata against the oracle under the rules above."""
+    codes, S, Z, r = oracle.quantize_vector(x, bits)
+    rep.vectors += 1
+    rep.elements += codes.size
+    if (gpu_S, gpu_Z) != (S, Z):
+        s_ex, z_ex = oracle.meta_exact(x, bits)
+        for name, ex, a, b in (("S", s_ex, gpu_S, S), ("Z", z_ex, gpu_Z, Z)):
+            if a != b and not _near_midpoint(ex, a, b):
+                rep.failures.append(f"{where}: {name} gpu={a:#06x} oracle={b:#06x} exact={ex!r}")
+                return
+        rep.meta_mismatch_groups += 1
+        S, Z = gpu_S, gpu_Z
+        codes = oracle.codes_given_meta(r, bits, S, Z)
+    diff = np.asarray(gpu_codes, dtype=np.int64) - codes.astype(np.int64)
+    bad = np.nonzero(diff)[0]
+    if bad.size:
+        q = oracle.quotients(r, S, Z)
+        frac = np.abs(q[bad] - np.floor(q[bad]) - 0.5)
+        if np.any(np.abs(diff[bad]) > 1) or np.any(frac > NEAR_TIE):
+            rep.failures.append(f"{where}: codes differ away from ties at {bad[:8].tolist()}")
+        rep.code_mismatches += int(bad.size)
+
+
+def check_pool_tokens(rep: QuantReport, gpu_pool: np.ndarray, num_blocks: int, hkv: int, k_rows, v_rows,
+                      in_dtype: int, slots, tokens, heads=None):
+    """Check (token, head) groups: k_rows/v_rows hold [n, Hkv, 128] raw input rows."""
+    g = oracle.geom(num_blocks=num_blocks, num_kv_heads=hkv)
+    heads = range(hkv) if heads is None else heads
+    for t in tokens:
+        s = int(slots[t])
+        if s < 0:
+            continue
+        p, o = divmod(s, 16)
+        for h in heads:
+            kc, Sk, Zk, vc, Sv, Zv = oracle.unpack_token(g, gpu_pool, p, o, h)
+            check_vector(rep, to_f64(k_rows[t, h], in_dtype), 4, kc, Sk, Zk, f"t{t} h{h} K")
+            check_vector(rep, to_f64(v_rows[t, h], in_dtype), 2, vc, Sv, Zv, f"t{t} h{h} V")

@@ -1,0 +1,109 @@
+"""The C-ABI library loads without a GPU, exports every symbol include/kvq.h
+declares, and its host-only entry points and argument checks behave as
+documented.  No kernel is launched here."""
+import ctypes
+
+import numpy as np
+import pytest
+
+
+def test_every_declared_symbol_is_exported(kvq):
+    names = kvq.header_functions()
+    assert "kvq_quantize_append" in names and "kvq_decode_attention" in names and "kvq_block_table" in names
+    raw = ctypes.CDLL(kvq.LIB_PATH)
+    missing = [n for n in names if not hasattr(raw, n)]
+    assert not missing, missing
+
+
+def test_parse_dtype(kvq):
+    assert kvq.kvq_parse_dtype("kvarn_k4v2_g128") == (0, (4, 2, 128))
+    rc, parsed = kvq.kvq_parse_dtype("kvarn_k4v4_g128")
+    assert rc == kvq.KVQ_ERR_UNSUPPORTED and parsed == (4, 4, 128)
+    for bad in ("fp8", "kvarn_k4v2_g128x", "kvarn_k4v2", "kvarn_kv2_g128", ""):
+        assert kvq.kvq_parse_dtype(bad)[0] == kvq.KVQ_ERR_INVALID
+
+
+def test_error_strings(kvq):
+    for code in range(0, -8, -1):
+        assert kvq.kvq_error_string(code)
+    assert kvq.kvq_error_string(-99) == "unknown status"
+
+
+def test_cache_bytes(kvq):
+    assert kvq.kvq_cache_bytes(kvq.make_desc(1024, 8)) == 1024 * 8 * 1664
+    d = kvq.make_desc(4, 2)
+    d.head_dim = 64
+    assert kvq.kvq_cache_bytes(d) == 0
+    # 104 bytes per token per kv head: 64 B of 4-bit keys, 32 B of 2-bit values, 4 fp16
+    assert 1664 / 16 == 104
+
+
+def test_block_table_identity_and_shuffle(kvq):
+    lens = [40, 0, 16, 17]
+    bt, used = kvq.kvq_block_table(10, lens, 4, shuffle_seed=0)
+    assert used == 3 + 0 + 1 + 2
+    assert bt.tolist() == [[0, 1, 2, -1], [-1] * 4, [3, -1, -1, -1], [4, 5, -1, -1]]
+    bt2, used2 = kvq.kvq_block_table(10, lens, 4, shuffle_seed=1234)
+    assert used2 == used
+    flat = bt2[bt2 >= 0]
+    assert len(set(flat.tolist())) == used and flat.min() >= 0 and flat.max() < 10
+    assert (bt2 >= 0).tolist() == (bt >= 0).tolist()
+    again, _ = kvq.kvq_block_table(10, lens, 4, shuffle_seed=1234)
+    assert np.array_equal(bt2, again)
+
+
+def test_block_table_errors(kvq):
+    with pytest.raises(kvq.KvqError) as e:
+        kvq.kvq_block_table(2, [40], 4)
+    assert e.value.status == kvq.KVQ_ERR_POOL_EXHAUSTED
+    with pytest.raises(kvq.KvqError) as e:
+        kvq.kvq_block_table(100, [80], 4)
+    assert e.value.status == kvq.KVQ_ERR_INVALID
+
+
+def test_slot_mapping(kvq):
+    bt = np.array([[7, 3, -1], [5, -1, -1]], dtype=np.int32)
+    slots = kvq.kvq_slot_mapping(bt, positions=[0, 15, 16, 31, 2, 16], seq_ids=[0, 0, 0, 0, 1, 1])
+    assert slots.tolist() == [112, 127, 48, 63, 82, -1]
+    with pytest.raises(kvq.KvqError):
+        kvq.kvq_slot_mapping(bt, positions=[48], seq_ids=[0])
+
+
+def test_argument_checks_need_no_device(kvq):
+    L = kvq.lib()
+    d = kvq.make_desc(4, 2)
+    # null pool / inputs
+    assert L.kvq_quantize_append(ctypes.byref(d), None, None, kvq.KVQ_BF16, 1, 256, None, None) == kvq.KVQ_ERR_INVALID
+    # zero tokens is a no-op even with null pointers
+    assert L.kvq_quantize_append(ctypes.byref(d), None, None, kvq.KVQ_BF16, 0, 256, None, None) == kvq.KVQ_OK
+    # fp32 cache input is not a supported write dtype
+    assert L.kvq_quantize_append(ctypes.byref(d), None, None, kvq.KVQ_F32, 1, 256, None, None) == kvq.KVQ_ERR_UNSUPPORTED
+    # misaligned pointers
+    d.pool = 0x1000
+    assert L.kvq_quantize_append(ctypes.byref(d), ctypes.c_void_p(0x1008), ctypes.c_void_p(0x2000), kvq.KVQ_BF16, 1,
+                                 256, ctypes.c_void_p(0x3000), None) == kvq.KVQ_ERR_INVALID
+    # token stride shorter than a row
+    assert L.kvq_quantize_append(ctypes.byref(d), ctypes.c_void_p(0x1000), ctypes.c_void_p(0x2000), kvq.KVQ_BF16, 1,
+                                 128, ctypes.c_void_p(0x3000), None) == kvq.KVQ_ERR_INVALID
+    # unsupported GQA group (24 / 8 = 3) and a non-multiple
+    args = (ctypes.c_void_p(0x1000), kvq.KVQ_BF16, 1)
+    assert L.kvq_decode_attention(ctypes.byref(d), *args, 6, None, 1, None, 16, 0.0, None, kvq.KVQ_F32, None, 0,
+                                  None) == kvq.KVQ_ERR_UNSUPPORTED
+    assert L.kvq_decode_attention(ctypes.byref(d), *args, 3, None, 1, None, 16, 0.0, None, kvq.KVQ_F32, None, 0,
+                                  None) == kvq.KVQ_ERR_UNSUPPORTED
+    # missing workspace
+    one = ctypes.c_void_p(0x4000)
+    assert L.kvq_decode_attention(ctypes.byref(d), *args, 2, one, 1, one, 16, 0.0, one, kvq.KVQ_F32, None, 0,
+                                  None) == kvq.KVQ_ERR_WORKSPACE
+    # bad head dim
+    d.head_dim = 64
+    assert L.kvq_decode_attention(ctypes.byref(d), *args, 2, one, 1, one, 16, 0.0, one, kvq.KVQ_F32, one, 1 << 20,
+                                  None) == kvq.KVQ_ERR_UNSUPPORTED
+
+
+def test_workspace_bytes(kvq):
+    n = kvq.kvq_decode_workspace_bytes(1024, 8, 1, 64, 16384)
+    assert n > 0 and n % 4 == 0
+    n1 = kvq.kvq_decode_workspace_bytes(1024, 8, 1, 64, 16384, blocks_per_split=1024)
+    assert n1 == 256 + 64 * 1 * 132 * 4
+    assert kvq.kvq_decode_workspace_bytes(1024, 8, 1, 60, 16384) == 0

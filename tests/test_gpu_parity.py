@@ -1,0 +1,325 @@
+"""GPU parity: the CUDA path through the C-ABI against the CPU oracle on the
+same seeded inputs.  Quantized codes must be bit-exact except at near-ties
+(tests/helpers.py); decode outputs must be within 2e-3 (max abs, fp32) of the
+oracle's double-precision attention read from the same codes, which here are
+always written by the oracle and uploaded (no oracle input comes from the
+CUDA path)."""
+import math
+
+import numpy as np
+import pytest
+
+import helpers
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dev_u16(arr, dtype):
+    torch = _torch()
+    t = torch.from_numpy(np.ascontiguousarray(arr).view(np.int16)).cuda()
+    return t.view(torch.float16 if dtype == synth.F16 else torch.bfloat16)
+
+
+def _oracle_pool(wl):
+    g = oracle.geom(num_blocks=wl.num_blocks, num_kv_heads=wl.hkv)
+    pool = oracle.new_pool(g)
+    k = wl.kv_rows(synth.TID_K, 0, wl.total_tokens)
+    v = wl.kv_rows(synth.TID_V, 0, wl.total_tokens)
+    assert oracle.quantize_append(g, pool, k, v, wl.dtype, wl.slots()) == 0
+    return g, pool, k, v
+
+
+def _gpu_decode(kvq, wl, pool_np, q_np, q_dtype, out_dtype="f32", bps=0, max_seq_len=None, seq_lens=None,
+                block_table=None):
+    torch = _torch()
+    pool = torch.from_numpy(pool_np).cuda()
+    if q_dtype == synth.F32:
+        q = torch.from_numpy(q_np.astype(np.float32)).cuda()
+    else:
+        q = _dev_u16(q_np, q_dtype)
+    lens = wl.seq_lens if seq_lens is None else np.asarray(seq_lens, np.int32)
+    bt = torch.from_numpy(wl.block_table if block_table is None else block_table).cuda()
+    sl = torch.from_numpy(lens).cuda()
+    msl = int(lens.max()) if max_seq_len is None else max_seq_len
+    out = torch.empty((wl.batch, wl.hq, 128), dtype={"f32": torch.float32, "bf16": torch.bfloat16,
+                                                      "f16": torch.float16}[out_dtype], device="cuda")
+    ws = kvq.new_workspace(wl.num_blocks, wl.hkv, wl.batch, wl.hq, msl, bps)
+    kvq.kvq_decode_attention(pool, wl.num_blocks, wl.hkv, q, bt, sl, msl, out, ws, blocks_per_split=bps)
+    torch.cuda.synchronize()
+    return out.float().cpu().numpy().astype(np.float64), ws
+
+
+# ------------------------------------------------------------------ write path
+
+def _run_quantize(kvq, wl, slots, k, v, pool_fill=0x5A):
+    torch = _torch()
+    pool = torch.full((kvq.kvq_cache_bytes(kvq.make_desc(wl.num_blocks, wl.hkv)),), pool_fill, dtype=torch.uint8,
+                      device="cuda")
+    kd = _dev_u16(k, wl.dtype).reshape(k.shape[0], -1)
+    vd = _dev_u16(v, wl.dtype).reshape(v.shape[0], -1)
+    sd = torch.from_numpy(np.ascontiguousarray(slots, np.int32)).cuda()
+    kvq.kvq_quantize_append(pool, wl.num_blocks, wl.hkv, kd, vd, sd)
+    assert kvq.kvq_last_device_status() == 0
+    return pool.cpu().numpy()
+
+
+@pytest.mark.parametrize("make", [lambda: synth.tiny(0),
+                                  lambda: synth.Workload("q", 3, 16, 8, 128, [70, 1, 33], 16, synth.BF16, 3, 10.0,
+                                                         30.0, seed=11)])
+def test_quantize_matches_oracle(kvq, cuda, make):
+    wl = make()
+    k = wl.kv_rows(synth.TID_K, 0, wl.total_tokens)
+    v = wl.kv_rows(synth.TID_V, 0, wl.total_tokens)
+    slots = wl.slots()
+    gpu = _run_quantize(kvq, wl, slots, k, v)
+    rep = helpers.QuantReport()
+    helpers.check_pool_tokens(rep, gpu, wl.num_blocks, wl.hkv, k, v, wl.dtype, slots, range(wl.total_tokens))
+    assert rep.ok(), rep
+    # bytes of the pool no token maps to are untouched
+    written = np.zeros((wl.num_blocks, wl.hkv, 16), bool)
+    for s in slots:
+        written[s // 16, :, s % 16] = True
+    seg = gpu.reshape(wl.num_blocks, wl.hkv, 1664)
+    for p in range(wl.num_blocks):
+        for o in range(16):
+            if not written[p, 0, o]:
+                assert np.all(seg[p, :, o * 64:(o + 1) * 64] == 0x5A)
+                assert np.all(seg[p, :, 1024 + o * 32:1024 + (o + 1) * 32] == 0x5A)
+
+
+def test_quantize_edge_inputs(kvq, cuda):
+    """Zero vectors, one-hot vectors (flat after rotation: S = 0), skipped
+    slots, a strided (non-dense) token layout and a lone token in a block."""
+    torch = _torch()
+    hkv, n = 2, 40
+    wl = synth.Workload("e", 1, 2, hkv, 128, [n], 16, synth.BF16, 3, 10.0, 30.0, seed=12, extra_blocks=2,
+                        shuffle=False)
+    k = wl.kv_rows(synth.TID_K, 0, n)
+    v = wl.kv_rows(synth.TID_V, 0, n)
+    k[0] = 0
+    v[1] = 0
+    k[2, :, :] = 0
+    k[2, :, 0] = np.array([2.5], np.float32).view(np.uint32)[0] >> 16  # bf16 bits of 2.5
+    slots = wl.slots().copy()
+    slots[5] = -1
+    slots[7] = wl.num_blocks * 16 - 1  # last slot of the pool
+    # strided rows: each token row padded to 3*128 elements
+    stride = 3 * 128
+    kp = np.zeros((n, stride), np.uint16)
+    vp = np.zeros((n, stride), np.uint16)
+    kp[:, :hkv * 128] = k.reshape(n, -1)
+    vp[:, :hkv * 128] = v.reshape(n, -1)
+    pool = torch.full((wl.num_blocks * hkv * 1664,), 0x33, dtype=torch.uint8, device="cuda")
+    kvq.kvq_quantize_append(pool, wl.num_blocks, hkv, _dev_u16(kp, wl.dtype), _dev_u16(vp, wl.dtype),
+                            torch.from_numpy(slots).cuda())
+    assert kvq.kvq_last_device_status() == 0
+    gpu = pool.cpu().numpy()
+    rep = helpers.QuantReport()
+    helpers.check_pool_tokens(rep, gpu, wl.num_blocks, hkv, k, v, wl.dtype, slots, range(n))
+    assert rep.ok(), rep
+    g = oracle.geom(num_blocks=wl.num_blocks, num_kv_heads=hkv)
+    kc, Sk, Zk, *_ = oracle.unpack_token(g, gpu, slots[0] // 16, slots[0] % 16, 0)
+    assert Sk == 0 and Zk == 0 and not kc.any()
+    kc, Sk, Zk, *_ = oracle.unpack_token(g, gpu, slots[2] // 16, slots[2] % 16, 0)
+    assert Sk == 0 and not kc.any()
+    s5 = wl.slots()[5]
+    seg = gpu.reshape(wl.num_blocks, hkv, 1664)
+    assert np.all(seg[s5 // 16, :, (s5 % 16) * 64:(s5 % 16 + 1) * 64] == 0x33)
+
+
+def test_quantize_reports_slot_outside_pool(kvq, cuda):
+    torch = _torch()
+    wl = synth.Workload("e", 1, 1, 1, 128, [3], 16, synth.F16, 0, 1.0, 1.0, seed=13)
+    k = wl.kv_rows(synth.TID_K, 0, 3)
+    pool = torch.zeros(wl.num_blocks * 1664, dtype=torch.uint8, device="cuda")
+    slots = torch.tensor([0, 16 * wl.num_blocks + 3, 1], dtype=torch.int32, device="cuda")
+    kvq.kvq_quantize_append(pool, wl.num_blocks, 1, _dev_u16(k, wl.dtype).reshape(3, -1),
+                            _dev_u16(k, wl.dtype).reshape(3, -1), slots)
+    assert kvq.kvq_last_device_status() == kvq.KVQ_ERR_OUT_OF_RANGE
+    assert kvq.kvq_last_device_status() == 0  # read-and-clear
+
+
+# ------------------------------------------------------------------ read path
+
+def _check_decode(wl, g, pool, q, q_dtype, got, rel=0.0):
+    """max |got - want| <= 2e-3 (+ rel*|want| for a bf16/fp16 output)."""
+    want = oracle.decode_attention(g, pool, q, q_dtype, wl.block_table, wl.seq_lens, nthreads=8)
+    assert np.all(np.isfinite(got))
+    excess = np.abs(got - want) - (helpers.ATTN_TOL + rel * np.abs(want))
+    assert excess.max() <= 0, (np.max(np.abs(got - want)), excess.max())
+    return float(np.max(np.abs(got - want)))
+
+
+def test_decode_tiny(kvq, cuda):
+    wl = synth.tiny(0)
+    g, pool, _, _ = _oracle_pool(wl)
+    q = wl.query()
+    got, _ = _gpu_decode(kvq, wl, pool, q, wl.dtype)
+    _check_decode(wl, g, pool, q, wl.dtype, got)
+
+
+@pytest.mark.parametrize("bps", [0, 1, 3, 1000])
+def test_decode_ragged_gqa8(kvq, cuda, bps):
+    wl = synth.Workload("r", 6, 16, 2, 128, [1, 15, 16, 17, 100, 0], 16, synth.BF16, 3, 10.0, 30.0, seed=21,
+                        extra_blocks=3)
+    g, pool, _, _ = _oracle_pool(wl)
+    q = wl.query()
+    got, _ = _gpu_decode(kvq, wl, pool, q, wl.dtype, bps=bps)
+    _check_decode(wl, g, pool, q, wl.dtype, got)
+    assert not got[5].any()  # length 0 -> zeros
+
+
+@pytest.mark.parametrize("G", [1, 2, 4])
+def test_decode_group_sizes(kvq, cuda, G):
+    wl = synth.Workload("g", 2, 4 * G, 4, 128, [129, 47], 16, synth.F16, 4, 20.0, 20.0, seed=30 + G)
+    g, pool, _, _ = _oracle_pool(wl)
+    q = wl.query()
+    got, _ = _gpu_decode(kvq, wl, pool, q, wl.dtype)
+    _check_decode(wl, g, pool, q, wl.dtype, got)
+
+
+@pytest.mark.parametrize("q_dtype,out_dtype,rel", [(synth.F32, "f32", 0.0), (synth.F16, "bf16", 2.0 ** -8),
+                                                   (synth.BF16, "f16", 2.0 ** -11)])
+def test_decode_dtypes(kvq, cuda, q_dtype, out_dtype, rel):
+    wl = synth.Workload("d", 2, 16, 2, 128, [90, 200], 16, synth.BF16, 3, 10.0, 30.0, seed=40)
+    g, pool, _, _ = _oracle_pool(wl)
+    q = synth.normal(wl.seed, synth.TID_Q, wl.batch * wl.hq * 128, q_dtype).reshape(wl.batch, wl.hq, 128)
+    got, _ = _gpu_decode(kvq, wl, pool, q, q_dtype, out_dtype=out_dtype)
+    # bf16/f16 outputs carry their own rounding on top of the 2e-3 kernel bound
+    _check_decode(wl, g, pool, q, q_dtype, got, rel=rel)
+
+
+def test_decode_workspace_is_reusable(kvq, cuda):
+    """Tickets reset themselves: the same workspace serves repeated calls."""
+    torch = _torch()
+    wl = synth.Workload("w", 2, 16, 2, 128, [300, 77], 16, synth.BF16, 3, 10.0, 30.0, seed=50)
+    g, pool, _, _ = _oracle_pool(wl)
+    q = wl.query()
+    got1, ws = _gpu_decode(kvq, wl, pool, q, wl.dtype, bps=2)
+    tickets = ws[:256].view(torch.int32)[: wl.batch * wl.hkv]
+    assert not tickets.any()
+    dpool = torch.from_numpy(pool).cuda()
+    out = torch.empty((wl.batch, wl.hq, 128), dtype=torch.float32, device="cuda")
+    for _ in range(3):
+        kvq.kvq_decode_attention(dpool, wl.num_blocks, wl.hkv, _dev_u16(q, wl.dtype),
+                                 torch.from_numpy(wl.block_table).cuda(), torch.from_numpy(wl.seq_lens).cuda(),
+                                 int(wl.seq_lens.max()), out, ws, blocks_per_split=2)
+    torch.cuda.synchronize()
+    assert np.array_equal(out.cpu().numpy().astype(np.float64), got1)
+
+
+def test_decode_reports_bad_block_id(kvq, cuda):
+    wl = synth.Workload("b", 1, 8, 1, 128, [64], 16, synth.BF16, 3, 10.0, 30.0, seed=60, extra_blocks=1)
+    g, pool, _, _ = _oracle_pool(wl)
+    q = wl.query()
+    bt = wl.block_table.copy()
+    bt[0, 2] = wl.num_blocks + 5
+    got, _ = _gpu_decode(kvq, wl, pool, q, wl.dtype, block_table=bt)
+    assert kvq.kvq_last_device_status() == kvq.KVQ_ERR_OUT_OF_RANGE
+    assert np.all(np.isfinite(got))
+    # the bad block's tokens are skipped: the oracle over the other three blocks agrees
+    keep = [0, 1, 3]
+    bt3 = np.full((1, 3), -1, np.int32)
+    bt3[0] = wl.block_table[0, keep]
+    pool2 = pool.copy()
+    want = oracle.decode_attention(g, pool2, q, wl.dtype, bt3, np.array([48], np.int32))
+    assert np.max(np.abs(got - want)) <= helpers.ATTN_TOL
+
+
+def test_end_to_end_against_unquantized(kvq, cuda):
+    """GPU write then GPU read against oracle write then oracle read; also
+    reports (does not gate) the error of the quantised cache against fp16
+    attention on the raw inputs."""
+    torch = _torch()
+    wl = synth.Workload("x", 2, 16, 2, 128, [256, 93], 16, synth.BF16, 3, 10.0, 30.0, seed=70)
+    g, opool, k, v = _oracle_pool(wl)
+    gpool = _run_quantize(kvq, wl, wl.slots(), k, v)
+    q = wl.query()
+    got, _ = _gpu_decode(kvq, wl, gpool, q, wl.dtype)
+    want = oracle.decode_attention(g, opool, q, wl.dtype, wl.block_table, wl.seq_lens)
+    assert np.max(np.abs(got - want)) <= helpers.ATTN_TOL
+    dense_err = 0.0
+    for b in range(wl.batch):
+        L = int(wl.seq_lens[b])
+        off = int(wl.token_offsets[b])
+        for j in range(wl.hq):
+            ref = oracle.attention_dense(k[off:off + L], v[off:off + L], wl.dtype, q[b, j], wl.dtype, wl.hq, j)
+            dense_err = max(dense_err, float(np.max(np.abs(got[b, j] - ref))))
+    print(f"\nk4v2_g128 decode vs unquantized attention: max abs err {dense_err:.4f}")
+    assert math.isfinite(dense_err)
+
+
+# ------------------------------------------------------------------ full sizes
+
+def _full_size_decode(kvq, wl, sample_heads, sample_batches):
+    """Pool written by the GPU for every head, then the sampled kv heads'
+    segments replaced by oracle-written bytes; GPU decode in the default
+    (benchmarked) launch configuration; sampled outputs against the oracle."""
+    torch = _torch()
+    T = wl.total_tokens
+    k = wl.kv_rows(synth.TID_K, 0, T)
+    v = wl.kv_rows(synth.TID_V, 0, T)
+    slots = wl.slots()
+    pool = torch.zeros(wl.num_blocks * wl.hkv * 1664, dtype=torch.uint8, device="cuda")
+    kvq.kvq_quantize_append(pool, wl.num_blocks, wl.hkv, _dev_u16(k, wl.dtype).reshape(T, -1),
+                            _dev_u16(v, wl.dtype).reshape(T, -1), torch.from_numpy(slots).cuda())
+    assert kvq.kvq_last_device_status() == 0
+    # sampled write-path parity on the GPU-written pool
+    rng = np.random.default_rng(wl.seed)
+    host = pool.cpu().numpy()
+    rep = helpers.QuantReport()
+    helpers.check_pool_tokens(rep, host, wl.num_blocks, wl.hkv, k, v, wl.dtype, slots,
+                              rng.choice(T, 48, replace=False))
+    assert rep.ok(), rep
+    G = wl.hq // wl.hkv
+    q = wl.query()
+    seg = pool.view(wl.num_blocks, wl.hkv, 1664)
+    g1 = oracle.geom(num_blocks=wl.num_blocks, num_kv_heads=1)
+    opools = {}
+    for h in sample_heads:
+        op = oracle.new_pool(g1)
+        sel = np.zeros(T, bool)
+        for b in sample_batches:
+            off = int(wl.token_offsets[b])
+            sel[off:off + int(wl.seq_lens[b])] = True
+        idx = np.nonzero(sel)[0]
+        assert oracle.quantize_append(g1, op, np.ascontiguousarray(k[idx, h:h + 1]),
+                                      np.ascontiguousarray(v[idx, h:h + 1]), wl.dtype, slots[idx]) == 0
+        opools[h] = op
+        opv = torch.from_numpy(op.reshape(wl.num_blocks, 1664)).cuda()
+        used = torch.from_numpy(np.unique(slots[idx] // 16)).cuda().long()
+        seg[used, h] = opv[used]
+    msl = int(wl.seq_lens.max())
+    out = torch.empty((wl.batch, wl.hq, 128), dtype=torch.float32, device="cuda")
+    ws = kvq.new_workspace(wl.num_blocks, wl.hkv, wl.batch, wl.hq, msl)
+    kvq.kvq_decode_attention(pool, wl.num_blocks, wl.hkv, _dev_u16(q, wl.dtype), torch.from_numpy(wl.block_table)
+                             .cuda(), torch.from_numpy(wl.seq_lens).cuda(), msl, out, ws)
+    got = out.cpu().numpy().astype(np.float64)
+    assert kvq.kvq_last_device_status() == 0
+    worst = 0.0
+    for h in sample_heads:
+        for b in sample_batches:
+            qh = np.ascontiguousarray(q[b:b + 1, h * G:(h + 1) * G])
+            want = oracle.decode_attention(g1, opools[h], qh, wl.dtype, wl.block_table[b:b + 1],
+                                           wl.seq_lens[b:b + 1], nthreads=1)
+            worst = max(worst, float(np.max(np.abs(got[b, h * G:(h + 1) * G] - want[0]))))
+    print(f"\n{wl.name}: sampled decode max abs err {worst:.2e}")
+    assert worst <= helpers.ATTN_TOL
+    return worst
+
+
+def test_full_size_qwen3_32b_layer(kvq, cuda):
+    _full_size_decode(kvq, synth.qwen3_32b_layer(0), sample_heads=[0, 5], sample_batches=[0])
+
+
+def test_full_size_batched_ragged(kvq, cuda):
+    wl = synth.batched(0)
+    _full_size_decode(kvq, wl, sample_heads=[3], sample_batches=[int(np.argmax(wl.seq_lens)),
+                                                                int(np.argmin(wl.seq_lens))])
