@@ -1,0 +1,439 @@
+"""Benchmark of the quantized paged KV cache on B200.
+
+One step = one decode token through the attention cache of every layer of a
+Qwen3-32B-shaped model at 16K context: for each of 64 layers, the new
+token's K/V (8 kv heads x 128, bf16) is quantize-appended into that layer's
+packed k4v2_g128 pool, then decode attention runs for 64 query heads over the
+16384 cached tokens.  The 64 layers' pools (13.6 MB each, 872 MB together)
+are separate buffers, so every step reads the whole cache from HBM (inputs
+larger than L2, no flush needed).  A step is captured once in a CUDA graph and
+replayed.
+
+Printed (rank 0, one JSON line): decode tokens/s of the whole job; the decode
+kernel's effective HBM GB/s on packed-cache bytes against the measured copy
+bandwidth; quantize GB/s of a 16 x 16384-token prefill append; an end-to-end
+figure with pinned host copies inside the timed region; and the CPU oracle's
+throughput on a bounded sample.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kvq|reference]
+                    [--workload qwen3-32b-16k|batched|long|mixed]
+
+For N > 1 (torchrun), every rank runs an independent replica (the path has
+no cross-GPU step); the timing is the max over ranks and the value sums all
+ranks' tokens.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "decode attention tokens/s and effective HBM GB/s (% of roofline), quantize GB/s"
+SEG = 1664
+BYTES_PER_TOKEN_HEAD = 104
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# --------------------------------------------------------------------------- ranks
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, backend):
+    if world <= 1:
+        return None
+    import datetime
+    import torch.distributed as dist
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def aggregate(dist, local_ms: float, local_units: float, device=None):
+    """Max of the elapsed time and sum of the work over ranks."""
+    if dist is None:
+        return local_ms, local_units
+    import torch
+    t = torch.tensor([local_ms], dtype=torch.float64, device=device)
+    u = torch.tensor([local_units], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t[0]), float(u[0])
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.index), "-lms", "200"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 8:
+                    rows.append(parts)
+        if not rows:
+            return None
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(rows[0][1]) if rows[0][1].replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------- the step
+
+class QwenStep:
+    """64 layers of a Qwen3-32B-shaped attention cache at 16K context, batch 1."""
+
+    layers = 64
+    batch = 1
+    hq = 64
+    hkv = 8
+    context = 16384
+
+    def __init__(self, kvq, torch, dev, seed=0):
+        self.kvq, self.torch, self.dev = kvq, torch, dev
+        wl = synth.qwen3_32b_layer(seed, self.context)
+        self.wl = wl
+        self.nblocks = wl.num_blocks
+        T = wl.total_tokens
+        slots = wl.slots()
+        # layer 0's cache from the seeded workload; the other layers get copies
+        # of its bytes in their own buffers (identical work, distinct addresses)
+        k = torch.from_numpy(wl.kv_rows(synth.TID_K, 0, T).view(np.int16)).to(dev).view(torch.bfloat16)
+        v = torch.from_numpy(wl.kv_rows(synth.TID_V, 0, T).view(np.int16)).to(dev).view(torch.bfloat16)
+        pool0 = kvq.new_pool(self.nblocks, self.hkv, device=dev)
+        kvq.kvq_quantize_append(pool0, self.nblocks, self.hkv, k.reshape(T, -1), v.reshape(T, -1),
+                                torch.from_numpy(slots).to(dev))
+        torch.cuda.synchronize()
+        del k, v
+        self.pools = [pool0] + [pool0.clone() for _ in range(self.layers - 1)]
+        self.bt = torch.from_numpy(wl.block_table).to(dev)
+        self.lens = torch.from_numpy(wl.seq_lens).to(dev)
+        self.slot_new = torch.from_numpy(slots[-1:].copy()).to(dev)  # position 16383
+        # per-layer new token K/V and query (bf16), and outputs
+        nk = synth.kv(seed, synth.TID_NEWK, 0, self.layers, self.hkv, 128, 3, 10.0, 30.0, synth.BF16)
+        nv = synth.kv(seed, synth.TID_NEWV, 0, self.layers, self.hkv, 128, 3, 10.0, 30.0, synth.BF16)
+        qq = synth.normal(seed, synth.TID_Q, self.layers * self.hq * 128, synth.BF16)
+        self.h_in = torch.empty(self.layers * (2 * self.hkv + self.hq) * 128, dtype=torch.bfloat16).pin_memory()
+        hv = self.h_in.view(torch.int16).numpy()
+        n_kv = self.layers * self.hkv * 128
+        hv[:n_kv] = nk.reshape(-1).view(np.int16)
+        hv[n_kv:2 * n_kv] = nv.reshape(-1).view(np.int16)
+        hv[2 * n_kv:] = qq.view(np.int16)
+        self.d_in = self.h_in.to(dev)
+        self.new_k = self.d_in[:n_kv].view(self.layers, 1, self.hkv * 128)
+        self.new_v = self.d_in[n_kv:2 * n_kv].view(self.layers, 1, self.hkv * 128)
+        self.q = self.d_in[2 * n_kv:].view(self.layers, self.batch, self.hq, 128)
+        self.out = torch.empty((self.layers, self.batch, self.hq, 128), dtype=torch.bfloat16, device=dev)
+        self.h_out = torch.empty(self.out.shape, dtype=torch.bfloat16).pin_memory()
+        self.ws = kvq.new_workspace(self.nblocks, self.hkv, self.batch, self.hq, self.context, device=dev)
+
+    @property
+    def packed_bytes_per_decode(self):
+        return self.context * self.hkv * BYTES_PER_TOKEN_HEAD
+
+    def launches_per_step(self):
+        return 2 * self.layers
+
+    def step(self, decode_only=False):
+        kvq = self.kvq
+        for l in range(self.layers):
+            if not decode_only:
+                kvq.kvq_quantize_append(self.pools[l], self.nblocks, self.hkv, self.new_k[l], self.new_v[l],
+                                        self.slot_new)
+            kvq.kvq_decode_attention(self.pools[l], self.nblocks, self.hkv, self.q[l], self.bt, self.lens,
+                                     self.context, self.out[l], self.ws)
+
+    def tokens_per_step(self):
+        return self.batch
+
+
+def graph_of(torch, fn):
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()  # warm (attribute caches, first-launch setup) outside capture
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def time_replays(torch, g, n, barrier=None, pre=None, post=None):
+    """Device time (ms) of n replays of g, events on the replay stream."""
+    if barrier:
+        barrier()
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(n):
+        if pre:
+            pre()
+        g.replay()
+        if post:
+            post()
+    e1.record(s)
+    torch.cuda.synchronize()
+    if barrier:
+        barrier()
+    return e0.elapsed_time(e1)
+
+
+def prefill_quantize_gbs(kvq, torch, dev, seed=0, seqs=16, tokens=16384, reps=10):
+    """Quantize-append of 16 x 16384 fresh tokens, 8 kv heads, bf16."""
+    hkv = 8
+    T = seqs * tokens
+    nblocks = T // 16
+    # inputs: one seeded sequence's worth, repeated (the kernel's work does not
+    # depend on the values); slots: a seeded permutation of the pool
+    base = synth.kv(seed, synth.TID_K, 0, tokens, hkv, 128, 3, 10.0, 30.0, synth.BF16)
+    kb = torch.from_numpy(base.view(np.int16)).to(dev).view(torch.bfloat16).reshape(tokens, -1)
+    k = kb.repeat(seqs, 1)
+    v = torch.roll(k, 1, 0).contiguous()
+    perm = synth.permutation(seed, synth.TID_PERM, nblocks).astype(np.int64)
+    slots = (perm[np.arange(T) // 16] * 16 + np.arange(T) % 16).astype(np.int32)
+    sl = torch.from_numpy(slots).to(dev)
+    pool = kvq.new_pool(nblocks, hkv, device=dev)
+    kvq.kvq_quantize_append(pool, nblocks, hkv, k, v, sl)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        kvq.kvq_quantize_append(pool, nblocks, hkv, k, v, sl)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    nbytes = T * hkv * (2 * 128 * 2 + BYTES_PER_TOKEN_HEAD) + T * 4
+    status = kvq.kvq_last_device_status()
+    del k, v, pool, kb
+    return {"us": ms * 1e3, "gbs": nbytes / (ms * 1e-3) / 1e9, "bytes": nbytes, "status": status}
+
+
+# --------------------------------------------------------------------------- CPU oracle
+
+class OracleSample:
+    """The oracle, as it stands, on a bounded sample of one step: the 1-token
+    write plus the decode of one kv head (8 query heads over 16384 tokens) of
+    one layer.  A step is 64 layers x 8 kv heads of such units.  The cache
+    state it reads is written by the oracle itself, once, untimed."""
+
+    desc = ("oracle 1-token write + decode of 1 kv head (8 query heads x 16384 tokens) of 1 layer, single "
+            "thread; one step = 64 layers x 8 kv heads of these units")
+
+    def __init__(self, seed=0):
+        import oracle
+        self.oracle = oracle
+        wl = synth.qwen3_32b_layer(seed, QwenStep.context)
+        T = wl.total_tokens
+        self.wl = wl
+        self.k = np.ascontiguousarray(wl.kv_rows(synth.TID_K, 0, T)[:, :1])
+        self.v = np.ascontiguousarray(wl.kv_rows(synth.TID_V, 0, T)[:, :1])
+        self.g = oracle.geom(num_blocks=wl.num_blocks, num_kv_heads=1)
+        self.pool = oracle.new_pool(self.g)
+        self.slots = wl.slots()
+        assert oracle.quantize_append(self.g, self.pool, self.k, self.v, wl.dtype, self.slots) == 0
+        self.q = np.ascontiguousarray(wl.query()[:, :8])
+
+    def unit(self) -> float:
+        o, wl = self.oracle, self.wl
+        t0 = time.perf_counter()
+        assert o.quantize_append(self.g, self.pool, self.k[-1:], self.v[-1:], wl.dtype, self.slots[-1:]) == 0
+        o.decode_attention(self.g, self.pool, self.q, wl.dtype, wl.block_table, wl.seq_lens, nthreads=1)
+        return time.perf_counter() - t0
+
+
+# --------------------------------------------------------------------------- main
+
+def run_reference(args, world, rank):
+    """The reference arm: the CPU oracle timed on the machine's host cores."""
+    if rank != 0:
+        return 0
+    units_per_step = QwenStep.layers * QwenStep.hkv
+    sample = OracleSample()
+    for _ in range(args.warmup):
+        sample.unit()
+    samples = [sample.unit() for _ in range(args.steps)]
+    per_unit = sum(samples) / len(samples)
+    desc = sample.desc + f"; each timed step runs one unit, {args.steps} steps"
+    step_s = per_unit * units_per_step
+    value = QwenStep.batch / step_s
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "qwen3-32b-16k-64layers", "batch": 1, "num_q_heads": 64, "num_kv_heads": 8,
+                       "head_dim": 128, "context": 16384, "layers": 64, "block_size": 16},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+
+    import torch
+    import bit_kv_cache_18_b200 as kvq
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    dist = init_dist(world, "nccl")
+    barrier = (lambda: dist.barrier(device_ids=[local])) if dist else None
+
+    stepper = QwenStep(kvq, torch, dev)
+    g_step = graph_of(torch, stepper.step)
+    g_dec = graph_of(torch, lambda: stepper.step(decode_only=True))
+    for _ in range(args.warmup):
+        g_step.replay()
+    torch.cuda.synchronize()
+    if kvq.kvq_last_device_status() != 0:
+        raise RuntimeError("device status set during warm-up")
+
+    # timed region: K steps
+    with ClockSampler(local) as clocks:
+        ms = time_replays(torch, g_step, args.steps, barrier)
+    ms_max, tokens = aggregate(dist, ms, args.steps * stepper.tokens_per_step(), dev)
+    value = tokens / (ms_max * 1e-3)
+    ms_per_step = ms_max / args.steps
+
+    # decode kernel alone (roofline): the same 64 launches without the appends
+    for _ in range(3):
+        g_dec.replay()
+    dec_reps = max(args.steps, 10)
+    dms = time_replays(torch, g_dec, dec_reps) / (dec_reps * stepper.layers)
+    achieved = stepper.packed_bytes_per_decode / (dms * 1e-3) / 1e9
+    peak, peak_kind = measured_peaks()
+
+    # end to end: pinned host inputs in, outputs back, every step
+    def h2d():
+        stepper.d_in.copy_(stepper.h_in, non_blocking=True)
+
+    def d2h():
+        stepper.h_out.copy_(stepper.out, non_blocking=True)
+
+    e2e_ms = time_replays(torch, g_step, args.steps, barrier, pre=h2d, post=d2h)
+    e2e_ms_max, e2e_tokens = aggregate(dist, e2e_ms, args.steps * stepper.tokens_per_step(), dev)
+
+    quant = prefill_quantize_gbs(kvq, torch, dev)
+    status = kvq.kvq_last_device_status()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        sample = OracleSample()
+        per_unit = sum(sample.unit() for _ in range(3)) / 3
+        cpu_value = 1.0 / (per_unit * stepper.layers * stepper.hkv)
+        cpu = {"value": cpu_value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+               "sample": sample.desc + "; mean of 3 units"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": "qwen3-32b-16k-64layers", "batch": 1, "num_q_heads": 64, "num_kv_heads": 8,
+                       "head_dim": 128, "context": 16384, "layers": 64, "block_size": 16,
+                       "cache": "kvarn_k4v2_g128", "step": "per layer: 1-token quantize-append + decode attention",
+                       "l2": "inputs larger than L2: 64 distinct 13.6 MB pools (872 MB) per step",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "kernel": "decode", "peak_kind": peak_kind,
+                         "us_per_launch": dms * 1e3, "bytes_per_launch": stepper.packed_bytes_per_decode,
+                         "frac_of_8000": achieved / 8000.0},
+            "decode": {"us_per_layer": dms * 1e3, "effective_gbs": achieved,
+                       "layer_tokens_per_s": stepper.batch / (dms * 1e-3),
+                       "context_tokens_per_s": stepper.context * stepper.batch / (dms * 1e-3)},
+            "quantize": {"workload": "prefill append 16 x 16384 tokens, 8 kv heads, bf16", "us": quant["us"],
+                         "gbs": quant["gbs"], "bytes": quant["bytes"], "frac": quant["gbs"] / peak},
+            "e2e": {"value": e2e_tokens / (e2e_ms_max * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": stepper.h_in.numel() * 2, "d2h_bytes_per_step": stepper.h_out.numel() * 2},
+            "gpu_launches": stepper.launches_per_step() * args.steps,
+            "clocks": clocks.summary(),
+            "device_status": status,
+        }
+        if cpu:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line))
+    if dist:
+        del g_step, g_dec
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -70,26 +70,41 @@ int device_sm_count() {
   return n;
 }
 
-// Split-K plan.  The context of every sequence is cut into splits of
-// blocks_per_split blocks; one CTA owns one (sequence, kv head, split).  By
-// default the split is sized so that batch*Hkv*nsplit fills every SM twice
-// (two resident CTAs per SM), capped at 64 blocks (1024 tokens) so long
-// contexts get many even waves.
+// Split-K plan.  The context of every sequence is cut into nsplit splits of
+// blocks_per_split blocks; one CTA owns one (sequence, kv head, split).  The
+// default picks nsplit (at most decode_max_splits()) by a small cost model:
+// CTAs run in waves of (SMs x resident CTAs per SM), a CTA costs its blocks
+// plus a fixed prologue worth about 4 blocks, and every extra split adds
+// about half a block of merge work.  A requested blocks_per_split is raised
+// if it would need more splits than the cap.
 int plan_decode(int32_t batch, int32_t num_kv_heads, int32_t num_q_heads, int32_t max_seq_len,
                 int32_t bps_request, DecodePlan* plan) {
   if (batch < 0 || num_kv_heads <= 0 || num_q_heads <= 0 || max_seq_len < 0 || bps_request < 0)
     return KVQ_ERR_INVALID;
   const int64_t nb = (static_cast<int64_t>(max_seq_len) + kBlockSize - 1) / kBlockSize;
+  const int64_t cap = decode_max_splits();
   int64_t bps = bps_request;
-  if (bps == 0) {
+  if (nb == 0) {
+    bps = 1;
+  } else if (bps == 0) {
     const int64_t units = static_cast<int64_t>(batch) * num_kv_heads;
-    const int64_t target = 2ll * device_sm_count();
-    bps = units > 0 ? (units * nb + target - 1) / target : 1;
-    if (bps > 64) bps = 64;
-    if (bps < 1) bps = 1;
+    const int64_t slots = static_cast<int64_t>(device_sm_count()) * decode_ctas_per_sm();
+    double best = 1e300;
+    bps = nb;
+    for (int64_t n = 1; n <= cap && n <= nb; ++n) {
+      const int64_t b = (nb + n - 1) / n;
+      if ((nb + b - 1) / b != n) continue;
+      const int64_t waves = (units * n + slots - 1) / slots;
+      const double cost = static_cast<double>(waves) * (b + 4) + 0.5 * n;
+      if (cost < best) {
+        best = cost;
+        bps = b;
+      }
+    }
+  } else if ((nb + bps - 1) / bps > cap) {
+    bps = (nb + cap - 1) / cap;
   }
-  int64_t nsplit = nb > 0 ? (nb + bps - 1) / bps : 1;
-  if (nsplit > 65535) return KVQ_ERR_UNSUPPORTED;
+  const int64_t nsplit = nb > 0 ? (nb + bps - 1) / bps : 1;
   plan->blocks_per_split = static_cast<int32_t>(bps);
   plan->nsplit = static_cast<int32_t>(nsplit);
   plan->ticket_bytes = ((static_cast<size_t>(batch) * num_kv_heads * sizeof(int32_t)) + 255) / 256 * 256;

@@ -112,5 +112,22 @@ int plan_decode(int32_t batch, int32_t num_kv_heads, int32_t num_q_heads, int32_
                 int32_t blocks_per_split_request, DecodePlan* plan);
 
 int device_sm_count();
+int decode_ctas_per_sm();  // resident decode CTAs per SM on the current device
+int decode_max_splits();   // upper bound the split plan respects
+
+// Raise a kernel's dynamic shared-memory limit once per device (a host call
+// that is not a stream operation, so it is also safe while a stream is being
+// captured into a graph).
+template <auto kKernel>
+cudaError_t ensure_smem_limit(int bytes) {
+  static bool done[64] = {};  // one flag array per kernel (template argument)
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
+  e = cudaFuncSetAttribute(kKernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = true;
+  return e;
+}
 
 }  // namespace kvq

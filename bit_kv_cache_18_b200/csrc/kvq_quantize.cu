@@ -372,25 +372,20 @@ cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream) {
   const int64_t n_vec = static_cast<int64_t>(a.n_tokens) * a.num_kv_heads;
   const int64_t tiles = 2 * ((n_vec + kRows - 1) / kRows);
   const int smem = kWarps * 2 * kTileBytes;
-  static bool attr_set[2] = {false, false};
   const int sms = device_sm_count();
   int64_t grid = (tiles + kWarps - 1) / kWarps;
   const int64_t cap = static_cast<int64_t>(sms) * 3;
   if (grid > cap) grid = cap;
   const int64_t stride_bytes = a.token_stride * 2;
   if (a.in_dtype == KVQ_BF16) {
-    if (!attr_set[1]) {
-      cudaFuncSetAttribute(quantize_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      attr_set[1] = true;
-    }
+    const cudaError_t e = ensure_smem_limit<quantize_kernel<true>>(smem);
+    if (e != cudaSuccess) return e;
     quantize_kernel<true><<<static_cast<unsigned>(grid), kWarps * 32, smem, stream>>>(
         a.pool, a.num_blocks, a.num_kv_heads, static_cast<const uint8_t*>(a.k),
         static_cast<const uint8_t*>(a.v), a.n_tokens, stride_bytes, a.slots, a.status);
   } else {
-    if (!attr_set[0]) {
-      cudaFuncSetAttribute(quantize_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      attr_set[0] = true;
-    }
+    const cudaError_t e = ensure_smem_limit<quantize_kernel<false>>(smem);
+    if (e != cudaSuccess) return e;
     quantize_kernel<false><<<static_cast<unsigned>(grid), kWarps * 32, smem, stream>>>(
         a.pool, a.num_blocks, a.num_kv_heads, static_cast<const uint8_t*>(a.k),
         static_cast<const uint8_t*>(a.v), a.n_tokens, stride_bytes, a.slots, a.status);

@@ -323,3 +323,18 @@ def test_full_size_batched_ragged(kvq, cuda):
     wl = synth.batched(0)
     _full_size_decode(kvq, wl, sample_heads=[3], sample_batches=[int(np.argmax(wl.seq_lens)),
                                                                 int(np.argmin(wl.seq_lens))])
+
+
+def test_decode_ignores_garbage_in_unused_slots(kvq, cuda):
+    """Rows past the end of a sequence hold whatever the pool held before
+    (here 0xFF bytes: NaN scales and zero points); they must not leak in."""
+    wl = synth.Workload("n", 3, 16, 2, 128, [17, 5, 250], 16, synth.BF16, 3, 10.0, 30.0, seed=80, extra_blocks=2)
+    g = oracle.geom(num_blocks=wl.num_blocks, num_kv_heads=wl.hkv)
+    pool = oracle.new_pool(g, fill=0xFF)
+    k = wl.kv_rows(synth.TID_K, 0, wl.total_tokens)
+    v = wl.kv_rows(synth.TID_V, 0, wl.total_tokens)
+    assert oracle.quantize_append(g, pool, k, v, wl.dtype, wl.slots()) == 0
+    q = wl.query()
+    for bps in (0, 1):
+        got, _ = _gpu_decode(kvq, wl, pool, q, wl.dtype, bps=bps)
+        _check_decode(wl, g, pool, q, wl.dtype, got)
