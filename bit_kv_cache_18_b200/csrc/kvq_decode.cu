@@ -46,42 +46,84 @@
 namespace kvq {
 namespace {
 
-constexpr int kStages = 8;          // segments in flight per warp
+#ifndef KVQ_DECODE_WARPS
+#define KVQ_DECODE_WARPS 8
+#endif
+constexpr int kDecodeWarps = KVQ_DECODE_WARPS;          // warps per CTA
+constexpr int kStages = kDecodeWarps == 8 ? 6 : 8;      // segments in flight per warp
+constexpr int kMinCtasPerSm = kDecodeWarps == 8 ? 2 : 3;
+constexpr float kRescaleLog2 = 8.0f;  // lazy running-max threshold (log2 units)
 constexpr int kMaxSplits = 64;      // the plan never cuts a sequence finer
 
 template <int W>
 struct __align__(128) DecodeSmem {
   uint8_t stage[W][kStages][kSegBytes];  // per-warp segment rings (then merge scratch)
+  uint64_t bar[W][kStages];              // one mbarrier per stage
+  uint4 qfrag[8][32];                    // QK A fragments, [k-step][lane]
   float q[8][kHeadDim];                  // rotated query rows (then the merged output)
   float qsum[8];
   float wm[W][8];
   float wl[W][8];
+  float wf[8][W];  // per head: weight of each warp in the CTA merge
+  float hm[8];
+  float hl[8];
   int is_last;
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src));
+// ---- TMA bulk copies completed on mbarriers ---------------------------------
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N));
+// One 1664-byte segment, global -> shared, by the TMA engine, issued by the
+// lanes whose predicate is set (one per warp) without a branch: an
+// async-proxy fence (orders earlier reads of the slot), the barrier's
+// expected byte count, and the bulk copy that completes it.
+__device__ __forceinline__ void bulk_load_segment_if(bool pred, uint8_t* dst, const uint8_t* src, uint64_t* bar) {
+  asm volatile(
+      "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n"
+      "@p fence.proxy.async.shared::cta;\n"
+      "@p mbarrier.arrive.expect_tx.shared::cta.b64 _, [%2], %3;\n"
+      "@p cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %3, [%2]; }" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(smem_u32(bar)), "r"(kSegBytes), "r"(static_cast<uint32_t>(pred))
+      : "memory");
 }
-
-// 1664-byte segment, 104 chunks of 16 B: lane l copies chunks l, l+32, l+64
-// and, for l < 8, l+96.
-__device__ __forceinline__ void copy_segment(uint8_t* dst, const uint8_t* src, int lane) {
-  const uint32_t d = smem_u32(dst);
-#pragma unroll
-  for (int k = 0; k < 3; ++k) cp_async16(d + (lane + 32 * k) * 16, src + (lane + 32 * k) * 16);
-  if (lane < 8) cp_async16(d + (lane + 96) * 16, src + (lane + 96) * 16);
+// One 1664-byte segment, global -> shared, by the TMA engine; the barrier
+// expects the bytes and completes its phase when they have landed.
+__device__ __forceinline__ void bulk_load_segment(uint8_t* dst, const uint8_t* src, uint64_t* bar) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(kSegBytes)
+               : "memory");
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(kSegBytes), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+      : "=r"(done)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+// Bounded, warp-uniform wait for a barrier phase (every lane polls; the warp
+// leaves together): false if the copy never arrived, in which case the caller
+// records KVQ_ERR_DEVICE_TIMEOUT instead of hanging.
+constexpr uint32_t kWaitLimit = 1u << 22;
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  for (uint32_t it = 0; it < kWaitLimit; ++it)
+    if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+  return false;
 }
 
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -101,40 +143,53 @@ __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& hi, uin
   lo = pack_half2(x0 - f.x, x1 - f.y);
 }
 
-// (1024 + c) - 1024 = c exactly, for both halves.
 constexpr uint32_t kBias = 0x64006400u;
-__device__ __forceinline__ uint32_t unbias(uint32_t x) {
-  uint32_t d;
-  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(x), "r"(kBias));
+// (x & mask) | bias in one LOP3 (mask an immediate, bias a register), then
+// the bias subtracted: the masked codes as exact fp16 numbers.
+template <uint32_t kMask>
+__device__ __forceinline__ uint32_t codes_f16(uint32_t x, uint32_t bias) {
+  uint32_t t, d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(t) : "r"(x), "n"(kMask), "r"(bias));
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(t), "r"(bias));
   return d;
 }
+
 
 __device__ __forceinline__ float2 half2_at(const uint8_t* p) {
   return __half22float2(*reinterpret_cast<const __half2*>(p));
 }
 
-// In-place FWHT of 8 rows of 128 floats in smem and the 1/sqrt(128) factor.
-template <int kThreads>
-__device__ __forceinline__ void fwht8_smem(float (*rows)[kHeadDim]) {
-#pragma unroll 1
-  for (int s = 1; s < kHeadDim; s <<= 1) {
-    for (int w = threadIdx.x; w < 8 * (kHeadDim / 2); w += kThreads) {
-      const int g = w / (kHeadDim / 2);
-      const int k = w % (kHeadDim / 2);
-      const int i = (k / s) * 2 * s + (k % s);
-      const float x = rows[g][i], y = rows[g][i + s];
-      rows[g][i] = x + y;
-      rows[g][i + s] = x - y;
+// Walsh-Hadamard transform of one 128-vector held by a warp, element
+// lane + 32k in x[k]: the stride-32 and stride-64 butterflies in registers,
+// strides 1..16 by shuffles (the lower index of a pair keeps u + v, the upper
+// one u - v), then the 1/sqrt(128) factor times `scale`.
+__device__ __forceinline__ void fwht_warp(float (&x)[4], int lane, float scale) {
+  const float y0 = x[0] + x[1], y1 = x[0] - x[1], y2 = x[2] + x[3], y3 = x[2] - x[3];
+  x[0] = y0 + y2;
+  x[2] = y0 - y2;
+  x[1] = y1 + y3;
+  x[3] = y1 - y3;
+#pragma unroll
+  for (int st = 1; st < 32; st <<= 1) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float o = __shfl_xor_sync(0xffffffffu, x[k], st);
+      x[k] = (lane & st) ? o - x[k] : x[k] + o;
     }
-    __syncthreads();
   }
-  for (int w = threadIdx.x; w < 8 * kHeadDim; w += kThreads)
-    rows[w / kHeadDim][w % kHeadDim] *= 0.088388347648318440550f;
-  __syncthreads();
+  const float f = 0.088388347648318440550f * scale;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) x[k] *= f;
+}
+
+__device__ __forceinline__ float ex2(float x) {  // 2^x (MUFU.EX2); ex2(-inf) = 0
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 template <int G, int W>
-__global__ void __launch_bounds__(W * 32, 1) decode_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(W * 32, kMinCtasPerSm) decode_kernel(DecodeArgs a) {
   constexpr int kThreads = W * 32;
   extern __shared__ __align__(128) uint8_t smem_raw[];
   DecodeSmem<W>& sm = *reinterpret_cast<DecodeSmem<W>*>(smem_raw);
@@ -165,68 +220,81 @@ __global__ void __launch_bounds__(W * 32, 1) decode_kernel(DecodeArgs a) {
   const int64_t pstride = static_cast<int64_t>(a.num_kv_heads) * kSegBytes;
 
   // ---- 1. block-table windows (lane l holds the entry of local block 32k+l)
-  //      and the first kStages segments in flight
+  //      and the first kStages segments in flight (lane 0 drives the TMA)
   int32_t win0 = lane < nmine ? bt_row[W * lane] : -1;
   int32_t win1 = 32 + lane < nmine ? bt_row[W * (32 + lane)] : -1;
   int wbase = 0;
-  uint32_t valid_bits = 0;  // bit s: the segment staged in slot s is real
+  if (lane == 0) {
+#pragma unroll
+    for (int s2 = 0; s2 < kStages; ++s2) mbar_init(&sm.bar[warp][s2], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncwarp();
+  uint32_t valid_bits = 0;  // bit s: a copy into slot s is in flight / landed
+  uint32_t phase_bits = 0;  // bit s: parity of slot s's next completion
 #pragma unroll
   for (int i = 0; i < kStages; ++i) {
     const int32_t p = __shfl_sync(0xffffffffu, win0, i);
     if (i < nmine) {
       if (p >= 0 && p < a.num_blocks) {
-        copy_segment(sm.stage[warp][i], pool_h + p * pstride, lane);
+        if (lane == 0) bulk_load_segment(sm.stage[warp][i], pool_h + p * pstride, &sm.bar[warp][i]);
         valid_bits |= 1u << i;
       } else if (lane == 0) {
         record_status(a.status, KVQ_ERR_OUT_OF_RANGE);
       }
     }
-    cp_async_commit();
   }
 
-  // ---- 2. rotate the query (overlaps the copies in flight)
-  for (int i = tid; i < 8 * kHeadDim; i += kThreads) {
-    const int gg = i / kHeadDim;
-    float v = 0.0f;
+  // ---- 2. rotate the query (overlaps the copies in flight): warp w < 8
+  //      owns query head w of this kv head.  tau*log2(e) is folded into q~,
+  //      so scores come out of the MMA already in base-2 logits.
+  for (int gg = warp; gg < 8; gg += W) {
+    float x[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     if (gg < G) {
-      const int64_t qi = (static_cast<int64_t>(b) * a.num_q_heads + h * G + gg) * kHeadDim + i % kHeadDim;
-      v = load_as_f32(a.q, a.q_dtype, qi);
-    }
-    sm.q[gg][i % kHeadDim] = v;
-  }
-  __syncthreads();
-  fwht8_smem<kThreads>(sm.q);
-  if (warp < 8) {
-    const int gg = warp;
-    float s = sm.q[gg][lane] + sm.q[gg][lane + 32] + sm.q[gg][lane + 64] + sm.q[gg][lane + 96];
+      const int64_t q0 = (static_cast<int64_t>(b) * a.num_q_heads + h * G + gg) * kHeadDim;
 #pragma unroll
-    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (lane == 0) sm.qsum[gg] = s;
+      for (int k = 0; k < 4; ++k) x[k] = load_as_f32(a.q, a.q_dtype, q0 + lane + 32 * k);
+    }
+    fwht_warp(x, lane, a.scale_log2);
+    float s4 = (x[0] + x[1]) + (x[2] + x[3]);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) s4 += __shfl_xor_sync(0xffffffffu, s4, o);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) sm.q[gg][lane + 32 * k] = x[k];
+    if (lane == 0) sm.qsum[gg] = s4;
   }
   __syncthreads();
 
-  // QK A fragments.  k-step kk reads word w = 4c + kk/2 of a key row (dims
-  // 8w..8w+7).  Slots (2c, 2c+1) take dims (8w+e, 8w+e+4) and slots
-  // (2c+8, 2c+9) take (8w+e+1, 8w+e+5), e = 0 for even kk and 2 for odd kk;
-  // the second pair's codes sit 4 bits higher (x16), so its q is /16.
-  uint32_t qa[8][4];
-#pragma unroll
-  for (int kk = 0; kk < 8; ++kk) {
+  // QK A fragments in smem, [k-step][lane], built by warp kk for its k-step
+  // and read back with one 16-byte load per k-step.  k-step kk reads word
+  // w = 4c + kk/2 of a key row (dims 8w..8w+7).  Slots (2c, 2c+1) take dims
+  // (8w+e, 8w+e+4) and slots (2c+8, 2c+9) take (8w+e+1, 8w+e+5), e = 0 for
+  // even kk and 2 for odd kk; the second pair's codes sit 4 bits higher (x16),
+  // so its q is /16.
+  for (int kk = warp; kk < 8; kk += W) {
     const int w = 4 * c + (kk >> 1);
     const int e = (kk & 1) ? 2 : 0;
     const float* qr = sm.q[g];
-    split_pair(qr[8 * w + e], qr[8 * w + e + 4], qa[kk][0], qa[kk][1]);
-    split_pair(qr[8 * w + e + 1] * 0.0625f, qr[8 * w + e + 5] * 0.0625f, qa[kk][2], qa[kk][3]);
+    uint4 f;
+    split_pair(qr[8 * w + e], qr[8 * w + e + 4], f.x, f.y);
+    split_pair(qr[8 * w + e + 1] * 0.0625f, qr[8 * w + e + 5] * 0.0625f, f.z, f.w);
+    sm.qfrag[kk][lane] = f;
   }
-  const float zq = a.scale_log2 * sm.qsum[g];
-  const float kscale = a.scale_log2;
+  const float zq = sm.qsum[g];
+  __syncthreads();
 
-  // PV B operand: n-tile nt covers dims 8nt..8nt+7, column g is dim 8nt+g:
-  // byte 2(nt&1) + g/4 of word nt/2 of a value row, crumb g%4 (kept in place,
-  // so column g's codes carry a factor 4^(g%4)).
-  const uint32_t vsel0 = static_cast<uint32_t>((g >> 2) | ((4 + (g >> 2)) << 8));
-  const uint32_t vsel1 = static_cast<uint32_t>((2 + (g >> 2)) | ((6 + (g >> 2)) << 8));
-  const uint32_t vmask = 0x00030003u << (2 * (g & 3));
+  // PV B operand through ldmatrix.trans: 8x8 tiles of 16-bit elements of the
+  // value rows (tokens x 8 crumbs).  Tile i covers tokens 8(i/2)..8(i/2)+7 and
+  // dims 64(i%2)..64(i%2)+63; after the transpose lane (g, c) holds, for
+  // tokens (2c, 2c+1) of the tile, the 16 bits of dims 64h+8g .. 64h+8g+7.
+  // n-tile (h, k) takes crumb k of those 16 bits, i.e. column g is dim
+  // 64h + 8g + k.  Crumbs 0..4 are masked in place (code times 4^k), crumbs
+  // 5..7 after a 10-bit shift (code times 4^(k-5)).
+  const int ld_tok = ((lane >> 4) << 3) + (lane & 7);
+  const int ld_half = (lane >> 3) & 1;
+
+  uint32_t bias;
+  asm volatile("mov.b32 %0, %1;" : "=r"(bias) : "n"(kBias));
 
   float o[16][4];
 #pragma unroll
@@ -235,105 +303,129 @@ __global__ void __launch_bounds__(W * 32, 1) decode_kernel(DecodeArgs a) {
   float l_part = 0.0f, z_part = 0.0f;
 
   // ---- 3. the paged scan
+  bool timed_out = false;
+  int slot = 0;
 #pragma unroll 1
-  for (int i = 0; i < nmine; ++i) {
-    const int slot = i % kStages;
-    cp_async_wait<kStages - 1>();
-    __syncwarp();
+  for (int i = 0; i < nmine; ++i, slot = (slot + 1 == kStages) ? 0 : slot + 1) {
+    if (valid_bits & (1u << slot)) {
+      if (!mbar_wait(&sm.bar[warp][slot], (phase_bits >> slot) & 1u)) {
+        timed_out = true;
+        break;
+      }
+      phase_bits ^= 1u << slot;
+    }
     if (valid_bits & (1u << slot)) {
       const uint8_t* sg = sm.stage[warp][slot];
       const int ntok = min(kBlockSize, L - (blk0 + warp + W * i) * kBlockSize);
 
-      // scores: n-tile j holds tokens 8j..8j+7, column g is token 8j+g; two
-      // accumulator chains per n-tile (even / odd k-steps) halve the latency
-      float sacc[2][2][4];
+      // scores: n-tile j holds tokens 8j..8j+7, column g is token 8j+g
+      float sacc[2][2][4];  // [n-tile][chain: even / odd k-steps]
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
+      for (int j = 0; j < 2; ++j)
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) sacc[j][ch][0] = sacc[j][ch][1] = sacc[j][ch][2] = sacc[j][ch][3] = 0.0f;
-      }
       const uint4 kw0 = *reinterpret_cast<const uint4*>(sg + kOffK + g * kKRowBytes + 16 * c);
       const uint4 kw1 = *reinterpret_cast<const uint4*>(sg + kOffK + (8 + g) * kKRowBytes + 16 * c);
       const uint32_t words[2][4] = {{kw0.x, kw0.y, kw0.z, kw0.w}, {kw1.x, kw1.y, kw1.z, kw1.w}};
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
+        const uint4 f = sm.qfrag[kk][lane];
+        const uint32_t qa[4] = {f.x, f.y, f.z, f.w};
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
           const uint32_t w = (kk & 1) ? (words[j][kk >> 1] >> 8) : words[j][kk >> 1];
-          mma16816(sacc[j][kk & 1], qa[kk], unbias((w & 0x000F000Fu) | kBias), unbias((w & 0x00F000F0u) | kBias));
+          mma16816(sacc[j][kk & 1], qa, codes_f16<0x000F000Fu>(w, bias), codes_f16<0x00F000F0u>(w, bias));
         }
       }
-      // fold S_K, Z_K: s = tau log2e (S_K 2^24 (hi + lo) + Z_K sum q~)
+      // fold S_K, Z_K: s = tau log2e (S_K (hi + lo) + Z_K sum q~)
       float sc[4];
-      float mx = -CUDART_INF_F;
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const float2 sk = half2_at(sg + kOffSK + 4 * (4 * j + c));
         const float2 zk = half2_at(sg + kOffZK + 4 * (4 * j + c));
-        const int t0 = 8 * j + 2 * c;
         const float d0 = (sacc[j][0][0] + sacc[j][1][0]) + (sacc[j][0][2] + sacc[j][1][2]);
         const float d1 = (sacc[j][0][1] + sacc[j][1][1]) + (sacc[j][0][3] + sacc[j][1][3]);
-        sc[2 * j] = t0 < ntok ? fmaf(kscale * sk.x, d0, zk.x * zq) : -CUDART_INF_F;
-        sc[2 * j + 1] = t0 + 1 < ntok ? fmaf(kscale * sk.y, d1, zk.y * zq) : -CUDART_INF_F;
-        mx = fmaxf(mx, fmaxf(sc[2 * j], sc[2 * j + 1]));
+        sc[2 * j] = fmaf(sk.x, d0, zk.x * zq);
+        sc[2 * j + 1] = fmaf(sk.y, d1, zk.y * zq);
       }
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      if (mx > m_ref) {  // new running max for head g: rescale this thread's state
-        const float alpha = m_ref == -CUDART_INF_F ? 0.0f : exp2f(m_ref - mx);
+      if (ntok < kBlockSize) {  // the last block of a sequence: drop the empty rows
 #pragma unroll
-        for (int nt = 0; nt < 16; ++nt) {
-          o[nt][0] *= alpha;
-          o[nt][1] *= alpha;
-          o[nt][2] *= alpha;
-          o[nt][3] *= alpha;
-        }
-        l_part *= alpha;
-        z_part *= alpha;
-        m_ref = mx;
+        for (int q = 0; q < 4; ++q)
+          if (8 * (q >> 1) + 2 * c + (q & 1) >= ntok) sc[q] = -CUDART_INF_F;
       }
+      // Lazy running max: rescale only when a score exceeds the reference by
+      // more than 8 (base 2).  Probabilities are taken relative to m_ref + 8,
+      // p = 2^(s - m_ref - 8) <= 1, so p' = p S_V <= S_V always fits fp16;
+      // o, l and zeta all carry the same factor, which the final o / l
+      // cancels.  One warp vote decides; the head max (shuffles) and the
+      // rescale run only when some lane needs them.
+      const float mloc = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+      if (__any_sync(0xffffffffu, mloc > m_ref + kRescaleLog2)) {
+        float mx = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        if (mx > m_ref + kRescaleLog2) {
+          const float alpha = m_ref == -CUDART_INF_F ? 0.0f : ex2(m_ref - mx);
+#pragma unroll
+          for (int nt = 0; nt < 16; ++nt) {
+            o[nt][0] *= alpha;
+            o[nt][1] *= alpha;
+            o[nt][2] *= alpha;
+            o[nt][3] *= alpha;
+          }
+          l_part *= alpha;
+          z_part *= alpha;
+          m_ref = mx;
+        }
+      }
+      const float m8 = m_ref + kRescaleLog2;
       // probabilities with the value scale folded in: p' = p S_V
       float pv[4];
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
-        const float2 sv = half2_at(sg + kOffSV + 4 * (4 * j + c));
-        const float2 zv = half2_at(sg + kOffZV + 4 * (4 * j + c));
-        const int t0 = 8 * j + 2 * c;
-        const float p0 = t0 < ntok ? exp2f(sc[2 * j] - m_ref) : 0.0f;
-        const float p1 = t0 + 1 < ntok ? exp2f(sc[2 * j + 1] - m_ref) : 0.0f;
+        float2 sv = half2_at(sg + kOffSV + 4 * (4 * j + c));
+        float2 zv = half2_at(sg + kOffZV + 4 * (4 * j + c));
+        if (ntok < kBlockSize) {  // rows past the end may hold NaN metadata
+          if (8 * j + 2 * c >= ntok) sv.x = zv.x = 0.0f;
+          if (8 * j + 2 * c + 1 >= ntok) sv.y = zv.y = 0.0f;
+        }
+        const float p0 = ex2(sc[2 * j] - m8);
+        const float p1 = ex2(sc[2 * j + 1] - m8);
         l_part += p0 + p1;
-        pv[2 * j] = t0 < ntok ? p0 * sv.x : 0.0f;
-        pv[2 * j + 1] = t0 + 1 < ntok ? p1 * sv.y : 0.0f;
-        if (t0 < ntok) z_part = fmaf(p0, zv.x, z_part);
-        if (t0 + 1 < ntok) z_part = fmaf(p1, zv.y, z_part);
+        z_part = fmaf(p0, zv.x, fmaf(p1, zv.y, z_part));
+        pv[2 * j] = p0 * sv.x;
+        pv[2 * j + 1] = p1 * sv.y;
       }
       uint32_t pa[4];
       split_pair(pv[0], pv[1], pa[0], pa[1]);
       split_pair(pv[2], pv[3], pa[2], pa[3]);
 
-      // p'.c_V: value rows of tokens 2c, 2c+1, 8+2c, 9+2c
-      const uint4* vr = reinterpret_cast<const uint4*>(sg + kOffV);
-      const uint4 va0 = vr[(2 * c) * 2], va1 = vr[(2 * c) * 2 + 1];
-      const uint4 vb0 = vr[(2 * c + 1) * 2], vb1 = vr[(2 * c + 1) * 2 + 1];
-      const uint4 vc0 = vr[(8 + 2 * c) * 2], vc1 = vr[(8 + 2 * c) * 2 + 1];
-      const uint4 vd0 = vr[(9 + 2 * c) * 2], vd1 = vr[(9 + 2 * c) * 2 + 1];
-      const uint32_t tA[8] = {va0.x, va0.y, va0.z, va0.w, va1.x, va1.y, va1.z, va1.w};
-      const uint32_t tB[8] = {vb0.x, vb0.y, vb0.z, vb0.w, vb1.x, vb1.y, vb1.z, vb1.w};
-      const uint32_t tC[8] = {vc0.x, vc0.y, vc0.z, vc0.w, vc1.x, vc1.y, vc1.z, vc1.w};
-      const uint32_t tD[8] = {vd0.x, vd0.y, vd0.z, vd0.w, vd1.x, vd1.y, vd1.z, vd1.w};
+      // p'.c_V: one ldmatrix.x4.trans gives this lane's value operands
+      uint32_t vr[4];
+      {
+        const uint32_t addr = smem_u32(sg + kOffV + ld_tok * kVRowBytes + 16 * ld_half);
+        asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(vr[0]), "=r"(vr[1]), "=r"(vr[2]), "=r"(vr[3])
+                     : "r"(addr));
+      }
+      const uint32_t vs[4] = {vr[0] >> 10, vr[1] >> 10, vr[2] >> 10, vr[3] >> 10};
 #pragma unroll
-      for (int nt = 0; nt < 16; ++nt) {
-        const uint32_t sel = (nt & 1) ? vsel1 : vsel0;
-        const uint32_t b0 = unbias((__byte_perm(tA[nt >> 1], tB[nt >> 1], sel) & vmask) | kBias);
-        const uint32_t b1 = unbias((__byte_perm(tC[nt >> 1], tD[nt >> 1], sel) & vmask) | kBias);
-        mma16816(o[nt], pa, b0, b1);
+      for (int h2 = 0; h2 < 2; ++h2) {
+        mma16816(o[8 * h2 + 0], pa, codes_f16<0x00030003u>(vr[h2], bias), codes_f16<0x00030003u>(vr[2 + h2], bias));
+        mma16816(o[8 * h2 + 1], pa, codes_f16<0x000C000Cu>(vr[h2], bias), codes_f16<0x000C000Cu>(vr[2 + h2], bias));
+        mma16816(o[8 * h2 + 2], pa, codes_f16<0x00300030u>(vr[h2], bias), codes_f16<0x00300030u>(vr[2 + h2], bias));
+        mma16816(o[8 * h2 + 3], pa, codes_f16<0x00C000C0u>(vr[h2], bias), codes_f16<0x00C000C0u>(vr[2 + h2], bias));
+        mma16816(o[8 * h2 + 4], pa, codes_f16<0x03000300u>(vr[h2], bias), codes_f16<0x03000300u>(vr[2 + h2], bias));
+        mma16816(o[8 * h2 + 5], pa, codes_f16<0x00030003u>(vs[h2], bias), codes_f16<0x00030003u>(vs[2 + h2], bias));
+        mma16816(o[8 * h2 + 6], pa, codes_f16<0x000C000Cu>(vs[h2], bias), codes_f16<0x000C000Cu>(vs[2 + h2], bias));
+        mma16816(o[8 * h2 + 7], pa, codes_f16<0x00300030u>(vs[h2], bias), codes_f16<0x00300030u>(vs[2 + h2], bias));
       }
     } else if (lane == 0 && i >= kStages) {
       record_status(a.status, KVQ_ERR_OUT_OF_RANGE);
     }
-    __syncwarp();
+    __syncwarp();  // every lane is done reading the slot before it is refilled
     // refill this slot with the warp's block j = i + kStages
     const int j = i + kStages;
+    valid_bits &= ~(1u << slot);
     if (j < nmine) {
       if (j >= wbase + 32) {  // slide the block-table window by 32 entries
         win0 = win1;
@@ -342,15 +434,20 @@ __global__ void __launch_bounds__(W * 32, 1) decode_kernel(DecodeArgs a) {
       }
       const int32_t p = __shfl_sync(0xffffffffu, win0, j - wbase);
       if (p >= 0 && p < a.num_blocks) {
-        copy_segment(sm.stage[warp][slot], pool_h + p * pstride, lane);
+        bulk_load_segment_if(lane == 0, sm.stage[warp][slot], pool_h + p * pstride, &sm.bar[warp][slot]);
         valid_bits |= 1u << slot;
-      } else {
-        valid_bits &= ~(1u << slot);
       }
     }
-    cp_async_commit();
   }
-  cp_async_wait<0>();
+  if (timed_out) {
+    // a copy never landed: report it, give the others a bounded chance to
+    // finish, and leave this warp's contribution empty
+    if (lane == 0) record_status(a.status, KVQ_ERR_DEVICE_TIMEOUT);
+    for (int s2 = 0; s2 < kStages; ++s2)
+      if (valid_bits & (1u << s2)) mbar_wait(&sm.bar[warp][s2], (phase_bits >> s2) & 1u);
+    m_ref = -CUDART_INF_F;
+    l_part = z_part = 0.0f;
+  }
 
   // ---- 4. merge: lanes of a head, then warps, then splits
   l_part += __shfl_xor_sync(0xffffffffu, l_part, 1);
@@ -360,13 +457,17 @@ __global__ void __launch_bounds__(W * 32, 1) decode_kernel(DecodeArgs a) {
   __syncthreads();  // every warp is done with its stages: reuse them
   float(*wo)[8][kHeadDim] = reinterpret_cast<float(*)[8][kHeadDim]>(&sm.stage[0][0][0]);
   {
-    // column n of n-tile nt is dim 8nt + n with code factor 4^(n%4) 2^-24
-    const float f0 = 1.0f / static_cast<float>(1 << (2 * ((2 * c) & 3)));
-    const float f1 = 1.0f / static_cast<float>(1 << (2 * ((2 * c + 1) & 3)));
+    // n-tile (h, k) column n is dim 64h + 8n + k; its codes carry 4^k
+    // (k <= 4) or 4^(k-5) (k >= 5)
 #pragma unroll
-    for (int nt = 0; nt < 16; ++nt) {
-      wo[warp][g][8 * nt + 2 * c] = fmaf(o[nt][0] + o[nt][2], f0, z_part);
-      wo[warp][g][8 * nt + 2 * c + 1] = fmaf(o[nt][1] + o[nt][3], f1, z_part);
+    for (int h2 = 0; h2 < 2; ++h2) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float f = 1.0f / static_cast<float>(1 << (2 * (k < 5 ? k : k - 5)));
+        const int nt = 8 * h2 + k;
+        wo[warp][g][64 * h2 + 16 * c + k] = fmaf(o[nt][0] + o[nt][2], f, z_part);
+        wo[warp][g][64 * h2 + 16 * c + 8 + k] = fmaf(o[nt][1] + o[nt][3], f, z_part);
+      }
     }
     if (c == 0) {
       sm.wm[warp][g] = m_ref;
@@ -374,21 +475,30 @@ __global__ void __launch_bounds__(W * 32, 1) decode_kernel(DecodeArgs a) {
     }
   }
   __syncthreads();
-  for (int t = tid; t < G * kHeadDim; t += kThreads) {
-    const int gg = t / kHeadDim, d = t % kHeadDim;
+  // per head: the warps' common max, their weights 2^(m_w - M), and l
+  if (tid < G) {
+    const int gg = tid;
     float M = -CUDART_INF_F;
 #pragma unroll
     for (int w = 0; w < W; ++w)
       if (sm.wl[w][gg] > 0.0f) M = fmaxf(M, sm.wm[w][gg]);
-    float lsum = 0.0f, acc = 0.0f;
+    float lsum = 0.0f;
 #pragma unroll
     for (int w = 0; w < W; ++w) {
-      if (sm.wl[w][gg] > 0.0f) {
-        const float f = exp2f(sm.wm[w][gg] - M);
-        lsum = fmaf(sm.wl[w][gg], f, lsum);
-        acc = fmaf(wo[w][gg][d], f, acc);
-      }
+      const float f = sm.wl[w][gg] > 0.0f ? ex2(sm.wm[w][gg] - M) : 0.0f;
+      sm.wf[gg][w] = f;
+      lsum = fmaf(sm.wl[w][gg], f, lsum);
     }
+    sm.hm[gg] = M;
+    sm.hl[gg] = lsum;
+  }
+  __syncthreads();
+  for (int t = tid; t < G * kHeadDim; t += kThreads) {
+    const int gg = t / kHeadDim, d = t % kHeadDim;
+    float acc = 0.0f;
+#pragma unroll
+    for (int w = 0; w < W; ++w) acc = fmaf(wo[w][gg][d], sm.wf[gg][w], acc);
+    const float M = sm.hm[gg], lsum = sm.hl[gg];
     float* rec =
         a.partials + ((static_cast<int64_t>(b) * a.num_q_heads + h * G + gg) * a.nsplit + split) * kPartialFloats;
     if (a.nsplit == 1) {
@@ -424,8 +534,7 @@ __global__ void __launch_bounds__(W * 32, 1) decode_kernel(DecodeArgs a) {
       mls[G * ns + t] = ml.y;
     }
     __syncthreads();
-    if (warp < G) {
-      const int gg = warp;
+    for (int gg = warp; gg < G; gg += W) {
       float M = -CUDART_INF_F;
       for (int s = lane; s < ns; s += 32)
         if (mls[G * ns + gg * ns + s] > 0.0f) M = fmaxf(M, mls[gg * ns + s]);
@@ -434,14 +543,14 @@ __global__ void __launch_bounds__(W * 32, 1) decode_kernel(DecodeArgs a) {
       float lsum = 0.0f;
       for (int s = lane; s < ns; s += 32) {
         const float l = mls[G * ns + gg * ns + s];
-        if (l > 0.0f) lsum = fmaf(l, exp2f(mls[gg * ns + s] - M), lsum);
+        if (l > 0.0f) lsum = fmaf(l, ex2(mls[gg * ns + s] - M), lsum);
       }
 #pragma unroll
       for (int off = 16; off; off >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
       const float inv = lsum > 0.0f ? 1.0f / lsum : 0.0f;
       for (int s = lane; s < ns; s += 32) {
         const float l = mls[G * ns + gg * ns + s];
-        mls[2 * G * ns + gg * ns + s] = l > 0.0f ? exp2f(mls[gg * ns + s] - M) * inv : 0.0f;
+        mls[2 * G * ns + gg * ns + s] = l > 0.0f ? ex2(mls[gg * ns + s] - M) * inv : 0.0f;
       }
     }
     __syncthreads();
@@ -480,19 +589,19 @@ __global__ void __launch_bounds__(W * 32, 1) decode_kernel(DecodeArgs a) {
     }
     if (tid == 0) a.tickets[b * a.num_kv_heads + h] = 0;  // ready for the next call
   }
-  for (int t = G * kHeadDim + tid; t < 8 * kHeadDim; t += kThreads) sm.q[t / kHeadDim][t % kHeadDim] = 0.0f;
   __syncthreads();
 
-  // rotate back once and store
-  fwht8_smem<kThreads>(sm.q);
-  for (int i = tid; i < G * kHeadDim; i += kThreads) {
-    const int gg = i / kHeadDim;
-    const int64_t oi = (static_cast<int64_t>(b) * a.num_q_heads + h * G + gg) * kHeadDim + i % kHeadDim;
-    store_from_f32(a.out, a.out_dtype, oi, sm.q[gg][i % kHeadDim]);
+  // rotate back once (warp w owns heads w, w+W, ...) and store
+  for (int gg = warp; gg < G; gg += W) {
+    float x[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) x[k] = sm.q[gg][lane + 32 * k];
+    fwht_warp(x, lane, 1.0f);
+    const int64_t o0 = (static_cast<int64_t>(b) * a.num_q_heads + h * G + gg) * kHeadDim;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) store_from_f32(a.out, a.out_dtype, o0 + lane + 32 * k, x[k]);
   }
 }
-
-constexpr int kDecodeWarps = 8;
 
 template <int G>
 cudaError_t launch_g(const DecodeArgs& a, cudaStream_t stream) {
