@@ -71,6 +71,8 @@ def lib():
                                                         ctypes.c_int, vp, sz, vp]),
                 "kvq_decode_attention_ex": (ctypes.c_int, [dp, vp, ctypes.c_int, i32, i32, vp, i32, vp, i32, f32,
                                                            vp, ctypes.c_int, vp, sz, i32, vp]),
+                "kvq_decode_attention_noalloc": (ctypes.c_int, [dp, vp, ctypes.c_int, i32, i32, vp, i32, vp, i32, f32,
+                                                                vp, ctypes.c_int, vp]),
                 "kvq_last_device_status": (ctypes.c_int, [vp]),
                 "kvq_error_string": (ctypes.c_char_p, [ctypes.c_int]),
             }
@@ -197,6 +199,18 @@ def kvq_decode_attention(pool, num_blocks, num_kv_heads, q, block_table, seq_len
                                        _dtype_code(out), _ptr(workspace), workspace.numel(), blocks_per_split,
                                        _stream_ptr(stream))
     _check(rc, "kvq_decode_attention")
+
+
+def kvq_decode_attention_noalloc(pool, num_blocks, num_kv_heads, q, block_table, seq_lens, max_seq_len, out,
+                                 softmax_scale=0.0, stream=None):
+    """kvq_decode_attention with the library's fixed device scratch instead of
+    a caller workspace (for callers that cannot allocate at call time)."""
+    desc = make_desc(num_blocks, num_kv_heads, pool)
+    batch, hq, _ = q.shape
+    rc = lib().kvq_decode_attention_noalloc(ctypes.byref(desc), _ptr(q), _dtype_code(q), batch, hq,
+                                            _ptr(block_table), block_table.shape[1], _ptr(seq_lens), max_seq_len,
+                                            softmax_scale, _ptr(out), _dtype_code(out), _stream_ptr(stream))
+    _check(rc, "kvq_decode_attention_noalloc")
 
 
 def kvq_last_device_status(stream=None) -> int:

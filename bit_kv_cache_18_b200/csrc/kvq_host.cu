@@ -45,6 +45,27 @@ uint64_t splitmix64(uint64_t x) {
 
 }  // namespace
 
+// Fixed split-K scratch for kvq_decode_attention_noalloc.  It lives in the
+// module image, so every GPU that loads this library holds the full 32 MiB
+// until the process exits.  Host code must never pass the symbol itself to
+// a kernel (on the host it is only a stand-in): the device address comes
+// from cudaGetSymbolAddress, once per device, with that device current.
+constexpr size_t kStaticScratchBytes = size_t(32) << 20;
+static __device__ __align__(256) uint8_t g_kvq_scratch[kStaticScratchBytes];
+void* g_scratch_ptr[kMaxDevices] = {nullptr};
+
+void* device_scratch_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_attr_mutex);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_kvq_scratch) != cudaSuccess || !p) return nullptr;
+    g_scratch_ptr[dev] = p;
+  }
+  return g_scratch_ptr[dev];
+}
+
 int* device_status_ptr() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
@@ -317,6 +338,30 @@ int kvq_decode_attention(const kvq_cache_desc* desc, const void* q, kvq_dtype q_
   return kvq_decode_attention_ex(desc, q, q_dtype, batch, num_q_heads, block_table, max_blocks_per_seq,
                                  seq_lens, max_seq_len, softmax_scale, out, out_dtype, workspace, ws_bytes,
                                  0, stream);
+}
+
+int kvq_decode_attention_noalloc(const kvq_cache_desc* desc, const void* q, kvq_dtype q_dtype,
+                                 int32_t batch, int32_t num_q_heads, const int32_t* block_table,
+                                 int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                                 int32_t max_seq_len, float softmax_scale, void* out,
+                                 kvq_dtype out_dtype, void* stream) {
+  int rc = check_desc(desc);
+  if (rc != KVQ_OK) return rc;
+  if (batch < 0 || num_q_heads <= 0 || num_q_heads % desc->num_kv_heads != 0) return KVQ_ERR_INVALID;
+  if (batch == 0) return KVQ_OK;
+  DecodePlan plan;
+  rc = plan_decode(batch, desc->num_kv_heads, num_q_heads, max_seq_len, 0, &plan);
+  if (rc != KVQ_OK) return rc;
+  if (plan.total_bytes > kStaticScratchBytes) return KVQ_ERR_WORKSPACE;  // beyond the fixed scratch
+  void* scratch = device_scratch_ptr();
+  if (!scratch) return KVQ_ERR_CUDA;
+  // The scratch keeps whatever the previous call left; the tickets must start
+  // at zero (the partials are always written before they are read).
+  if (cudaMemsetAsync(scratch, 0, plan.ticket_bytes, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return KVQ_ERR_CUDA;
+  return kvq_decode_attention_ex(desc, q, q_dtype, batch, num_q_heads, block_table, max_blocks_per_seq,
+                                 seq_lens, max_seq_len, softmax_scale, out, out_dtype, scratch,
+                                 kStaticScratchBytes, 0, stream);
 }
 
 int kvq_last_device_status(void* stream) {

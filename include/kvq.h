@@ -179,6 +179,30 @@ int kvq_decode_attention_ex(const kvq_cache_desc* desc, const void* q, kvq_dtype
                             kvq_dtype out_dtype, void* workspace, size_t ws_bytes,
                             int32_t blocks_per_split, void* stream);
 
+/* kvq_decode_attention without a caller-provided workspace, for callers that
+ * cannot allocate device memory at call time: code that runs inside a memory
+ * pool or allocator that forbids runtime allocations, embedded or plugin
+ * callers that receive only input and output buffers, and hosts whose
+ * allocation calls would synchronise the device in the middle of a step.
+ * (The pages have no counterpart; this is a packaging convenience.)
+ * Arguments are those of kvq_decode_attention minus the workspace; the
+ * default split plan is used.  The split-K scratch is a fixed 32 MiB array
+ * inside the library's device image, so every GPU that loads the library
+ * holds it until the process exits; a problem whose scratch would exceed
+ * 32 MiB returns KVQ_ERR_WORKSPACE and launches nothing.  No allocation is
+ * made by this call: it clears the scratch's ticket area with an
+ * asynchronous memset and launches the decode kernel on the stream.  The
+ * first call on each device looks up the scratch's device address (a one-time
+ * set-up), so make that first call before any stream capture.  All calls on
+ * a device share the one scratch array: calls that may overlap on the GPU
+ * (different streams without ordering between them) race and give wrong
+ * results; order them on one stream. */
+int kvq_decode_attention_noalloc(const kvq_cache_desc* desc, const void* q, kvq_dtype q_dtype,
+                                 int32_t batch, int32_t num_q_heads, const int32_t* block_table,
+                                 int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                                 int32_t max_seq_len, float softmax_scale, void* out,
+                                 kvq_dtype out_dtype, void* stream);
+
 /* Synchronise the stream, then read and clear the current device's status
  * word: KVQ_OK, or the first error that a kernel recorded since the last
  * read (KVQ_ERR_OUT_OF_RANGE, KVQ_ERR_DEVICE_TIMEOUT).  Returns
