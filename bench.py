@@ -16,7 +16,10 @@ figure with pinned host copies inside the timed region; and the CPU oracle's
 throughput on a bounded sample.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kvq|reference]
-                    [--workload qwen3-32b-16k|batched|long|mixed]
+                    [--profile qwen3-32b-16k|batched|long|mixed]
+
+--profile times the decode kernel alone on one workload and prints its
+per-launch time; it is the command the ncu summaries are taken with.
 
 For N > 1 (torchrun), every rank runs an independent replica (the path has
 no cross-GPU step); the timing is the max over ranks and the value sums all
@@ -43,6 +46,23 @@ import synth  # noqa: E402
 METRIC = "decode attention tokens/s and effective HBM GB/s (% of roofline), quantize GB/s"
 SEG = 1664
 BYTES_PER_TOKEN_HEAD = 104
+
+
+# DRAM bytes (read + write) of one decode launch on the Qwen3-32B layer
+# workload, from `ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum`
+# (cache control on: every replay starts cold, as every launch of the step
+# does), with the SHA-256 of the kernel source it was taken on.  Reported as
+# roofline.traffic only while the source still has that hash.
+DECODE_TRAFFIC = {"sha256": "aed9f72ee907e32f8499707fabf6e67699a33c58775e209cd6e4de5755febc69",
+                  "bytes": 13783296}
+
+
+def decode_traffic():
+    import hashlib
+    path = os.path.join(ROOT, "bit_kv_cache_18_b200", "csrc", "kvq_decode.cu")
+    with open(path, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    return DECODE_TRAFFIC["bytes"] if sha == DECODE_TRAFFIC["sha256"] else None
 
 
 def measured_peaks():
@@ -88,22 +108,62 @@ def aggregate(dist, local_ms: float, local_units: float, device=None):
 # --------------------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi samples every 200 ms while the timed region runs."""
+    """SM clock and clock-event reasons sampled while a timed region runs.
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    Reads NVML from a background thread every ~2 ms (read-only queries; the
+    timed regions here last tens of milliseconds, too short for
+    nvidia-smi's 200 ms loop), falling back to `nvidia-smi -lms 200`.  The
+    samples are written to gpurun_out/clocks_rank<i>.csv."""
 
-    def __init__(self, index: int):
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4), ("hw_power_brake_slowdown", 0x80))
+
+    def __init__(self, index: int, uuid: str | None = None, period_s: float = 0.002):
         self.index = index
+        self.uuid = uuid
+        self.period = period_s
+        self.rows = []  # (t, sm_mhz, max_mhz, power_w, reasons bitmask)
         self.proc = None
+        self.thread = None
+        self.nvml = None
         self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
 
+    def _poll(self):
+        nv, h = self.nvml, self.handle
+        max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        while not self.stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+            except Exception:  # noqa: BLE001 - a failed read ends sampling, not the bench
+                break
+            self.rows.append((time.perf_counter(), sm, max_mhz, pw, rs))
+            self.stop.wait(self.period)
+
     def __enter__(self):
+        import threading
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            # by UUID: NVML enumerates every GPU of the machine, CUDA only the visible ones
+            self.handle = (pynvml.nvmlDeviceGetHandleByUUID(self.uuid) if self.uuid
+                           else pynvml.nvmlDeviceGetHandleByIndex(self.index))
+            self.stop = threading.Event()
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            deadline = time.perf_counter() + 2.0
+            while not self.rows and time.perf_counter() < deadline:
+                time.sleep(0.001)
+            return self
+        except Exception:  # noqa: BLE001
+            self.nvml = None
         try:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+            fields = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={fields}", "--format=csv,noheader,nounits",
                                           "-i", str(self.index), "-lms", "200"], stdout=self.f,
                                          stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
@@ -111,6 +171,18 @@ class ClockSampler:
         return self
 
     def __exit__(self, *exc):
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
+            try:
+                os.makedirs(os.path.dirname(self.path), exist_ok=True)
+                with open(self.path, "w") as f:
+                    f.write("t_s,sm_mhz,max_sm_mhz,power_w,reasons_hex\n")
+                    for t, sm, mx, pw, rs in self.rows:
+                        f.write(f"{t:.4f},{sm},{mx},{pw:.1f},{rs:#x}\n")
+            except OSError:
+                pass
+            self.nvml.nvmlShutdown()
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -118,24 +190,30 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
             self.f.close()
+            with open(self.path) as f:
+                for line in f:
+                    p = [x.strip() for x in line.split(",")]
+                    if len(p) >= 4 and p[0].replace(".", "").isdigit():
+                        rs = int(p[3], 16) if p[3].lower().startswith("0x") else 0
+                        self.rows.append((0.0, float(p[0]), float(p[1]), float(p[2] or 0), rs))
 
     def summary(self):
-        if self.proc is None or not os.path.exists(self.path):
+        if not self.rows:
             return None
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [x.strip() for x in line.split(",")]
-                if len(parts) >= 8:
-                    rows.append(parts)
-        if not rows:
-            return None
-        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": float(rows[0][1]) if rows[0][1].replace(".", "").isdigit() else None,
-                "reasons": reasons, "samples": len(rows)}
+        sm = [r[1] for r in self.rows]
+        mask = 0
+        for r in self.rows:
+            mask |= int(r[4])
+        return {"sm_mhz": statistics.median(sm), "sm_min_mhz": min(sm), "sm_max_mhz": float(self.rows[0][2]),
+                "reasons": [n for n, bit in self.REASONS if mask & bit], "samples": len(self.rows),
+                "source": "nvml" if self.thread is not None else "nvidia-smi"}
+
+
+def device_uuid(torch, dev):
+    try:
+        return "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:  # noqa: BLE001
+        return None
 
 
 # --------------------------------------------------------------------------- the step
@@ -307,6 +385,72 @@ class OracleSample:
         return time.perf_counter() - t0
 
 
+# --------------------------------------------------------------------------- profile mode
+
+PROFILE_WORKLOADS = {
+    "qwen3-32b-16k": lambda: synth.qwen3_32b_layer(0),
+    "batched": lambda: synth.batched(0),
+    "long": lambda: synth.long_context(0),
+    "mixed": lambda: synth.mixed_decode(0),
+}
+
+
+def profile_decode(args):
+    """Decode launches alone on one workload, for ncu captures and sweeps.
+
+    The pool is filled from the seeded workload: the first min(16384, total)
+    tokens are quantized through the library and their segments repeated over
+    the rest of the pool (same value distribution, no host-side generation of
+    gigabytes).  Prints one JSON line with the per-launch device time."""
+    import torch
+    import bit_kv_cache_18_b200 as kvq
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    wl = PROFILE_WORKLOADS[args.profile]()
+    T0 = min(16384, wl.total_tokens)
+    nb0 = (T0 + 15) // 16
+    k = torch.from_numpy(wl.kv_rows(synth.TID_K, 0, T0).view(np.int16)).to(dev).view(torch.bfloat16)
+    v = torch.from_numpy(wl.kv_rows(synth.TID_V, 0, T0).view(np.int16)).to(dev).view(torch.bfloat16)
+    base = kvq.new_pool(nb0, wl.hkv, device=dev)
+    kvq.kvq_quantize_append(base, nb0, wl.hkv, k.reshape(T0, -1), v.reshape(T0, -1),
+                            torch.arange(T0, dtype=torch.int32, device=dev))
+    del k, v
+    pool = kvq.new_pool(wl.num_blocks, wl.hkv, device=dev)
+    seg = pool.view(wl.num_blocks, -1)
+    b0 = base.view(nb0, -1)
+    for s in range(0, wl.num_blocks, nb0):
+        n = min(nb0, wl.num_blocks - s)
+        seg[s:s + n].copy_(b0[:n])
+    q = torch.from_numpy(wl.query().view(np.int16)).to(dev).view(torch.bfloat16)
+    bt = torch.from_numpy(wl.block_table).to(dev)
+    lens = torch.from_numpy(wl.seq_lens).to(dev)
+    msl = int(wl.seq_lens.max())
+    out = torch.empty((wl.batch, wl.hq, 128), dtype=torch.bfloat16, device=dev)
+    ws = kvq.new_workspace(wl.num_blocks, wl.hkv, wl.batch, wl.hq, msl, device=dev)
+
+    def launch():
+        kvq.kvq_decode_attention(pool, wl.num_blocks, wl.hkv, q, bt, lens, msl, out, ws)
+
+    for _ in range(args.warmup):
+        launch()
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(args.steps):
+        launch()
+    e1.record(s)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / args.steps
+    nbytes = wl.total_tokens * wl.hkv * BYTES_PER_TOKEN_HEAD
+    peak, kind = measured_peaks()
+    gbs = nbytes / (us * 1e-6) / 1e9
+    print(json.dumps({"profile": args.profile, "launches": args.steps, "us_per_launch": us,
+                      "bytes_per_launch": nbytes, "gbs": gbs, "frac": gbs / peak, "peak_kind": kind,
+                      "device_status": kvq.kvq_last_device_status()}))
+    return 0
+
+
 # --------------------------------------------------------------------------- main
 
 def run_reference(args, world, rank):
@@ -341,9 +485,13 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", choices=sorted(PROFILE_WORKLOADS), default=None,
+                    help="time decode launches alone on one workload (1 GPU; for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.profile:
+        return profile_decode(args)
     world, rank, local = dist_env()
     if args.impl == "reference":
         return run_reference(args, world, rank)
@@ -365,7 +513,7 @@ def main():
         raise RuntimeError("device status set during warm-up")
 
     # timed region: K steps
-    with ClockSampler(local) as clocks:
+    with ClockSampler(local, device_uuid(torch, dev)) as clocks:
         ms = time_replays(torch, g_step, args.steps, barrier)
     ms_max, tokens = aggregate(dist, ms, args.steps * stepper.tokens_per_step(), dev)
     value = tokens / (ms_max * 1e-3)
@@ -411,7 +559,7 @@ def main():
                        "l2": "inputs larger than L2: 64 distinct 13.6 MB pools (872 MB) per step",
                        "parallelism": f"replicas x{world}"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": None,
+                         "frac": achieved / peak, "traffic": decode_traffic(),
                          "kernel": "decode", "peak_kind": peak_kind,
                          "us_per_launch": dms * 1e3, "bytes_per_launch": stepper.packed_bytes_per_decode,
                          "frac_of_8000": achieved / 8000.0},
