@@ -1,107 +1,161 @@
-// kvq_decode.cu -- decode attention over the packed paged cache.
+// kvq_decode.cu -- decode attention over the packed paged cache on the
+// fifth-generation tensor cores (tcgen05), warp-specialised, in exact
+// integer arithmetic.
 //
-// One CTA owns one (sequence b, kv head h, split of the context); its eight
-// warps take the split's blocks round robin.  The CTA
-//   1. rotates the G query heads of kv head h once, q~ = R q (in-smem FWHT),
-//      and sums them: zero points enter every score as Z_K,t * sum(q~);
-//   2. per warp, streams its 16-token segments (1664 B each) into a private
-//      ring of shared-memory stages with 16-byte cp.async copies, eight
-//      segments in flight, reading block-table entries 32 at a time one
-//      window ahead;
-//   3. per segment, computes q~.c_K for all G heads and 16 tokens on the
-//      tensor cores, folds the key scale and zero point into the score,
-//      updates a base-2 online softmax, folds the value scale into the
-//      probabilities, p' = p S_V, and accumulates p'.c_V on the tensor cores
-//      plus zeta += p Z_V;
-//   4. merges its warps, writes the split's partial (o~, m, l); the last CTA
-//      of (b, h) to take a ticket merges the splits and rotates the result
-//      back once, o = R o~ / l.
-// Scale folding at read time and the single rotations of the query and the
-// output follow the KVarN pipeline list ("KVarN vs TurboQuant", dothoosh.com,
-// fourth stage) and the definitions in include/kvq.h.  No CTA ever waits for
-// another.
+// One CTA owns one (sequence b, kv head h, split of the context) and walks
+// the split in chunks of 8 blocks = 128 tokens.  Two kinds of warps work on
+// different chunks at the same time and hand buffers to each other through
+// mbarrier rings:
+//   * loader warps 0-3 (thread t <-> token t of a chunk <-> TMEM lane t):
+//     read their two segments of each chunk with coalesced 16-byte loads
+//     straight into registers one chunk ahead (after an L2 prefetch of the
+//     segments five chunks ahead);
+//     spread the 4-bit key codes to one byte each into tensor memory (A of
+//     QK) and the 2-bit value codes to one byte each into shared memory (A of
+//     PV), and publish the per-token factors;
+//   * softmax warps 4-7 (thread t <-> token t of S, value position t of O):
+//     read a token's row of S, form the base-2 score of each of the G heads
+//       s_g = S_K,t c1 (S0 + S1/254 + S2/254^2) + Z_K,t sum(q~_g),
+//     the probability p = 2^(s_g - m_g) and P'_g = p S_V,t as a 30-bit fixed
+//     point whose four bytes are four u8 digit columns of the PV operand,
+//     and keep l_g = sum p and zeta_g = sum p Z_V in registers.  One lane of
+//     warp 4 issues every tensor-core instruction:
+//       QK:  S  = codes_K (128 tok x 128) . digits(q~)^T  (u8 x s8 -> s32)
+//       PV:  O += codes_V^T (128 pos x 128 tok) . digits(P') (u8 x u8 -> s32)
+//     (tcgen05.mma, M = 128, N = 32): the QK of chunk c+2 as soon as the four
+//     warps have read S of chunk c, the PV of chunk c once its P' is written.
+// Before the scan the softmax warps rotate the G query heads once (warp
+// FWHT, softmax scale times log2(e) folded in) and write q~ as three signed
+// 8-bit digits, q~/c1 = Q0 + Q1/254 + Q2/254^2 with c1 = max|q~|/127.  After
+// it they convert O to fp32 (o~ = sum P' c_V + zeta), write the split's
+// partial (o~, m, l); the last CTA of (b, h) to take a ticket merges the
+// splits and rotates back once, o = R o~ / l.  Scale folding at read time and
+// the single rotations of the query and the output follow the KVarN pipeline
+// list ("KVarN vs TurboQuant", dothoosh.com, fourth stage) and the
+// definitions in include/kvq.h.  No CTA ever waits for another.
 //
-// Tensor-core mapping (mma.sync m16n8k16, fp16 in, fp32 accumulate).  Rows
-// m = 0..7 hold the G <= 8 query heads, rows 8..15 the same heads again as the
-// low half of a two-term fp16 split (x = hi + lo, hi = fp16(x), lo =
-// fp16(x - hi)), so the split that keeps 22 bits of the rotated query and of
-// p S_V costs no extra instruction: it fills rows a single head group would
-// leave empty.  QK: A = q~ (16 x 16 dims), B = codes (16 dims x 8 tokens).
-// PV: A = p' (16 x 16 tokens), B = codes (16 tokens x 8 dims).  The QK
-// accumulator layout is exactly the PV A-operand layout, so probabilities
-// never leave registers.
+// Why integers: a tcgen05.mma with M = 128 costs about as much for N = 32
+// as for N = 16, so each one should carry as much work as it can: u8 codes
+// times 8-bit digits give K = 32 per instruction, the digits of q~ and P'
+// fill the N columns a GQA group of 8 heads would leave empty, spreading a
+// packed word to bytes is one or two logic operations per four codes, and
+// every product and sum is exact.  The only roundings are the digit
+// expansion of q~ (about 2^-22 of max|q~|) and the fixed point of P'
+// (a step of 2^-27, with P' < 2^3).  The step must be that fine: tokens
+// whose P' rounds to zero drop their S_V c_V but keep their p Z_V and p, and
+// since codes are never negative that loss is a bias, not noise.
 //
-// Code unpacking.  A 4-bit or 2-bit code masked in place into the mantissa of
-// fp16 1024.0 (0x6400) and the bias then subtracted (one packed fp16 sub per
-// two codes) gives the code, times a power of two fixed by its bit position,
-// as an exact normal fp16 number.  The power of two of each operand slot is
-// known statically and folded into the query fragment (keys) or into the
-// final output scaling (values).  Leaving the codes as fp16 subnormals would
-// save the subtraction, but measured on B200 that loses accuracy in the
-// tensor-core sums (decode error about 2e-3 instead of 3e-5).
+// Lazy running max.  m_g tracks the largest s_g + E_t, E_t the exponent
+// bound of S_V,t (S_V,t < 2^E_t, floored at -24), and only moves when some
+// token has s_g + E_t > m_g + 2.9: then P' < 2^3 always fits the fixed
+// point.  A move is decided by one vote of the softmax warps per chunk and is
+// rare; the integer accumulator is then folded into fp32 registers with the
+// factor 2^(m_old - m_new) and restarted.  It is also restarted every 128
+// chunks, which keeps every s32 sum below 2^31.
+//
+// Code order.  The byte spreading permutes the 128 positions of a row
+// (keys: position 8i + 4h + j holds dim 8i + 2j + h; values: position
+// 16i + 4k + j holds dim 16i + 4j + k, times 4^k).  The query digits are
+// written in the key order, so S is exact, and the output rows are put back
+// in dim order, and divided by 4^k, when O is read.
 #include <math_constants.h>
+
+#include <type_traits>
 
 #include "kvq_internal.cuh"
 
 namespace kvq {
 namespace {
 
-#ifndef KVQ_DECODE_WARPS
-#define KVQ_DECODE_WARPS 8
-#endif
-constexpr int kDecodeWarps = KVQ_DECODE_WARPS;          // warps per CTA
-constexpr int kStages = kDecodeWarps == 8 ? 6 : 8;      // segments in flight per warp
-constexpr int kMinCtasPerSm = kDecodeWarps == 8 ? 2 : 3;
-constexpr float kRescaleLog2 = 8.0f;  // lazy running-max threshold (log2 units)
-constexpr int kMaxSplits = 64;      // the plan never cuts a sequence finer
+constexpr int kLoadWarps = 4;                          // warps 0-3
+constexpr int kSoftWarps = 4;                          // warps 4-7
+constexpr int kMmaWarp = kLoadWarps + kSoftWarps;        // warp 8: tensor memory owner, MMA issue
+constexpr int kThreads = 32 * (kMmaWarp + 1);             // 288
+constexpr int kChunkBlocks = 8;
+constexpr int kChunkTokens = kChunkBlocks * kBlockSize;  // 128
+constexpr int kMaxSplits = 64;     // the plan never cuts a sequence finer
+constexpr int kNS = 2;             // score buffers in tensor memory
+constexpr int kNV = 3;             // key-code buffers in tensor memory; value / P' / factor buffers in smem
+constexpr int kFlushChunks = 128;  // integer accumulator restarted at least this often
+constexpr float kFix = 134217728.0f;  // P'_int = rne(P' 2^27) < 2^30
+constexpr float kFixInv = 1.0f / 134217728.0f;
+constexpr float kTrigger = 2.9f;    // move the max when s + E > m + kTrigger
+// The running max before any token: far below every score (|s| stays far
+// below 2^20 for fp16 factors), so the first token moves it and
+// 2^(kNoMax - m) = 0, yet finite, so that s - m + m loses only the bits that
+// the lazy max can spare.
+constexpr float kNoMax = -1048576.0f;
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColA = 0;    // key codes of chunk c: kColA + 32 (c % 3)
+constexpr uint32_t kColS = 96;   // S of chunk c: kColS + 32 (c % 2)
+constexpr uint32_t kColO = 160;  // O accumulator
+constexpr uint32_t kWaitLimit = 1u << 22;
+constexpr int kBarSoftSync = 1;  // named barrier of the 128 softmax threads
+constexpr int kBarSoftVote = 2;  // named barrier for their vote
 
-template <int W>
-struct __align__(128) DecodeSmem {
-  uint8_t stage[W][kStages][kSegBytes];  // per-warp segment rings (then merge scratch)
-  uint64_t bar[W][kStages];              // one mbarrier per stage
-  uint4 qfrag[8][32];                    // QK A fragments, [k-step][lane]
-  float q[8][kHeadDim];                  // rotated query rows (then the merged output)
-  float qsum[8];
-  float wm[W][8];
-  float wl[W][8];
-  float wf[8][W];  // per head: weight of each warp in the CTA merge
-  float hm[8];
-  float hl[8];
+// Instruction descriptors (kind::i8, D = s32, M = 128, N = 32):
+//   QK: A = u8 key codes (TMEM, K-major), B = s8 query digits (smem, K-major)
+//   PV: A = u8 value codes (smem, MN-major), B = u8 P' digits (smem, MN-major)
+constexpr uint32_t kIdescQK = (2u << 4) | (0u << 7) | (1u << 10) | ((32u >> 3) << 17) | ((128u >> 4) << 24);
+constexpr uint32_t kIdescPV =
+    (2u << 4) | (0u << 7) | (0u << 10) | (1u << 15) | (1u << 16) | ((32u >> 3) << 17) | ((128u >> 4) << 24);
+
+// Shared memory.  Operand tiles use the no-swizzle canonical layouts of
+// 8-row x 16-byte core matrices:
+//   vt (A of PV, MN-major): byte (tok, pos) at (tok/8)*1024 + (pos/16)*128 + (tok%8)*16 + pos%16
+//   pm (B of PV, MN-major): byte (tok, n)   at (tok/8)*256  + (n/16)*128   + (tok%8)*16 + n%16
+//   qb (B of QK, K-major):  byte (n, pos)   at (pos/16)*512 + (n/8)*128    + (n%8)*16   + pos%16
+// S column n = 8j + g holds digit j of head g (rows 24..31 of qb are zero);
+// P' and O column n = 4g + j hold byte j of head g.
+struct __align__(1024) Smem {
+  uint8_t vt[kNV][kChunkTokens * kHeadDim];  // 3 x 16 KB
+  uint8_t pm[kNV][kChunkTokens * 32];        // 3 x 4 KB
+  uint8_t qb[32 * kHeadDim];                 // 4 KB
+  float meta[kNV][4][kChunkTokens];          // per token: S_K c1, Z_K, S_V 2^27 (< 0: no token), Z_V
+  float obuf[8][kHeadDim];                   // o~ (epilogue)
+  float2 hq[8];                              // per head: sum(q~), max|q~|
+  float red[kSoftWarps][8][2];               // cross-warp reductions
+  float hm[8], hl[8], hz[8];
+  uint64_t kv_ready[kNV];  // loaders -> MMA warp, softmax: codes and factors of chunk c written
+  uint64_t qk_done[kNS];   // QK(c) complete -> softmax: S of chunk c ready (and PV(c-3) complete)
+  uint64_t s_free[kNS];    // softmax -> MMA warp: S of chunk c read
+  uint64_t p_ready[kNV];   // softmax -> MMA warp: P' of chunk c written
+  uint64_t pv_done[kNV];   // PV(c) complete -> loaders, softmax (and QK(c+1) complete)
+  uint64_t fin;            // every MMA issued is complete
+  uint32_t tmem_base;
+  int fresh[kNV];          // the PV of chunk c starts the accumulator afresh
   int is_last;
+  int abort;              // a wait ran out: every other wait gives up at once
+};
+constexpr int kSmemBytes = static_cast<int>((sizeof(Smem) + 1023) / 1024 * 1024);
+static_assert(kSmemBytes <= 113 * 1024, "two CTAs per SM");
+
+// Position in a ring of three buffers and the parity of its current use.
+struct Ring3 {
+  int i;
+  uint32_t ph;
+  __device__ __forceinline__ void next() {
+    if (++i == 3) {
+      i = 0;
+      ph ^= 1u;
+    }
+  }
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
-// ---- TMA bulk copies completed on mbarriers ---------------------------------
+// sm_100 shared-memory matrix descriptor: start address, leading and stride
+// byte offsets in 16-byte units, version 1, no swizzle.
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
 }
-// One 1664-byte segment, global -> shared, by the TMA engine, issued by the
-// lanes whose predicate is set (one per warp) without a branch: an
-// async-proxy fence (orders earlier reads of the slot), the barrier's
-// expected byte count, and the bulk copy that completes it.
-__device__ __forceinline__ void bulk_load_segment_if(bool pred, uint8_t* dst, const uint8_t* src, uint64_t* bar) {
-  asm volatile(
-      "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n"
-      "@p fence.proxy.async.shared::cta;\n"
-      "@p mbarrier.arrive.expect_tx.shared::cta.b64 _, [%2], %3;\n"
-      "@p cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %3, [%2]; }" ::"r"(
-          smem_u32(dst)),
-      "l"(src), "r"(smem_u32(bar)), "r"(kSegBytes), "r"(static_cast<uint32_t>(pred))
-      : "memory");
-}
-// One 1664-byte segment, global -> shared, by the TMA engine; the barrier
-// expects the bytes and completes its phase when they have landed.
-__device__ __forceinline__ void bulk_load_segment(uint8_t* dst, const uint8_t* src, uint64_t* bar) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-               "r"(kSegBytes)
-               : "memory");
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(dst)),
-      "l"(src), "r"(kSegBytes), "r"(smem_u32(bar))
-      : "memory");
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("{ .reg .b64 st; mbarrier.arrive.shared::cta.b64 st, [%0]; }" ::"r"(smem_u32(bar)) : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t done;
@@ -112,51 +166,111 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return done != 0;
 }
-// Bounded, warp-uniform wait for a barrier phase (every lane polls; the warp
-// leaves together): false if the copy never arrived, in which case the caller
-// records KVQ_ERR_DEVICE_TIMEOUT instead of hanging.
-constexpr uint32_t kWaitLimit = 1u << 22;
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  for (uint32_t it = 0; it < kWaitLimit; ++it)
+// Bounded, warp-uniform wait for a barrier phase.  False if it never came or
+// another warp already gave up (then every later wait returns at once and
+// the kernel runs to its end on void data, which it reports).
+__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  for (uint32_t it = 0; it < kWaitLimit; ++it) {
     if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+    if ((it & 15u) == 15u && __any_sync(0xffffffffu, *abort != 0)) return false;
+  }
+  *abort = 1;
   return false;
 }
-
-__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+  return mbar_wait_slow(bar, parity, abort);
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void async_proxy_fence() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void soft_sync() { asm volatile("bar.sync %0, %1;" ::"n"(kBarSoftSync), "n"(128) : "memory"); }
+__device__ __forceinline__ bool soft_vote_any(bool x) {
+  uint32_t r;
+  asm volatile(
+      "{ .reg .pred p, q; setp.ne.u32 p, %1, 0; bar.red.or.pred q, %2, %3, p; selp.u32 %0, 1, 0, q; }"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(x)), "n"(kBarSoftVote), "n"(128)
+      : "memory");
+  return r != 0;
 }
 
-__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
-  const __half2 h = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&h);
+__device__ __forceinline__ void mma_qk(uint32_t d, uint32_t a, uint64_t bdesc, bool acc) {
+  asm volatile(
+      "{ .reg .pred p; setp.ne.b32 p, %3, 0;\n"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %4, p; }" ::"r"(d),
+      "r"(a), "l"(bdesc), "r"(static_cast<uint32_t>(acc)), "r"(kIdescQK)
+      : "memory");
+}
+__device__ __forceinline__ void mma_pv(uint32_t d, uint64_t adesc, uint64_t bdesc, bool acc) {
+  asm volatile(
+      "{ .reg .pred p; setp.ne.b32 p, %3, 0;\n"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %4, p; }" ::"r"(d),
+      "l"(adesc), "l"(bdesc), "r"(static_cast<uint32_t>(acc)), "r"(kIdescPV)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
 }
 
-// Two-term fp16 split of a pair: hi = fp16(x), lo = fp16(x - hi).
-__device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& hi, uint32_t& lo) {
-  const __half2 h = __floats2half2_rn(x0, x1);
-  const float2 f = __half22float2(h);
-  hi = *reinterpret_cast<const uint32_t*>(&h);
-  lo = pack_half2(x0 - f.x, x1 - f.y);
+// 16 lanes x 256 bits, 4 repetitions: registers 4j, 4j+1 go to lane
+// (addr lane) + t/4, columns 8j + 2(t%4) + {0, 1}; registers 4j+2, 4j+3 to
+// lane + 8 + t/4, same columns (t = thread in the warp).
+__device__ __forceinline__ void tmem_st16x256(uint32_t addr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x256b.x4.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          addr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t addr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(addr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld8(uint32_t addr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(addr)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ uint4 ldg16(const uint8_t* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
+}
+__device__ __forceinline__ uint2 ldg8(const uint8_t* p) {
+  uint2 r;
+  asm volatile("ld.global.nc.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+  return r;
+}
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
-constexpr uint32_t kBias = 0x64006400u;
-// (x & mask) | bias in one LOP3 (mask an immediate, bias a register), then
-// the bias subtracted: the masked codes as exact fp16 numbers.
-template <uint32_t kMask>
-__device__ __forceinline__ uint32_t codes_f16(uint32_t x, uint32_t bias) {
-  uint32_t t, d;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(t) : "r"(x), "n"(kMask), "r"(bias));
-  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(t), "r"(bias));
-  return d;
+__device__ __forceinline__ float ex2(float x) {  // 2^x (MUFU.EX2); ex2(-inf) = 0
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
-
-
-__device__ __forceinline__ float2 half2_at(const uint8_t* p) {
-  return __half22float2(*reinterpret_cast<const __half2*>(p));
+__device__ __forceinline__ float h2f(uint32_t bits) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(bits)));
+}
+// Exact int -> float for |v| < 2^22 without the conversion unit: the
+// integer added to the bits of 1.5 * 2^23 lands in the mantissa.
+__device__ __forceinline__ float small_i2f(uint32_t v) {
+  return __uint_as_float(v + 0x4B400000u) - 12582912.0f;
 }
 
 // Walsh-Hadamard transform of one 128-vector held by a warp, element
@@ -182,27 +296,48 @@ __device__ __forceinline__ void fwht_warp(float (&x)[4], int lane, float scale) 
   for (int k = 0; k < 4; ++k) x[k] *= f;
 }
 
-__device__ __forceinline__ float ex2(float x) {  // 2^x (MUFU.EX2); ex2(-inf) = 0
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
+// Position of dim d in a spread key row, and dim of position p in a spread
+// value row (the byte-spreading orders of the file comment).
+__device__ __forceinline__ int key_pos_of_dim(int d) {
+  return ((d >> 3) & 3) << 5 | (d >> 5) << 3 | (d & 1) << 2 | ((d >> 1) & 3);
 }
+__device__ __forceinline__ int value_dim_of_pos(int p) { return (p & ~15) | ((p & 3) << 2) | ((p >> 2) & 3); }
 
-template <int G, int W>
-__global__ void __launch_bounds__(W * 32, kMinCtasPerSm) decode_kernel(DecodeArgs a) {
-  constexpr int kThreads = W * 32;
-  extern __shared__ __align__(128) uint8_t smem_raw[];
-  DecodeSmem<W>& sm = *reinterpret_cast<DecodeSmem<W>*>(smem_raw);
+// One lane's share of a loader warp's two segments of one chunk, in
+// registers (coalesced 16-byte pieces; segment s = 0, 1):
+//   k[2s], k[2s+1]: key-code bytes 16 lane + [0, 16) and 512 + 16 lane + [0, 16)
+//                   (rows lane/4 and 8 + lane/4, dims 32 (lane%4) + [0, 32));
+//   v[s]:           value-code bytes 16 lane + [0, 16) (row lane/2, dims 64 (lane%2) + [0, 64));
+//   m:              factor bytes 8 (lane%16) + [0, 8) of segment lane/16
+//                   (four fp16 of kind (lane/4)%4 for rows 4 (lane%4) + [0, 4)).
+struct Stage {
+  uint4 k[4];
+  uint4 v[2];
+  uint2 m;
+  uint32_t ok;  // bit s: segment s is inside the split and the pool
+};
+
+// Bounded wait that ignores the abort flag: the issuer's last wait for its
+// own MMAs, so tensor memory is never released under a running MMA.
+__device__ __forceinline__ bool mbar_wait_final(uint64_t* bar, uint32_t parity) {
+  for (uint32_t it = 0; it < kWaitLimit; ++it)
+    if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+  return false;
+}
+template <int G>
+__global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
+  volatile int* abort = &sm.abort;
   const int split = blockIdx.x;
   const int h = blockIdx.y;
   const int b = blockIdx.z;
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int g = lane >> 2;  // fragment row group: query head g (hi), g+8 (lo)
-  const int c = lane & 3;   // fragment column pair
+  const bool is_loader = warp < kLoadWarps;
 
-  // effective length of this sequence
+  // ---- the split: blocks [blk0, blk1) of sequence b, in chunks of 8 -------
   int L = a.seq_lens[b];
   if (L < 0 || L > a.max_seq_len || L > a.max_blocks_per_seq * kBlockSize) {
     if (tid == 0) record_status(a.status, KVQ_ERR_OUT_OF_RANGE);
@@ -213,300 +348,447 @@ __global__ void __launch_bounds__(W * 32, kMinCtasPerSm) decode_kernel(DecodeArg
   const int nb = (L + kBlockSize - 1) / kBlockSize;
   const int blk0 = split * a.blocks_per_split;
   const int blk1 = min(nb, blk0 + a.blocks_per_split);
-  // this warp's blocks: blk0 + warp + W*j, j = 0 .. nmine-1
-  const int nmine = blk1 > blk0 + warp ? (blk1 - blk0 - warp + W - 1) / W : 0;
-  const int32_t* bt_row = a.block_table + static_cast<int64_t>(b) * a.max_blocks_per_seq + blk0 + warp;
+  const int nchunks = blk1 > blk0 ? (blk1 - blk0 + kChunkBlocks - 1) / kChunkBlocks : 0;
+  bool bad = false;      // a wait ran out: the results are void, the control flow is kept
+  bool bad_blk = false;  // a block-table entry outside the pool (its tokens are skipped)
+
+  // loader warp w owns blocks 2w and 2w+1 of every chunk (tokens 32w ..
+  // 32w + 31 = TMEM lanes of its quarter); lanes 0 and 1 keep the block
+  // ids of segment lane & 1
+  const int32_t* bt_row = a.block_table + static_cast<int64_t>(b) * a.max_blocks_per_seq;
   const uint8_t* pool_h = a.pool + static_cast<int64_t>(h) * kSegBytes;
   const int64_t pstride = static_cast<int64_t>(a.num_kv_heads) * kSegBytes;
+  const int mseg = lane >> 4;  // segment of my factor bytes
 
-  // ---- 1. block-table windows (lane l holds the entry of local block 32k+l)
-  //      and the first kStages segments in flight (lane 0 drives the TMA)
-  int32_t win0 = lane < nmine ? bt_row[W * lane] : -1;
-  int32_t win1 = 32 + lane < nmine ? bt_row[W * (32 + lane)] : -1;
-  int wbase = 0;
-  if (lane == 0) {
+  // physical block of segment lane & 1 of my warp in chunk c (-1: none)
+  auto bid_of = [&](int c) -> int32_t {
+    const int blk = blk0 + kChunkBlocks * c + 2 * warp + (lane & 1);
+    return blk < blk1 ? __ldg(bt_row + blk) : -1;
+  };
+  // my share of chunk c, segments in blocks p0, p1; blocks outside the split
+  // or the pool read block 0 and are marked absent
+  auto load_stage = [&](Stage& s, int c, int32_t p0, int32_t p1) {
+    const int blk = blk0 + kChunkBlocks * c + 2 * warp;
+    const bool live0 = blk < blk1, live1 = blk + 1 < blk1;
+    const bool ok0 = live0 && p0 >= 0 && p0 < a.num_blocks;
+    const bool ok1 = live1 && p1 >= 0 && p1 < a.num_blocks;
+    bad_blk |= (live0 && !ok0) || (live1 && !ok1);
+    s.ok = (ok0 ? 1u : 0u) | (ok1 ? 2u : 0u);
+    if (a.num_blocks > 0) {  // (an empty pool has no block 0)
+      const uint8_t* g0 = pool_h + static_cast<int64_t>(ok0 ? p0 : 0) * pstride;
+      const uint8_t* g1 = pool_h + static_cast<int64_t>(ok1 ? p1 : 0) * pstride;
+      s.k[0] = ldg16(g0 + kOffK + 16 * lane);
+      s.k[1] = ldg16(g0 + kOffK + 512 + 16 * lane);
+      s.k[2] = ldg16(g1 + kOffK + 16 * lane);
+      s.k[3] = ldg16(g1 + kOffK + 512 + 16 * lane);
+      s.v[0] = ldg16(g0 + kOffV + 16 * lane);
+      s.v[1] = ldg16(g1 + kOffV + 16 * lane);
+      s.m = ldg8((mseg ? g1 : g0) + kOffSK + 8 * (lane & 15));
+    }
+  };
+  auto prefetch_seg = [&](int32_t p) {
+    if (lane < 2 && p >= 0 && p < a.num_blocks) prefetch_l2(pool_h + static_cast<int64_t>(p) * pstride, kSegBytes);
+  };
+
+  // ---- 0. set-up: barriers and tensor memory; first loads; query digits ----
+  Stage st{};
+  int32_t bq[6];  // loaders: block ids of chunks c+1 .. c+6 at the start of iteration c
+  if (is_loader) {
+    const int32_t p0 = bid_of(0);
 #pragma unroll
-    for (int s2 = 0; s2 < kStages; ++s2) mbar_init(&sm.bar[warp][s2], 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  __syncwarp();
-  uint32_t valid_bits = 0;  // bit s: a copy into slot s is in flight / landed
-  uint32_t phase_bits = 0;  // bit s: parity of slot s's next completion
+    for (int i = 0; i < 6; ++i) bq[i] = bid_of(1 + i);
+    load_stage(st, 0, __shfl_sync(0xffffffffu, p0, 0), __shfl_sync(0xffffffffu, p0, 1));
 #pragma unroll
-  for (int i = 0; i < kStages; ++i) {
-    const int32_t p = __shfl_sync(0xffffffffu, win0, i);
-    if (i < nmine) {
-      if (p >= 0 && p < a.num_blocks) {
-        if (lane == 0) bulk_load_segment(sm.stage[warp][i], pool_h + p * pstride, &sm.bar[warp][i]);
-        valid_bits |= 1u << i;
-      } else if (lane == 0) {
-        record_status(a.status, KVQ_ERR_OUT_OF_RANGE);
+    for (int i = 0; i < 4; ++i) prefetch_seg(bq[i]);
+  } else if (warp == kMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sm.tmem_base)),
+                 "n"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    if (lane == 0) {
+#pragma unroll
+      for (int i = 0; i < kNV; ++i) {
+        mbar_init(&sm.kv_ready[i], 32 * kLoadWarps);
+        mbar_init(&sm.p_ready[i], 32 * kSoftWarps);
+        mbar_init(&sm.pv_done[i], 1);
       }
-    }
-  }
-
-  // ---- 2. rotate the query (overlaps the copies in flight): warp w < 8
-  //      owns query head w of this kv head.  tau*log2(e) is folded into q~,
-  //      so scores come out of the MMA already in base-2 logits.
-  for (int gg = warp; gg < 8; gg += W) {
-    float x[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    if (gg < G) {
-      const int64_t q0 = (static_cast<int64_t>(b) * a.num_q_heads + h * G + gg) * kHeadDim;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) x[k] = load_as_f32(a.q, a.q_dtype, q0 + lane + 32 * k);
-    }
-    fwht_warp(x, lane, a.scale_log2);
-    float s4 = (x[0] + x[1]) + (x[2] + x[3]);
-#pragma unroll
-    for (int o = 16; o; o >>= 1) s4 += __shfl_xor_sync(0xffffffffu, s4, o);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) sm.q[gg][lane + 32 * k] = x[k];
-    if (lane == 0) sm.qsum[gg] = s4;
-  }
-  __syncthreads();
-
-  // QK A fragments in smem, [k-step][lane], built by warp kk for its k-step
-  // and read back with one 16-byte load per k-step.  k-step kk reads word
-  // w = 4c + kk/2 of a key row (dims 8w..8w+7).  Slots (2c, 2c+1) take dims
-  // (8w+e, 8w+e+4) and slots (2c+8, 2c+9) take (8w+e+1, 8w+e+5), e = 0 for
-  // even kk and 2 for odd kk; the second pair's codes sit 4 bits higher (x16),
-  // so its q is /16.
-  for (int kk = warp; kk < 8; kk += W) {
-    const int w = 4 * c + (kk >> 1);
-    const int e = (kk & 1) ? 2 : 0;
-    const float* qr = sm.q[g];
-    uint4 f;
-    split_pair(qr[8 * w + e], qr[8 * w + e + 4], f.x, f.y);
-    split_pair(qr[8 * w + e + 1] * 0.0625f, qr[8 * w + e + 5] * 0.0625f, f.z, f.w);
-    sm.qfrag[kk][lane] = f;
-  }
-  const float zq = sm.qsum[g];
-  __syncthreads();
-
-  // PV B operand through ldmatrix.trans: 8x8 tiles of 16-bit elements of the
-  // value rows (tokens x 8 crumbs).  Tile i covers tokens 8(i/2)..8(i/2)+7 and
-  // dims 64(i%2)..64(i%2)+63; after the transpose lane (g, c) holds, for
-  // tokens (2c, 2c+1) of the tile, the 16 bits of dims 64h+8g .. 64h+8g+7.
-  // n-tile (h, k) takes crumb k of those 16 bits, i.e. column g is dim
-  // 64h + 8g + k.  Crumbs 0..4 are masked in place (code times 4^k), crumbs
-  // 5..7 after a 10-bit shift (code times 4^(k-5)).
-  const int ld_tok = ((lane >> 4) << 3) + (lane & 7);
-  const int ld_half = (lane >> 3) & 1;
-
-  uint32_t bias;
-  asm volatile("mov.b32 %0, %1;" : "=r"(bias) : "n"(kBias));
-
-  float o[16][4];
-#pragma unroll
-  for (int nt = 0; nt < 16; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.0f;
-  float m_ref = -CUDART_INF_F;
-  float l_part = 0.0f, z_part = 0.0f;
-
-  // ---- 3. the paged scan
-  bool timed_out = false;
-  int slot = 0;
-#pragma unroll 1
-  for (int i = 0; i < nmine; ++i, slot = (slot + 1 == kStages) ? 0 : slot + 1) {
-    if (valid_bits & (1u << slot)) {
-      if (!mbar_wait(&sm.bar[warp][slot], (phase_bits >> slot) & 1u)) {
-        timed_out = true;
-        break;
+      for (int i = 0; i < kNS; ++i) {
+        mbar_init(&sm.qk_done[i], 1);
+        mbar_init(&sm.s_free[i], 32 * kSoftWarps);
       }
-      phase_bits ^= 1u << slot;
+      mbar_init(&sm.fin, 1);
+      sm.abort = 0;
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (valid_bits & (1u << slot)) {
-      const uint8_t* sg = sm.stage[warp][slot];
-      const int ntok = min(kBlockSize, L - (blk0 + warp + W * i) * kBlockSize);
-
-      // scores: n-tile j holds tokens 8j..8j+7, column g is token 8j+g
-      float sacc[2][2][4];  // [n-tile][chain: even / odd k-steps]
+  } else {
+    // rotate the G query heads (warp sw: heads sw, sw + 4), then write their
+    // digits with one c1 for all heads
+    const int sw = warp - kLoadWarps;
+    const int stok = tid - 32 * kLoadWarps;
+    reinterpret_cast<uint4*>(sm.qb)[stok] = make_uint4(0, 0, 0, 0);
+    reinterpret_cast<uint4*>(sm.qb)[stok + 128] = make_uint4(0, 0, 0, 0);
+    float x[2][4];
 #pragma unroll
-      for (int j = 0; j < 2; ++j)
+    for (int i = 0; i < 2; ++i) {
+      const int g = sw + 4 * i;
+      if (g < G) {
+        const int64_t q0 = (static_cast<int64_t>(b) * a.num_q_heads + h * G + g) * kHeadDim;
 #pragma unroll
-        for (int ch = 0; ch < 2; ++ch) sacc[j][ch][0] = sacc[j][ch][1] = sacc[j][ch][2] = sacc[j][ch][3] = 0.0f;
-      const uint4 kw0 = *reinterpret_cast<const uint4*>(sg + kOffK + g * kKRowBytes + 16 * c);
-      const uint4 kw1 = *reinterpret_cast<const uint4*>(sg + kOffK + (8 + g) * kKRowBytes + 16 * c);
-      const uint32_t words[2][4] = {{kw0.x, kw0.y, kw0.z, kw0.w}, {kw1.x, kw1.y, kw1.z, kw1.w}};
+        for (int k = 0; k < 4; ++k) x[i][k] = load_as_f32(a.q, a.q_dtype, q0 + lane + 32 * k);
+        fwht_warp(x[i], lane, a.scale_log2);
+        float s4 = (x[i][0] + x[i][1]) + (x[i][2] + x[i][3]);
+        float mx = fmaxf(fmaxf(fabsf(x[i][0]), fabsf(x[i][1])), fmaxf(fabsf(x[i][2]), fabsf(x[i][3])));
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint4 f = sm.qfrag[kk][lane];
-        const uint32_t qa[4] = {f.x, f.y, f.z, f.w};
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const uint32_t w = (kk & 1) ? (words[j][kk >> 1] >> 8) : words[j][kk >> 1];
-          mma16816(sacc[j][kk & 1], qa, codes_f16<0x000F000Fu>(w, bias), codes_f16<0x00F000F0u>(w, bias));
+        for (int o = 16; o; o >>= 1) {
+          s4 += __shfl_xor_sync(0xffffffffu, s4, o);
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         }
+        if (lane == 0) sm.hq[g] = make_float2(s4, mx);
       }
-      // fold S_K, Z_K: s = tau log2e (S_K (hi + lo) + Z_K sum q~)
-      float sc[4];
+    }
+    soft_sync();
+    float mx = 0.0f;
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const float2 sk = half2_at(sg + kOffSK + 4 * (4 * j + c));
-        const float2 zk = half2_at(sg + kOffZK + 4 * (4 * j + c));
-        const float d0 = (sacc[j][0][0] + sacc[j][1][0]) + (sacc[j][0][2] + sacc[j][1][2]);
-        const float d1 = (sacc[j][0][1] + sacc[j][1][1]) + (sacc[j][0][3] + sacc[j][1][3]);
-        sc[2 * j] = fmaf(sk.x, d0, zk.x * zq);
-        sc[2 * j + 1] = fmaf(sk.y, d1, zk.y * zq);
-      }
-      if (ntok < kBlockSize) {  // the last block of a sequence: drop the empty rows
+    for (int g = 0; g < G; ++g) mx = fmaxf(mx, sm.hq[g].y);
+    const float inv = mx > 0.0f ? 127.0f / mx : 0.0f;
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          if (8 * (q >> 1) + 2 * c + (q & 1) >= ntok) sc[q] = -CUDART_INF_F;
-      }
-      // Lazy running max: rescale only when a score exceeds the reference by
-      // more than 8 (base 2).  Probabilities are taken relative to m_ref + 8,
-      // p = 2^(s - m_ref - 8) <= 1, so p' = p S_V <= S_V always fits fp16;
-      // o, l and zeta all carry the same factor, which the final o / l
-      // cancels.  One warp vote decides; the head max (shuffles) and the
-      // rescale run only when some lane needs them.
-      const float mloc = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
-      if (__any_sync(0xffffffffu, mloc > m_ref + kRescaleLog2)) {
-        float mx = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        if (mx > m_ref + kRescaleLog2) {
-          const float alpha = m_ref == -CUDART_INF_F ? 0.0f : ex2(m_ref - mx);
+    for (int i = 0; i < 2; ++i) {
+      const int g = sw + 4 * i;
+      if (g < G) {
 #pragma unroll
-          for (int nt = 0; nt < 16; ++nt) {
-            o[nt][0] *= alpha;
-            o[nt][1] *= alpha;
-            o[nt][2] *= alpha;
-            o[nt][3] *= alpha;
+        for (int k = 0; k < 4; ++k) {
+          const int pos = key_pos_of_dim(lane + 32 * k);
+          const float y = x[i][k] * inv;
+          const float q1 = rintf(y);
+          const float r1 = (y - q1) * 254.0f;
+          const float q2 = rintf(r1);
+          const float q3 = rintf((r1 - q2) * 254.0f);
+          const float dig[3] = {q1, q2, q3};
+#pragma unroll
+          for (int j = 0; j < 3; ++j) {
+            const int n = 8 * j + g;
+            const int v = max(-127, min(127, static_cast<int>(dig[j])));
+            sm.qb[(pos >> 4) * 512 + (n >> 3) * 128 + (n & 7) * 16 + (pos & 15)] = static_cast<uint8_t>(v & 0xFF);
           }
-          l_part *= alpha;
-          z_part *= alpha;
-          m_ref = mx;
         }
       }
-      const float m8 = m_ref + kRescaleLog2;
-      // probabilities with the value scale folded in: p' = p S_V
-      float pv[4];
+    }
+    async_proxy_fence();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = sm.tmem_base;
+  float c1 = 0.0f;
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        float2 sv = half2_at(sg + kOffSV + 4 * (4 * j + c));
-        float2 zv = half2_at(sg + kOffZV + 4 * (4 * j + c));
-        if (ntok < kBlockSize) {  // rows past the end may hold NaN metadata
-          if (8 * j + 2 * c >= ntok) sv.x = zv.x = 0.0f;
-          if (8 * j + 2 * c + 1 >= ntok) sv.y = zv.y = 0.0f;
-        }
-        const float p0 = ex2(sc[2 * j] - m8);
-        const float p1 = ex2(sc[2 * j + 1] - m8);
-        l_part += p0 + p1;
-        z_part = fmaf(p0, zv.x, fmaf(p1, zv.y, z_part));
-        pv[2 * j] = p0 * sv.x;
-        pv[2 * j + 1] = p1 * sv.y;
-      }
-      uint32_t pa[4];
-      split_pair(pv[0], pv[1], pa[0], pa[1]);
-      split_pair(pv[2], pv[3], pa[2], pa[3]);
+  for (int g = 0; g < G; ++g) c1 = fmaxf(c1, sm.hq[g].y);
+  c1 *= 1.0f / 127.0f;
 
-      // p'.c_V: one ldmatrix.x4.trans gives this lane's value operands
-      uint32_t vr[4];
+  // ---- 1. the paged scan ------------------------------------------------------
+  if (is_loader) {
+    const uint32_t my_lanes = tbase + (static_cast<uint32_t>(warp * 32) << 16);
+    // my value rows: row lane/2 of segment s, dims 64 (lane%2) + [0, 64)
+    uint32_t my_vt[2];
+#pragma unroll
+    for (int sg = 0; sg < 2; ++sg) {
+      const int tok = 32 * warp + 16 * sg + (lane >> 1);
+      my_vt[sg] = smem_u32(sm.vt[0]) + (tok >> 3) * 1024 + (lane & 1) * 512 + (tok & 7) * 16;
+    }
+    const int mrow0 = 4 * (lane & 3);    // my factor rows mrow0 .. mrow0+3 of segment mseg
+    const int mkind = (lane >> 2) & 3;  // S_K, Z_K, S_V, Z_V
+    const float mscale = mkind == 2 ? kFix : 1.0f;
+    const float mnone = mkind == 2 ? -1.0f : 0.0f;  // the factor of an absent token
+    float* my_meta = &sm.meta[0][mkind][32 * warp + 16 * mseg + mrow0];
+    Ring3 r{0, 0u};  // chunk c: key-code, value and factor buffer r.i
+    // chunk c: key codes -> TMEM, value codes and factors -> smem, then the
+    // loads of chunk c+1 into the registers just freed (the segments were
+    // prefetched into L2 four chunks earlier)
+#pragma unroll 1
+    for (int c = 0; c < nchunks; ++c) {
+      Stage& s = st;
+      if (c >= kNV) {  // both buffers r.i are free once PV(c-3) (issued after QK(c-2)) is done
+        if (!mbar_wait(&sm.pv_done[r.i], r.ph ^ 1u, abort)) bad = true;
+        tc_fence_after();
+      }
+#pragma unroll
+      for (int sg = 0; sg < 2; ++sg) {  // key codes of segment sg -> lanes 32 warp + 16 sg + [0, 16)
+        const uint4 ka = s.k[2 * sg], kb = s.k[2 * sg + 1];
+        const uint32_t wa[4] = {ka.x, ka.y, ka.z, ka.w}, wb[4] = {kb.x, kb.y, kb.z, kb.w};
+        uint32_t w[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          w[4 * j] = wa[j] & 0x0F0F0F0Fu;
+          w[4 * j + 1] = (wa[j] >> 4) & 0x0F0F0F0Fu;
+          w[4 * j + 2] = wb[j] & 0x0F0F0F0Fu;
+          w[4 * j + 3] = (wb[j] >> 4) & 0x0F0F0F0Fu;
+        }
+        tmem_st16x256(my_lanes + (static_cast<uint32_t>(16 * sg) << 16) + kColA + 32 * r.i, w);
+      }
+#pragma unroll
+      for (int sg = 0; sg < 2; ++sg) {  // value codes, one byte each
+        const uint32_t va = my_vt[sg] + r.i * (kChunkTokens * kHeadDim);
+        const uint32_t vw[4] = {s.v[sg].x, s.v[sg].y, s.v[sg].z, s.v[sg].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t x = vw[i];
+          sts128(va + 128 * i, x & 0x03030303u, x & 0x0C0C0C0Cu, x & 0x30303030u, x & 0xC0C0C0C0u);
+        }
+      }
+      {  // factors of my four rows; absent tokens get 0 (S_V: -1)
+        const int blk = blk0 + kChunkBlocks * c + 2 * warp + mseg;
+        const int nv = ((s.ok >> mseg) & 1u) ? min(4, max(0, L - blk * kBlockSize - mrow0)) : 0;
+        float4 o;
+        o.x = nv > 0 ? h2f(s.m.x) * mscale : mnone;
+        o.y = nv > 1 ? h2f(s.m.x >> 16) * mscale : mnone;
+        o.z = nv > 2 ? h2f(s.m.y) * mscale : mnone;
+        o.w = nv > 3 ? h2f(s.m.y >> 16) * mscale : mnone;
+        if (mkind == 0) {
+          o.x *= c1;
+          o.y *= c1;
+          o.z *= c1;
+          o.w *= c1;
+        }
+        *reinterpret_cast<float4*>(my_meta + r.i * (4 * kChunkTokens)) = o;
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      async_proxy_fence();
+      mbar_arrive(&sm.kv_ready[r.i]);
+
       {
-        const uint32_t addr = smem_u32(sg + kOffV + ld_tok * kVRowBytes + 16 * ld_half);
-        asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-                     : "=r"(vr[0]), "=r"(vr[1]), "=r"(vr[2]), "=r"(vr[3])
-                     : "r"(addr));
+        const int32_t q0 = __shfl_sync(0xffffffffu, bq[0], 0), q1 = __shfl_sync(0xffffffffu, bq[0], 1);
+        if (c + 1 < nchunks) load_stage(s, c + 1, q0, q1);
       }
-      const uint32_t vs[4] = {vr[0] >> 10, vr[1] >> 10, vr[2] >> 10, vr[3] >> 10};
+      prefetch_seg(bq[4]);
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        mma16816(o[8 * h2 + 0], pa, codes_f16<0x00030003u>(vr[h2], bias), codes_f16<0x00030003u>(vr[2 + h2], bias));
-        mma16816(o[8 * h2 + 1], pa, codes_f16<0x000C000Cu>(vr[h2], bias), codes_f16<0x000C000Cu>(vr[2 + h2], bias));
-        mma16816(o[8 * h2 + 2], pa, codes_f16<0x00300030u>(vr[h2], bias), codes_f16<0x00300030u>(vr[2 + h2], bias));
-        mma16816(o[8 * h2 + 3], pa, codes_f16<0x00C000C0u>(vr[h2], bias), codes_f16<0x00C000C0u>(vr[2 + h2], bias));
-        mma16816(o[8 * h2 + 4], pa, codes_f16<0x03000300u>(vr[h2], bias), codes_f16<0x03000300u>(vr[2 + h2], bias));
-        mma16816(o[8 * h2 + 5], pa, codes_f16<0x00030003u>(vs[h2], bias), codes_f16<0x00030003u>(vs[2 + h2], bias));
-        mma16816(o[8 * h2 + 6], pa, codes_f16<0x000C000Cu>(vs[h2], bias), codes_f16<0x000C000Cu>(vs[2 + h2], bias));
-        mma16816(o[8 * h2 + 7], pa, codes_f16<0x00300030u>(vs[h2], bias), codes_f16<0x00300030u>(vs[2 + h2], bias));
-      }
-    } else if (lane == 0 && i >= kStages) {
-      record_status(a.status, KVQ_ERR_OUT_OF_RANGE);
+      for (int i = 0; i < 5; ++i) bq[i] = bq[i + 1];
+      bq[5] = bid_of(c + 7);
+      r.next();
     }
-    __syncwarp();  // every lane is done reading the slot before it is refilled
-    // refill this slot with the warp's block j = i + kStages
-    const int j = i + kStages;
-    valid_bits &= ~(1u << slot);
-    if (j < nmine) {
-      if (j >= wbase + 32) {  // slide the block-table window by 32 entries
-        win0 = win1;
-        wbase += 32;
-        win1 = wbase + 32 + lane < nmine ? bt_row[W * (wbase + 32 + lane)] : -1;
+  } else if (warp == kMmaWarp) {
+    // one lane issues, in this order: QK(0), QK(1), PV(0), QK(2), PV(1), ...
+    const uint32_t qb0 = smem_u32(sm.qb);
+    const uint32_t vt0 = smem_u32(sm.vt[0]);
+    const uint32_t pm0 = smem_u32(sm.pm[0]);
+    Ring3 rq{0, 0u};  // QK(c)
+    Ring3 rp{0, 0u};  // PV(c - 1)
+#pragma unroll 1
+    for (int c = 0; c <= nchunks; ++c) {
+      if (c < nchunks) {  // QK(c): its codes are in, and S buffer c % 2 was read (chunk c-2)
+        const int P = c & 1;
+        if (!mbar_wait(&sm.kv_ready[rq.i], rq.ph, abort)) bad = true;
+        if (c >= kNS && !mbar_wait(&sm.s_free[P], static_cast<uint32_t>(((c - kNS) >> 1) & 1), abort)) bad = true;
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t acol = tbase + kColA + 32 * rq.i, scol = tbase + kColS + 32 * P;
+#pragma unroll
+          for (int s = 0; s < 4; ++s) mma_qk(scol, acol + 8 * s, sdesc(qb0 + 1024 * s, 512, 128), s > 0);
+          mma_commit(&sm.qk_done[P]);
+        }
+        __syncwarp();
+        rq.next();
       }
-      const int32_t p = __shfl_sync(0xffffffffu, win0, j - wbase);
-      if (p >= 0 && p < a.num_blocks) {
-        bulk_load_segment_if(lane == 0, sm.stage[warp][slot], pool_h + p * pstride, &sm.bar[warp][slot]);
-        valid_bits |= 1u << slot;
+      if (c >= 1) {  // PV(c-1) once its P' is written
+        if (!mbar_wait(&sm.p_ready[rp.i], rp.ph, abort)) bad = true;
+        tc_fence_after();
+        if (lane == 0) {
+          const bool fresh = sm.fresh[rp.i] != 0;
+          const uint32_t va = vt0 + rp.i * (kChunkTokens * kHeadDim), pa = pm0 + rp.i * (kChunkTokens * 32);
+#pragma unroll
+          for (int s = 0; s < 4; ++s)
+            mma_pv(tbase + kColO, sdesc(va + 4096 * s, 1024, 128), sdesc(pa + 1024 * s, 256, 128), !fresh || s > 0);
+          mma_commit(&sm.pv_done[rp.i]);
+        }
+        __syncwarp();
+        rp.next();
       }
     }
-  }
-  if (timed_out) {
-    // a copy never landed: report it, give the others a bounded chance to
-    // finish, and leave this warp's contribution empty
-    if (lane == 0) record_status(a.status, KVQ_ERR_DEVICE_TIMEOUT);
-    for (int s2 = 0; s2 < kStages; ++s2)
-      if (valid_bits & (1u << s2)) mbar_wait(&sm.bar[warp][s2], (phase_bits >> s2) & 1u);
-    m_ref = -CUDART_INF_F;
-    l_part = z_part = 0.0f;
-  }
+    if (lane == 0) mma_commit(&sm.fin);
+    __syncwarp();
+    if (!mbar_wait_final(&sm.fin, 0u)) bad = true;
+  } else {
+    // softmax warps: thread stok <-> token stok of S, value position stok of O
+    const int sw = warp - kLoadWarps;
+    const int stok = tid - 32 * kLoadWarps;
+    const uint32_t my_lanes = tbase + (static_cast<uint32_t>(sw * 32) << 16);
+    const uint32_t my_pm = smem_u32(sm.pm[0]) + (stok >> 3) * 256 + (stok & 7) * 16;
+    // output scale of my value position: the fixed point and the 4^k of the spread
+    const float oscale = kFixInv * __uint_as_float((127u - 2u * ((stok >> 2) & 3)) << 23);
+    float qs[G], mr[G], lr[G], zr[G], oacc[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      qs[g] = sm.hq[g].x;
+      mr[g] = kNoMax;
+      lr[g] = zr[g] = oacc[g] = 0.0f;
+    }
+    int fresh_c = 0;  // the chunk whose PV started the integer accumulator
 
-  // ---- 4. merge: lanes of a head, then warps, then splits
-  l_part += __shfl_xor_sync(0xffffffffu, l_part, 1);
-  l_part += __shfl_xor_sync(0xffffffffu, l_part, 2);
-  z_part += __shfl_xor_sync(0xffffffffu, z_part, 1);
-  z_part += __shfl_xor_sync(0xffffffffu, z_part, 2);
-  __syncthreads();  // every warp is done with its stages: reuse them
-  float(*wo)[8][kHeadDim] = reinterpret_cast<float(*)[8][kHeadDim]>(&sm.stage[0][0][0]);
-  {
-    // n-tile (h, k) column n is dim 64h + 8n + k; its codes carry 4^k
-    // (k <= 4) or 4^(k-5) (k >= 5)
+    // fold the integer accumulator (my lane = value position stok) into oacc
+    auto flush_o = [&](const float (&alpha)[G]) {
+      uint32_t r[16], r2[16];
+      tmem_ld16(my_lanes + kColO, r);
+      tmem_ld16(my_lanes + kColO + 16, r2);
+      tmem_wait_ld();
 #pragma unroll
-    for (int h2 = 0; h2 < 2; ++h2) {
+      for (int g = 0; g < G; ++g) {
+        const uint32_t* q = g < 4 ? r + 4 * g : r2 + 4 * g - 16;
+        const float v = fmaf(static_cast<float>(static_cast<int>(q[3])), 16777216.0f,
+                             fmaf(static_cast<float>(static_cast<int>(q[2])), 65536.0f,
+                                  fmaf(static_cast<float>(static_cast<int>(q[1])), 256.0f,
+                                       static_cast<float>(static_cast<int>(q[0])))));
+        oacc[g] = alpha[g] * fmaf(v, oscale, oacc[g]);
+      }
+    };
+
+    Ring3 r{0, 0u};  // chunk c: buffers r.i
+#pragma unroll 1
+    for (int c = 0; c < nchunks; ++c) {
+      const int P = c & 1;
+      if (!mbar_wait(&sm.qk_done[P], static_cast<uint32_t>((c >> 1) & 1), abort)) bad = true;
+      tc_fence_after();
+      uint32_t sr[16], sr2[8];
+      tmem_ld16(my_lanes + kColS + 32 * P, sr);
+      tmem_ld8(my_lanes + kColS + 32 * P + 16, sr2);
+      if (!mbar_wait(&sm.kv_ready[r.i], r.ph, abort)) bad = true;
+      const float4 mt = make_float4(sm.meta[r.i][0][stok], sm.meta[r.i][1][stok], sm.meta[r.i][2][stok],
+                                    sm.meta[r.i][3][stok]);  // S_K c1, Z_K, S_V 2^27 (< 0: no token), Z_V
+      const bool valid = mt.z >= 0.0f;
+      // E with S_V < 2^E, from the exponent of S_V 2^27; floored at -24
+      const int ex = static_cast<int>((__float_as_uint(mt.z) >> 23) & 0xFFu) - 153;
+      const float e = static_cast<float>(max(ex, -24));
+      tmem_wait_ld();
+      float dg[G];
+      float dmax = -CUDART_INF_F;
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const float f = 1.0f / static_cast<float>(1 << (2 * (k < 5 ? k : k - 5)));
-        const int nt = 8 * h2 + k;
-        wo[warp][g][64 * h2 + 16 * c + k] = fmaf(o[nt][0] + o[nt][2], f, z_part);
-        wo[warp][g][64 * h2 + 16 * c + 8 + k] = fmaf(o[nt][1] + o[nt][3], f, z_part);
+      for (int g = 0; g < G; ++g) {
+        const int e12 = static_cast<int>(sr[8 + g]) * 254 + static_cast<int>(sr2[g]);
+        const float xg = fmaf(__int2float_rn(e12), 1.0f / 64516.0f, small_i2f(sr[g]));
+        dg[g] = fmaf(mt.x, xg, fmaf(mt.y, qs[g], -mr[g]));
+        dmax = fmaxf(dmax, dg[g]);
+      }
+      const bool flag = valid && (dmax + e > kTrigger);
+      const bool any = soft_vote_any(flag) || c - fresh_c >= kFlushChunks;
+      if (any) {
+        // rare: move the running max of the heads to the chunk's max of s + E;
+        // the scores are formed again from S (still in tensor memory: it is
+        // released below), exactly, without the running max
+        tmem_ld16(my_lanes + kColS + 32 * P, sr);
+        tmem_ld8(my_lanes + kColS + 32 * P + 16, sr2);
+        tmem_wait_ld();
+        float sg[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const int e12 = static_cast<int>(sr[8 + g]) * 254 + static_cast<int>(sr2[g]);
+          const float xg = fmaf(__int2float_rn(e12), 1.0f / 64516.0f, small_i2f(sr[g]));
+          sg[g] = fmaf(mt.x, xg, mt.y * qs[g]);
+          float u = valid ? sg[g] + e : -CUDART_INF_F;
+#pragma unroll
+          for (int o = 16; o; o >>= 1) u = fmaxf(u, __shfl_xor_sync(0xffffffffu, u, o));
+          if (lane == 0) sm.red[sw][g][0] = u;
+        }
+        soft_sync();
+        float alpha[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float M = fmaxf(fmaxf(sm.red[0][g][0], sm.red[1][g][0]), fmaxf(sm.red[2][g][0], sm.red[3][g][0]));
+          const float mn = fmaxf(mr[g], M);
+          alpha[g] = ex2(mr[g] - mn);
+          lr[g] *= alpha[g];
+          zr[g] *= alpha[g];
+          dg[g] = sg[g] - mn;
+          mr[g] = mn;
+        }
+        if (c > fresh_c) {  // PVs of chunks fresh_c .. c-1 ran into O: fold it, restart
+          const int pi = r.i == 0 ? 2 : r.i - 1;
+          const uint32_t pph = r.i == 0 ? r.ph ^ 1u : r.ph;
+          if (!mbar_wait(&sm.pv_done[pi], pph, abort)) bad = true;
+          tc_fence_after();
+          flush_o(alpha);
+        } else {
+#pragma unroll
+          for (int g = 0; g < G; ++g) oacc[g] *= alpha[g];
+        }
+        fresh_c = c;
+        // the reductions above read sm.red: none writes it again before the next vote
+      }
+      tc_fence_before();
+      mbar_arrive(&sm.s_free[P]);  // S of chunk c is read
+      // P' of chunk c -> pm[r.i] (free: PV(c-3) was issued before QK(c), which is done)
+      uint32_t pw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float p = valid ? ex2(dg[g]) : 0.0f;
+        lr[g] += p;
+        zr[g] = fmaf(p, mt.w, zr[g]);
+        pw[g] = __float2uint_rn(p * mt.z);  // rne(P' 2^27) < 2^30
+      }
+      const uint32_t pa = my_pm + r.i * (kChunkTokens * 32);
+      sts128(pa, pw[0], pw[1], pw[2], pw[3]);
+      sts128(pa + 128, pw[4], pw[5], pw[6], pw[7]);
+      if (stok == 0) sm.fresh[r.i] = fresh_c == c;
+      async_proxy_fence();
+      tc_fence_before();
+      mbar_arrive(&sm.p_ready[r.i]);
+      r.next();
+    }
+    if (nchunks > 0) {  // the last PV, then the accumulator
+      const int pi = r.i == 0 ? 2 : r.i - 1;
+      const uint32_t pph = r.i == 0 ? r.ph ^ 1u : r.ph;
+      if (!mbar_wait(&sm.pv_done[pi], pph, abort)) bad = true;
+      tc_fence_after();
+      float one[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) one[g] = 1.0f;
+      flush_o(one);
+    }
+    // l and zeta over the 128 tokens' threads; o~ in dim order
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      float l = lr[g], z = zr[g];
+#pragma unroll
+      for (int o = 16; o; o >>= 1) {
+        l += __shfl_xor_sync(0xffffffffu, l, o);
+        z += __shfl_xor_sync(0xffffffffu, z, o);
+      }
+      if (lane == 0) {
+        sm.red[sw][g][0] = l;
+        sm.red[sw][g][1] = z;
       }
     }
-    if (c == 0) {
-      sm.wm[warp][g] = m_ref;
-      sm.wl[warp][g] = l_part;
+    soft_sync();
+    const int d = value_dim_of_pos(stok);
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float z = (sm.red[0][g][1] + sm.red[1][g][1]) + (sm.red[2][g][1] + sm.red[3][g][1]);
+      sm.obuf[g][d] = oacc[g] + z;
+      if (stok == g) {
+        sm.hl[g] = (sm.red[0][g][0] + sm.red[1][g][0]) + (sm.red[2][g][0] + sm.red[3][g][0]);
+        sm.hm[g] = mr[g];
+      }
     }
   }
+  if (bad) record_status(a.status, KVQ_ERR_DEVICE_TIMEOUT);
+  if (bad_blk && lane == 0) record_status(a.status, KVQ_ERR_OUT_OF_RANGE);
+  tc_fence_before();
   __syncthreads();
-  // per head: the warps' common max, their weights 2^(m_w - M), and l
-  if (tid < G) {
-    const int gg = tid;
-    float M = -CUDART_INF_F;
-#pragma unroll
-    for (int w = 0; w < W; ++w)
-      if (sm.wl[w][gg] > 0.0f) M = fmaxf(M, sm.wm[w][gg]);
-    float lsum = 0.0f;
-#pragma unroll
-    for (int w = 0; w < W; ++w) {
-      const float f = sm.wl[w][gg] > 0.0f ? ex2(sm.wm[w][gg] - M) : 0.0f;
-      sm.wf[gg][w] = f;
-      lsum = fmaf(sm.wl[w][gg], f, lsum);
-    }
-    sm.hm[gg] = M;
-    sm.hl[gg] = lsum;
-  }
+  tc_fence_after();
+  if (warp == kMmaWarp)  // every MMA and tensor-memory load is complete
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "n"(kTmemCols));
   __syncthreads();
+
+  // ---- 2. partial record, ticket, merge -------------------------------------
   for (int t = tid; t < G * kHeadDim; t += kThreads) {
-    const int gg = t / kHeadDim, d = t % kHeadDim;
-    float acc = 0.0f;
-#pragma unroll
-    for (int w = 0; w < W; ++w) acc = fmaf(wo[w][gg][d], sm.wf[gg][w], acc);
-    const float M = sm.hm[gg], lsum = sm.hl[gg];
-    float* rec =
-        a.partials + ((static_cast<int64_t>(b) * a.num_q_heads + h * G + gg) * a.nsplit + split) * kPartialFloats;
+    const int g = t / kHeadDim, d = t % kHeadDim;
+    const float lsum = sm.hl[g];
     if (a.nsplit == 1) {
-      sm.q[gg][d] = lsum > 0.0f ? acc / lsum : 0.0f;  // nothing to merge: finish here
+      sm.obuf[g][d] = lsum > 0.0f ? sm.obuf[g][d] / lsum : 0.0f;
     } else {
-      rec[d] = acc;
+      float* rec =
+          a.partials + ((static_cast<int64_t>(b) * a.num_q_heads + h * G + g) * a.nsplit + split) * kPartialFloats;
+      rec[d] = sm.obuf[g][d];
       if (d == 0) {
-        rec[kHeadDim] = M;
+        rec[kHeadDim] = sm.hm[g];
         rec[kHeadDim + 1] = lsum;
       }
     }
@@ -525,39 +807,40 @@ __global__ void __launch_bounds__(W * 32, kMinCtasPerSm) decode_kernel(DecodeArg
     // the last CTA of (b, h) merges the splits: (m, l) of every split into
     // smem, merge weights per head, then every output element as a weighted
     // sum of its nsplit partials (float4 loads, eight in flight per thread)
-    float* mls = reinterpret_cast<float*>(&sm.stage[0][0][0]);  // [G][nsplit] m, then l, then w
+    float* mls = reinterpret_cast<float*>(&sm.vt[0][0]);  // [G][nsplit] m, then l, then w
     const int ns = a.nsplit;
     const float* base = a.partials + (static_cast<int64_t>(b) * a.num_q_heads + h * G) * ns * kPartialFloats;
     for (int t = tid; t < G * ns; t += kThreads) {
-      const float2 ml = __ldcg(reinterpret_cast<const float2*>(base + static_cast<int64_t>(t) * kPartialFloats + kHeadDim));
+      const float2 ml =
+          __ldcg(reinterpret_cast<const float2*>(base + static_cast<int64_t>(t) * kPartialFloats + kHeadDim));
       mls[t] = ml.x;
       mls[G * ns + t] = ml.y;
     }
     __syncthreads();
-    for (int gg = warp; gg < G; gg += W) {
+    for (int g = warp; g < G; g += kThreads / 32) {
       float M = -CUDART_INF_F;
       for (int s = lane; s < ns; s += 32)
-        if (mls[G * ns + gg * ns + s] > 0.0f) M = fmaxf(M, mls[gg * ns + s]);
+        if (mls[G * ns + g * ns + s] > 0.0f) M = fmaxf(M, mls[g * ns + s]);
 #pragma unroll
       for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
       float lsum = 0.0f;
       for (int s = lane; s < ns; s += 32) {
-        const float l = mls[G * ns + gg * ns + s];
-        if (l > 0.0f) lsum = fmaf(l, ex2(mls[gg * ns + s] - M), lsum);
+        const float l = mls[G * ns + g * ns + s];
+        if (l > 0.0f) lsum = fmaf(l, ex2(mls[g * ns + s] - M), lsum);
       }
 #pragma unroll
       for (int off = 16; off; off >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
       const float inv = lsum > 0.0f ? 1.0f / lsum : 0.0f;
       for (int s = lane; s < ns; s += 32) {
-        const float l = mls[G * ns + gg * ns + s];
-        mls[2 * G * ns + gg * ns + s] = l > 0.0f ? ex2(mls[gg * ns + s] - M) * inv : 0.0f;
+        const float l = mls[G * ns + g * ns + s];
+        mls[2 * G * ns + g * ns + s] = l > 0.0f ? ex2(mls[g * ns + s] - M) * inv : 0.0f;
       }
     }
     __syncthreads();
     for (int t = tid; t < G * (kHeadDim / 4); t += kThreads) {
-      const int gg = t / (kHeadDim / 4), q4 = t % (kHeadDim / 4);
-      const float* w = mls + 2 * G * ns + gg * ns;
-      const float4* src = reinterpret_cast<const float4*>(base + static_cast<int64_t>(gg) * ns * kPartialFloats) + q4;
+      const int g = t / (kHeadDim / 4), q4 = t % (kHeadDim / 4);
+      const float* w = mls + 2 * G * ns + g * ns;
+      const float4* src = reinterpret_cast<const float4*>(base + static_cast<int64_t>(g) * ns * kPartialFloats) + q4;
       constexpr int kStride = kPartialFloats / 4;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
       int s = 0;
@@ -582,22 +865,22 @@ __global__ void __launch_bounds__(W * 32, kMinCtasPerSm) decode_kernel(DecodeArg
         acc.z = fmaf(v.z, wu, acc.z);
         acc.w = fmaf(v.w, wu, acc.w);
       }
-      sm.q[gg][4 * q4] = acc.x;
-      sm.q[gg][4 * q4 + 1] = acc.y;
-      sm.q[gg][4 * q4 + 2] = acc.z;
-      sm.q[gg][4 * q4 + 3] = acc.w;
+      sm.obuf[g][4 * q4] = acc.x;
+      sm.obuf[g][4 * q4 + 1] = acc.y;
+      sm.obuf[g][4 * q4 + 2] = acc.z;
+      sm.obuf[g][4 * q4 + 3] = acc.w;
     }
     if (tid == 0) a.tickets[b * a.num_kv_heads + h] = 0;  // ready for the next call
   }
   __syncthreads();
 
-  // rotate back once (warp w owns heads w, w+W, ...) and store
-  for (int gg = warp; gg < G; gg += W) {
+  // rotate back once (warp w owns heads w, w + 9, ...) and store
+  for (int g = warp; g < G; g += kThreads / 32) {
     float x[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) x[k] = sm.q[gg][lane + 32 * k];
+    for (int k = 0; k < 4; ++k) x[k] = sm.obuf[g][lane + 32 * k];
     fwht_warp(x, lane, 1.0f);
-    const int64_t o0 = (static_cast<int64_t>(b) * a.num_q_heads + h * G + gg) * kHeadDim;
+    const int64_t o0 = (static_cast<int64_t>(b) * a.num_q_heads + h * G + g) * kHeadDim;
 #pragma unroll
     for (int k = 0; k < 4; ++k) store_from_f32(a.out, a.out_dtype, o0 + lane + 32 * k, x[k]);
   }
@@ -605,12 +888,10 @@ __global__ void __launch_bounds__(W * 32, kMinCtasPerSm) decode_kernel(DecodeArg
 
 template <int G>
 cudaError_t launch_g(const DecodeArgs& a, cudaStream_t stream) {
-  constexpr int W = kDecodeWarps;
-  const int smem = static_cast<int>(sizeof(DecodeSmem<W>));
-  const cudaError_t e = ensure_smem_limit<decode_kernel<G, W>>(smem);
+  const cudaError_t e = ensure_smem_limit<decode_kernel<G>>(kSmemBytes);
   if (e != cudaSuccess) return e;
   const dim3 grid(a.nsplit, a.num_kv_heads, a.batch);
-  decode_kernel<G, W><<<grid, W * 32, smem, stream>>>(a);
+  decode_kernel<G><<<grid, kThreads, kSmemBytes, stream>>>(a);
   return cudaGetLastError();
 }
 
@@ -621,17 +902,17 @@ int decode_ctas_per_sm() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 1;
   if (cached[dev] > 0) return cached[dev];
-  constexpr int W = kDecodeWarps;
-  const int smem = static_cast<int>(sizeof(DecodeSmem<W>));
   int n = 0;
-  if (ensure_smem_limit<decode_kernel<8, W>>(smem) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<8, W>, W * 32, smem) != cudaSuccess || n < 1)
+  if (ensure_smem_limit<decode_kernel<8>>(kSmemBytes) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<8>, kThreads, kSmemBytes) != cudaSuccess ||
+      n < 1)
     n = 1;
-  cached[dev] = n;
-  return n;
+  cached[dev] = n < 2 ? n : 2;  // two CTAs' tensor memory (2 x 256 columns) fills an SM
+  return cached[dev];
 }
 
 int decode_max_splits() { return kMaxSplits; }
+int decode_chunk_blocks() { return kChunkBlocks; }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   switch (a.num_q_heads / a.num_kv_heads) {

@@ -92,18 +92,21 @@ int device_sm_count() {
 }
 
 // Split-K plan.  The context of every sequence is cut into nsplit splits of
-// blocks_per_split blocks; one CTA owns one (sequence, kv head, split).  The
-// default picks nsplit (at most decode_max_splits()) by a small cost model:
-// CTAs run in waves of (SMs x resident CTAs per SM), a CTA costs its blocks
-// plus a fixed prologue worth about 4 blocks, and every extra split adds
-// about half a block of merge work.  A requested blocks_per_split is raised
-// if it would need more splits than the cap.
+// blocks_per_split blocks; one CTA owns one (sequence, kv head, split) and
+// walks it in chunks of decode_chunk_blocks() blocks.  The default picks
+// nsplit (at most decode_max_splits()) by a small cost model: CTAs run in
+// waves of (SMs x resident CTAs per SM), a CTA costs its chunks plus a fixed
+// start-up worth about two chunks (the first loads, the query rotation, the
+// partial record), and every extra split adds a tenth of a chunk of merge
+// work.  Default splits are whole chunks.  A requested blocks_per_split is
+// raised if it would need more splits than the cap.
 int plan_decode(int32_t batch, int32_t num_kv_heads, int32_t num_q_heads, int32_t max_seq_len,
                 int32_t bps_request, DecodePlan* plan) {
   if (batch < 0 || num_kv_heads <= 0 || num_q_heads <= 0 || max_seq_len < 0 || bps_request < 0)
     return KVQ_ERR_INVALID;
   const int64_t nb = (static_cast<int64_t>(max_seq_len) + kBlockSize - 1) / kBlockSize;
   const int64_t cap = decode_max_splits();
+  const int64_t cb = decode_chunk_blocks();
   int64_t bps = bps_request;
   if (nb == 0) {
     bps = 1;
@@ -111,12 +114,15 @@ int plan_decode(int32_t batch, int32_t num_kv_heads, int32_t num_q_heads, int32_
     const int64_t units = static_cast<int64_t>(batch) * num_kv_heads;
     const int64_t slots = static_cast<int64_t>(device_sm_count()) * decode_ctas_per_sm();
     double best = 1e300;
-    bps = nb;
+    bps = (nb + cb - 1) / cb * cb;
+    int64_t last = -1;
     for (int64_t n = 1; n <= cap && n <= nb; ++n) {
-      const int64_t b = (nb + n - 1) / n;
-      if ((nb + b - 1) / b != n) continue;
-      const int64_t waves = (units * n + slots - 1) / slots;
-      const double cost = static_cast<double>(waves) * (b + 4) + 0.5 * n;
+      const int64_t b = ((nb + n - 1) / n + cb - 1) / cb * cb;  // whole chunks
+      const int64_t ns = (nb + b - 1) / b;
+      if (ns > cap || b == last) continue;
+      last = b;
+      const int64_t waves = (units * ns + slots - 1) / slots;
+      const double cost = static_cast<double>(waves) * (static_cast<double>(b) / cb + 2.0) + 0.1 * ns;
       if (cost < best) {
         best = cost;
         bps = b;

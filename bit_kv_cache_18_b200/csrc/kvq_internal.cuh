@@ -114,6 +114,7 @@ int plan_decode(int32_t batch, int32_t num_kv_heads, int32_t num_q_heads, int32_
 int device_sm_count();
 int decode_ctas_per_sm();  // resident decode CTAs per SM on the current device
 int decode_max_splits();   // upper bound the split plan respects
+int decode_chunk_blocks();  // blocks the decode kernel takes per step (splits are multiples of it)
 
 // Raise a kernel's dynamic shared-memory limit once per device (a host call
 // that is not a stream operation, so it is also safe while a stream is being
