@@ -7,9 +7,9 @@
 // different chunks at the same time and hand buffers to each other through
 // mbarrier rings:
 //   * loader warps 0-3 (thread t <-> token t of a chunk <-> TMEM lane t):
-//     read their two segments of each chunk with coalesced 16-byte loads
-//     straight into registers one chunk ahead (after an L2 prefetch of the
-//     segments five chunks ahead);
+//     bring their two segments of each chunk into a private three-slot
+//     shared-memory ring with bulk copies (TMA, one instruction per segment)
+//     three chunks ahead, after an L2 prefetch six chunks ahead;
 //     spread the 4-bit key codes to one byte each into tensor memory (A of
 //     QK) and the 2-bit value codes to one byte each into shared memory (A of
 //     PV), and publish the per-token factors;
@@ -112,7 +112,10 @@ struct __align__(1024) Smem {
   uint8_t pm[kNV][kChunkTokens * 32];        // 3 x 4 KB
   uint8_t qb[32 * kHeadDim];                 // 4 KB
   float meta[kNV][4][kChunkTokens];          // per token: S_K c1, Z_K, S_V 2^27 (< 0: no token), Z_V
-  float obuf[8][kHeadDim];                   // o~ (epilogue)
+  union {
+    uint8_t stg[kLoadWarps][kNV][2 * kSegBytes];  // loader warp w: its two segments of chunk c in slot c % 3
+    float obuf[8][kHeadDim];                      // o~ (epilogue, after the scan)
+  };
   float2 hq[8];                              // per head: sum(q~), max|q~|
   float red[kSoftWarps][8][2];               // cross-warp reductions
   float hm[8], hl[8], hz[8];
@@ -121,6 +124,7 @@ struct __align__(1024) Smem {
   uint64_t s_free[kNS];    // softmax -> MMA warp: S of chunk c read
   uint64_t p_ready[kNV];   // softmax -> MMA warp: P' of chunk c written
   uint64_t pv_done[kNV];   // PV(c) complete -> loaders, softmax (and QK(c+1) complete)
+  uint64_t full[kLoadWarps][kNV];  // TMA -> loader warp w: segments of chunk c in slot c % 3
   uint64_t fin;            // every MMA issued is complete
   uint32_t tmem_base;
   int fresh[kNV];          // the PV of chunk c starts the accumulator afresh
@@ -156,6 +160,17 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
 }
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("{ .reg .b64 st; mbarrier.arrive.shared::cta.b64 st, [%0]; }" ::"r"(smem_u32(bar)) : "memory");
+}
+// Arrive once and expect `bytes` more from the bulk copies tracked here.
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+// Bulk copy (TMA, no tensor map) of `bytes` from global to this CTA's shared
+// memory, completing on `bar`; both addresses 16-byte aligned, bytes % 16 == 0.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t done;
@@ -242,18 +257,18 @@ __device__ __forceinline__ void tmem_ld8(uint32_t addr, uint32_t (&r)[8]) {
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-__device__ __forceinline__ uint4 ldg16(const uint8_t* p) {
-  uint4 r;
-  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
-  return r;
-}
-__device__ __forceinline__ uint2 ldg8(const uint8_t* p) {
-  uint2 r;
-  asm volatile("ld.global.nc.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
-  return r;
-}
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 r;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(addr));
+  return r;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+  uint2 r;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(addr));
+  return r;
 }
 __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
@@ -303,20 +318,6 @@ __device__ __forceinline__ int key_pos_of_dim(int d) {
 }
 __device__ __forceinline__ int value_dim_of_pos(int p) { return (p & ~15) | ((p & 3) << 2) | ((p >> 2) & 3); }
 
-// One lane's share of a loader warp's two segments of one chunk, in
-// registers (coalesced 16-byte pieces; segment s = 0, 1):
-//   k[2s], k[2s+1]: key-code bytes 16 lane + [0, 16) and 512 + 16 lane + [0, 16)
-//                   (rows lane/4 and 8 + lane/4, dims 32 (lane%4) + [0, 32));
-//   v[s]:           value-code bytes 16 lane + [0, 16) (row lane/2, dims 64 (lane%2) + [0, 64));
-//   m:              factor bytes 8 (lane%16) + [0, 8) of segment lane/16
-//                   (four fp16 of kind (lane/4)%4 for rows 4 (lane%4) + [0, 4)).
-struct Stage {
-  uint4 k[4];
-  uint4 v[2];
-  uint2 m;
-  uint32_t ok;  // bit s: segment s is inside the split and the pool
-};
-
 // Bounded wait that ignores the abort flag: the issuer's last wait for its
 // own MMAs, so tensor memory is never released under a running MMA.
 __device__ __forceinline__ bool mbar_wait_final(uint64_t* bar, uint32_t parity) {
@@ -365,41 +366,18 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
     const int blk = blk0 + kChunkBlocks * c + 2 * warp + (lane & 1);
     return blk < blk1 ? __ldg(bt_row + blk) : -1;
   };
-  // my share of chunk c, segments in blocks p0, p1; blocks outside the split
-  // or the pool read block 0 and are marked absent
-  auto load_stage = [&](Stage& s, int c, int32_t p0, int32_t p1) {
-    const int blk = blk0 + kChunkBlocks * c + 2 * warp;
-    const bool live0 = blk < blk1, live1 = blk + 1 < blk1;
-    const bool ok0 = live0 && p0 >= 0 && p0 < a.num_blocks;
-    const bool ok1 = live1 && p1 >= 0 && p1 < a.num_blocks;
-    bad_blk |= (live0 && !ok0) || (live1 && !ok1);
-    s.ok = (ok0 ? 1u : 0u) | (ok1 ? 2u : 0u);
-    if (a.num_blocks > 0) {  // (an empty pool has no block 0)
-      const uint8_t* g0 = pool_h + static_cast<int64_t>(ok0 ? p0 : 0) * pstride;
-      const uint8_t* g1 = pool_h + static_cast<int64_t>(ok1 ? p1 : 0) * pstride;
-      s.k[0] = ldg16(g0 + kOffK + 16 * lane);
-      s.k[1] = ldg16(g0 + kOffK + 512 + 16 * lane);
-      s.k[2] = ldg16(g1 + kOffK + 16 * lane);
-      s.k[3] = ldg16(g1 + kOffK + 512 + 16 * lane);
-      s.v[0] = ldg16(g0 + kOffV + 16 * lane);
-      s.v[1] = ldg16(g1 + kOffV + 16 * lane);
-      s.m = ldg8((mseg ? g1 : g0) + kOffSK + 8 * (lane & 15));
-    }
-  };
   auto prefetch_seg = [&](int32_t p) {
     if (lane < 2 && p >= 0 && p < a.num_blocks) prefetch_l2(pool_h + static_cast<int64_t>(p) * pstride, kSegBytes);
   };
 
   // ---- 0. set-up: barriers and tensor memory; first loads; query digits ----
-  Stage st{};
-  int32_t bq[6];  // loaders: block ids of chunks c+1 .. c+6 at the start of iteration c
+  int32_t bfirst[kNV];  // loaders: block ids of chunks 0 .. 2
+  int32_t bq[6];        // loaders: block ids of chunks c+3 .. c+8 at the start of iteration c
   if (is_loader) {
-    const int32_t p0 = bid_of(0);
 #pragma unroll
-    for (int i = 0; i < 6; ++i) bq[i] = bid_of(1 + i);
-    load_stage(st, 0, __shfl_sync(0xffffffffu, p0, 0), __shfl_sync(0xffffffffu, p0, 1));
+    for (int i = 0; i < kNV; ++i) bfirst[i] = bid_of(i);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) prefetch_seg(bq[i]);
+    for (int i = 0; i < 6; ++i) bq[i] = bid_of(kNV + i);
   } else if (warp == kMmaWarp) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sm.tmem_base)),
                  "n"(kTmemCols)
@@ -418,6 +396,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
         mbar_init(&sm.s_free[i], 32 * kSoftWarps);
       }
       mbar_init(&sm.fin, 1);
+#pragma unroll
+      for (int w = 0; w < kLoadWarps; ++w)
+#pragma unroll
+        for (int i = 0; i < kNV; ++i) mbar_init(&sm.full[w][i], 1);
       sm.abort = 0;
       asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -488,32 +470,71 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
   // ---- 1. the paged scan ------------------------------------------------------
   if (is_loader) {
     const uint32_t my_lanes = tbase + (static_cast<uint32_t>(warp * 32) << 16);
+    const uint32_t my_stg = smem_u32(sm.stg[warp][0]);
     // my value rows: row lane/2 of segment s, dims 64 (lane%2) + [0, 64)
-    uint32_t my_vt[2];
-#pragma unroll
-    for (int sg = 0; sg < 2; ++sg) {
-      const int tok = 32 * warp + 16 * sg + (lane >> 1);
-      my_vt[sg] = smem_u32(sm.vt[0]) + (tok >> 3) * 1024 + (lane & 1) * 512 + (tok & 7) * 16;
-    }
+    const uint32_t my_vt = smem_u32(sm.vt[0]) + ((32 * warp + (lane >> 1)) >> 3) * 1024 + (lane & 1) * 512 +
+                           (lane >> 1 & 7) * 16;  // segment 1: + 2048
     const int mrow0 = 4 * (lane & 3);    // my factor rows mrow0 .. mrow0+3 of segment mseg
     const int mkind = (lane >> 2) & 3;  // S_K, Z_K, S_V, Z_V
-    const float mscale = mkind == 2 ? kFix : 1.0f;
+    const float mscale = mkind == 0 ? c1 : (mkind == 2 ? kFix : 1.0f);
     const float mnone = mkind == 2 ? -1.0f : 0.0f;  // the factor of an absent token
-    float* my_meta = &sm.meta[0][mkind][32 * warp + 16 * mseg + mrow0];
-    Ring3 r{0, 0u};  // chunk c: key-code, value and factor buffer r.i
-    // chunk c: key codes -> TMEM, value codes and factors -> smem, then the
-    // loads of chunk c+1 into the registers just freed (the segments were
-    // prefetched into L2 four chunks earlier)
+    const uint32_t my_meta = smem_u32(&sm.meta[0][mkind][32 * warp + 16 * mseg + mrow0]);
+    // lanes 0 and 1: bulk copy of segment lane & 1 of chunk c (block p) into
+    // staging slot `slot`; every lane gets the pair of segment flags
+    // (bit s: segment s is inside the split and the pool)
+    auto issue = [&](int c, int32_t p, int slot) -> uint32_t {
+      const int blk = blk0 + kChunkBlocks * c + 2 * warp + (lane & 1);
+      const bool live = blk < blk1;
+      const bool ok = live && p >= 0 && p < a.num_blocks;
+      if (lane < 2) {
+        bad_blk |= live && !ok;
+        uint64_t* bar = &sm.full[warp][slot];
+        if (lane == 0) mbar_arrive_expect_tx(bar, a.num_blocks > 0 ? 2u * kSegBytes : 0u);
+        if (a.num_blocks > 0)  // (an empty pool has no block 0 to stand in)
+          bulk_g2s(my_stg + slot * (2 * kSegBytes) + lane * kSegBytes,
+                   pool_h + static_cast<int64_t>(ok ? p : 0) * pstride, kSegBytes, bar);
+      }
+      return __ballot_sync(0xffffffffu, ok && lane < 2) & 3u;
+    };
+    uint32_t okq[kNV] = {0u, 0u, 0u};  // segment flags of chunks c .. c+2
+#pragma unroll
+    for (int i = 0; i < kNV; ++i)
+      if (i < nchunks) okq[i] = issue(i, bfirst[i], i);
+#pragma unroll
+    for (int i = 0; i < 3; ++i) prefetch_seg(bq[i]);
+    Ring3 r{0, 0u};  // chunk c: staging slot, key-code, value and factor buffers r.i
 #pragma unroll 1
     for (int c = 0; c < nchunks; ++c) {
-      Stage& s = st;
-      if (c >= kNV) {  // both buffers r.i are free once PV(c-3) (issued after QK(c-2)) is done
+      if (!mbar_wait(&sm.full[warp][r.i], r.ph, abort)) bad = true;
+      const uint32_t sb = my_stg + r.i * (2 * kSegBytes);
+      uint4 kr[4], vr[2];
+#pragma unroll
+      for (int sg = 0; sg < 2; ++sg) {
+        kr[2 * sg] = lds128(sb + sg * kSegBytes + kOffK + 16 * lane);
+        kr[2 * sg + 1] = lds128(sb + sg * kSegBytes + kOffK + 512 + 16 * lane);
+        vr[sg] = lds128(sb + sg * kSegBytes + kOffV + 16 * lane);
+      }
+      const uint2 mr2 = lds64(sb + mseg * kSegBytes + kOffSK + 8 * (lane & 15));
+      const uint32_t ok = okq[0];
+      // the slot is read: refill it with chunk c+3 (the reads above are
+      // ordered before the copy's writes by the proxy fence)
+      async_proxy_fence();
+      __syncwarp();
+      okq[0] = okq[1];
+      okq[1] = okq[2];
+      okq[2] = c + kNV < nchunks ? issue(c + kNV, bq[0], r.i) : 0u;
+      prefetch_seg(bq[3]);
+#pragma unroll
+      for (int i = 0; i < 5; ++i) bq[i] = bq[i + 1];
+      bq[5] = bid_of(c + kNV + 6);
+
+      if (c >= kNV) {  // buffers r.i are free once PV(c-3) (issued after QK(c-2)) is done
         if (!mbar_wait(&sm.pv_done[r.i], r.ph ^ 1u, abort)) bad = true;
         tc_fence_after();
       }
 #pragma unroll
       for (int sg = 0; sg < 2; ++sg) {  // key codes of segment sg -> lanes 32 warp + 16 sg + [0, 16)
-        const uint4 ka = s.k[2 * sg], kb = s.k[2 * sg + 1];
+        const uint4 ka = kr[2 * sg], kb = kr[2 * sg + 1];
         const uint32_t wa[4] = {ka.x, ka.y, ka.z, ka.w}, wb[4] = {kb.x, kb.y, kb.z, kb.w};
         uint32_t w[16];
 #pragma unroll
@@ -527,8 +548,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
       }
 #pragma unroll
       for (int sg = 0; sg < 2; ++sg) {  // value codes, one byte each
-        const uint32_t va = my_vt[sg] + r.i * (kChunkTokens * kHeadDim);
-        const uint32_t vw[4] = {s.v[sg].x, s.v[sg].y, s.v[sg].z, s.v[sg].w};
+        const uint32_t va = my_vt + sg * 2048 + r.i * (kChunkTokens * kHeadDim);
+        const uint32_t vw[4] = {vr[sg].x, vr[sg].y, vr[sg].z, vr[sg].w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const uint32_t x = vw[i];
@@ -537,33 +558,17 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
       }
       {  // factors of my four rows; absent tokens get 0 (S_V: -1)
         const int blk = blk0 + kChunkBlocks * c + 2 * warp + mseg;
-        const int nv = ((s.ok >> mseg) & 1u) ? min(4, max(0, L - blk * kBlockSize - mrow0)) : 0;
-        float4 o;
-        o.x = nv > 0 ? h2f(s.m.x) * mscale : mnone;
-        o.y = nv > 1 ? h2f(s.m.x >> 16) * mscale : mnone;
-        o.z = nv > 2 ? h2f(s.m.y) * mscale : mnone;
-        o.w = nv > 3 ? h2f(s.m.y >> 16) * mscale : mnone;
-        if (mkind == 0) {
-          o.x *= c1;
-          o.y *= c1;
-          o.z *= c1;
-          o.w *= c1;
-        }
-        *reinterpret_cast<float4*>(my_meta + r.i * (4 * kChunkTokens)) = o;
+        const int nv = ((ok >> mseg) & 1u) ? min(4, max(0, L - blk * kBlockSize - mrow0)) : 0;
+        sts128(my_meta + r.i * (4 * kChunkTokens * 4),
+               __float_as_uint(nv > 0 ? h2f(mr2.x) * mscale : mnone),
+               __float_as_uint(nv > 1 ? h2f(mr2.x >> 16) * mscale : mnone),
+               __float_as_uint(nv > 2 ? h2f(mr2.y) * mscale : mnone),
+               __float_as_uint(nv > 3 ? h2f(mr2.y >> 16) * mscale : mnone));
       }
       tmem_wait_st();
       tc_fence_before();
       async_proxy_fence();
       mbar_arrive(&sm.kv_ready[r.i]);
-
-      {
-        const int32_t q0 = __shfl_sync(0xffffffffu, bq[0], 0), q1 = __shfl_sync(0xffffffffu, bq[0], 1);
-        if (c + 1 < nchunks) load_stage(s, c + 1, q0, q1);
-      }
-      prefetch_seg(bq[4]);
-#pragma unroll
-      for (int i = 0; i < 5; ++i) bq[i] = bq[i + 1];
-      bq[5] = bid_of(c + 7);
       r.next();
     }
   } else if (warp == kMmaWarp) {
@@ -804,71 +809,53 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
     if (!sm.is_last) return;
     __threadfence();
 
-    // the last CTA of (b, h) merges the splits: (m, l) of every split into
-    // smem, merge weights per head, then every output element as a weighted
-    // sum of its nsplit partials (float4 loads, eight in flight per thread)
-    float* mls = reinterpret_cast<float*>(&sm.vt[0][0]);  // [G][nsplit] m, then l, then w
+    // the last CTA of (b, h) merges the splits: thread t owns four output
+    // dims of one head and reads that slice and (m, l) of every split in
+    // batches of eight, all loads of a batch in flight at once, merging
+    // online (max, rescale, weighted sum)
     const int ns = a.nsplit;
     const float* base = a.partials + (static_cast<int64_t>(b) * a.num_q_heads + h * G) * ns * kPartialFloats;
-    for (int t = tid; t < G * ns; t += kThreads) {
-      const float2 ml =
-          __ldcg(reinterpret_cast<const float2*>(base + static_cast<int64_t>(t) * kPartialFloats + kHeadDim));
-      mls[t] = ml.x;
-      mls[G * ns + t] = ml.y;
-    }
-    __syncthreads();
-    for (int g = warp; g < G; g += kThreads / 32) {
-      float M = -CUDART_INF_F;
-      for (int s = lane; s < ns; s += 32)
-        if (mls[G * ns + g * ns + s] > 0.0f) M = fmaxf(M, mls[g * ns + s]);
-#pragma unroll
-      for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-      float lsum = 0.0f;
-      for (int s = lane; s < ns; s += 32) {
-        const float l = mls[G * ns + g * ns + s];
-        if (l > 0.0f) lsum = fmaf(l, ex2(mls[g * ns + s] - M), lsum);
-      }
-#pragma unroll
-      for (int off = 16; off; off >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
-      const float inv = lsum > 0.0f ? 1.0f / lsum : 0.0f;
-      for (int s = lane; s < ns; s += 32) {
-        const float l = mls[G * ns + g * ns + s];
-        mls[2 * G * ns + g * ns + s] = l > 0.0f ? ex2(mls[g * ns + s] - M) * inv : 0.0f;
-      }
-    }
-    __syncthreads();
     for (int t = tid; t < G * (kHeadDim / 4); t += kThreads) {
       const int g = t / (kHeadDim / 4), q4 = t % (kHeadDim / 4);
-      const float* w = mls + 2 * G * ns + g * ns;
-      const float4* src = reinterpret_cast<const float4*>(base + static_cast<int64_t>(g) * ns * kPartialFloats) + q4;
-      constexpr int kStride = kPartialFloats / 4;
+      const float* hb = base + static_cast<int64_t>(g) * ns * kPartialFloats;
+      float M = -CUDART_INF_F, lsum = 0.0f;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      int s = 0;
-      for (; s + 8 <= ns; s += 8) {
+      for (int s0 = 0; s0 < ns; s0 += 8) {
+        float2 ml[8];
         float4 v[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) v[u] = __ldcg(src + (s + u) * kStride);
+        for (int u = 0; u < 8; ++u) {
+          const float* rec = hb + static_cast<int64_t>(min(s0 + u, ns - 1)) * kPartialFloats;
+          ml[u] = __ldcg(reinterpret_cast<const float2*>(rec + kHeadDim));
+          v[u] = __ldcg(reinterpret_cast<const float4*>(rec) + q4);
+          if (s0 + u >= ns) ml[u].y = 0.0f;  // (a repeated record, not counted)
+        }
+        float Mb = M;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (ml[u].y > 0.0f) Mb = fmaxf(Mb, ml[u].x);
+        const float f = M == -CUDART_INF_F ? 0.0f : ex2(M - Mb);
+        acc.x *= f;
+        acc.y *= f;
+        acc.z *= f;
+        acc.w *= f;
+        lsum *= f;
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          const float wu = w[s + u];
-          acc.x = fmaf(v[u].x, wu, acc.x);
-          acc.y = fmaf(v[u].y, wu, acc.y);
-          acc.z = fmaf(v[u].z, wu, acc.z);
-          acc.w = fmaf(v[u].w, wu, acc.w);
+          const float w = ml[u].y > 0.0f ? ex2(ml[u].x - Mb) : 0.0f;
+          lsum = fmaf(w, ml[u].y, lsum);
+          acc.x = fmaf(w, v[u].x, acc.x);
+          acc.y = fmaf(w, v[u].y, acc.y);
+          acc.z = fmaf(w, v[u].z, acc.z);
+          acc.w = fmaf(w, v[u].w, acc.w);
         }
+        M = Mb;
       }
-      for (; s < ns; ++s) {
-        const float4 v = __ldcg(src + s * kStride);
-        const float wu = w[s];
-        acc.x = fmaf(v.x, wu, acc.x);
-        acc.y = fmaf(v.y, wu, acc.y);
-        acc.z = fmaf(v.z, wu, acc.z);
-        acc.w = fmaf(v.w, wu, acc.w);
-      }
-      sm.obuf[g][4 * q4] = acc.x;
-      sm.obuf[g][4 * q4 + 1] = acc.y;
-      sm.obuf[g][4 * q4 + 2] = acc.z;
-      sm.obuf[g][4 * q4 + 3] = acc.w;
+      const float inv = lsum > 0.0f ? 1.0f / lsum : 0.0f;
+      sm.obuf[g][4 * q4] = acc.x * inv;
+      sm.obuf[g][4 * q4 + 1] = acc.y * inv;
+      sm.obuf[g][4 * q4 + 2] = acc.z * inv;
+      sm.obuf[g][4 * q4 + 3] = acc.w * inv;
     }
     if (tid == 0) a.tickets[b * a.num_kv_heads + h] = 0;  // ready for the next call
   }

@@ -70,9 +70,14 @@ def _run_quantize(kvq, wl, slots, k, v, pool_fill=0x5A):
     return pool.cpu().numpy()
 
 
+# The write path takes a warp per head vector for small appends (at most 1024
+# head vectors per tensor) and a thread per head vector above that; both
+# paths are covered, with ragged tails.
 @pytest.mark.parametrize("make", [lambda: synth.tiny(0),
                                   lambda: synth.Workload("q", 3, 16, 8, 128, [70, 1, 33], 16, synth.BF16, 3, 10.0,
-                                                         30.0, seed=11)])
+                                                         30.0, seed=11),
+                                  lambda: synth.Workload("qb", 2, 16, 8, 128, [70, 93], 16, synth.BF16, 3, 10.0,
+                                                         30.0, seed=14)])
 def test_quantize_matches_oracle(kvq, cuda, make):
     wl = make()
     k = wl.kv_rows(synth.TID_K, 0, wl.total_tokens)
@@ -94,11 +99,13 @@ def test_quantize_matches_oracle(kvq, cuda, make):
                 assert np.all(seg[p, :, 1024 + o * 32:1024 + (o + 1) * 32] == 0x5A)
 
 
-def test_quantize_edge_inputs(kvq, cuda):
+@pytest.mark.parametrize("n", [40, 600])
+def test_quantize_edge_inputs(kvq, cuda, n):
     """Zero vectors, one-hot vectors (flat after rotation: S = 0), skipped
-    slots, a strided (non-dense) token layout and a lone token in a block."""
+    slots, a strided (non-dense) token layout and a lone token in a block;
+    40 tokens take the small-append path, 600 the bulk path."""
     torch = _torch()
-    hkv, n = 2, 40
+    hkv = 2
     wl = synth.Workload("e", 1, 2, hkv, 128, [n], 16, synth.BF16, 3, 10.0, 30.0, seed=12, extra_blocks=2,
                         shuffle=False)
     k = wl.kv_rows(synth.TID_K, 0, n)
