@@ -337,6 +337,37 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const bool is_loader = warp < kLoadWarps;
+  const bool is_soft = warp >= kLoadWarps && warp < kMmaWarp;
+
+  // tensor memory and barriers touch no global memory: set up before
+  // waiting for the previous kernel in the stream
+  if (warp == kMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sm.tmem_base)),
+                 "n"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    if (lane == 0) {
+#pragma unroll
+      for (int i = 0; i < kNV; ++i) {
+        mbar_init(&sm.kv_ready[i], 32 * kLoadWarps);
+        mbar_init(&sm.p_ready[i], 32 * kSoftWarps);
+        mbar_init(&sm.pv_done[i], 1);
+      }
+#pragma unroll
+      for (int i = 0; i < kNS; ++i) {
+        mbar_init(&sm.qk_done[i], 1);
+        mbar_init(&sm.s_free[i], 32 * kSoftWarps);
+      }
+      mbar_init(&sm.fin, 1);
+#pragma unroll
+      for (int w = 0; w < kLoadWarps; ++w)
+#pragma unroll
+        for (int i = 0; i < kNV; ++i) mbar_init(&sm.full[w][i], 1);
+      sm.abort = 0;
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+  }
+  pdl_wait();
 
   // ---- the split: blocks [blk0, blk1) of sequence b, in chunks of 8 -------
   int L = a.seq_lens[b];
@@ -378,32 +409,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
     for (int i = 0; i < kNV; ++i) bfirst[i] = bid_of(i);
 #pragma unroll
     for (int i = 0; i < 6; ++i) bq[i] = bid_of(kNV + i);
-  } else if (warp == kMmaWarp) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sm.tmem_base)),
-                 "n"(kTmemCols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-    if (lane == 0) {
-#pragma unroll
-      for (int i = 0; i < kNV; ++i) {
-        mbar_init(&sm.kv_ready[i], 32 * kLoadWarps);
-        mbar_init(&sm.p_ready[i], 32 * kSoftWarps);
-        mbar_init(&sm.pv_done[i], 1);
-      }
-#pragma unroll
-      for (int i = 0; i < kNS; ++i) {
-        mbar_init(&sm.qk_done[i], 1);
-        mbar_init(&sm.s_free[i], 32 * kSoftWarps);
-      }
-      mbar_init(&sm.fin, 1);
-#pragma unroll
-      for (int w = 0; w < kLoadWarps; ++w)
-#pragma unroll
-        for (int i = 0; i < kNV; ++i) mbar_init(&sm.full[w][i], 1);
-      sm.abort = 0;
-      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-  } else {
+  } else if (is_soft) {
     // rotate the G query heads (warp sw: heads sw, sw + 4), then write their
     // digits with one c1 for all heads
     const int sw = warp - kLoadWarps;
@@ -780,6 +786,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
   tc_fence_after();
   if (warp == kMmaWarp)  // every MMA and tensor-memory load is complete
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "n"(kTmemCols));
+  pdl_trigger();  // this CTA holds no tensor memory any more
   __syncthreads();
 
   // ---- 2. partial record, ticket, merge -------------------------------------
@@ -878,8 +885,7 @@ cudaError_t launch_g(const DecodeArgs& a, cudaStream_t stream) {
   const cudaError_t e = ensure_smem_limit<decode_kernel<G>>(kSmemBytes);
   if (e != cudaSuccess) return e;
   const dim3 grid(a.nsplit, a.num_kv_heads, a.batch);
-  decode_kernel<G><<<grid, kThreads, kSmemBytes, stream>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(decode_kernel<G>, grid, dim3(kThreads), kSmemBytes, stream, a);
 }
 
 }  // namespace

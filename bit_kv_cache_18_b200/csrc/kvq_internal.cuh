@@ -62,6 +62,32 @@ __device__ __forceinline__ void store_from_f32(void* p, int dtype, int64_t i, fl
     static_cast<__half*>(p)[i] = __float2half_rn(v);
 }
 
+// ---- programmatic dependent launch ------------------------------------------
+// Every kernel here is launched with programmatic stream serialization: it
+// may become resident while the kernel before it in the stream is still
+// finishing.  It executes pdl_wait() before it reads or writes any memory
+// that an earlier kernel may touch (inputs, pool, workspace, outputs), and
+// pdl_trigger() once it holds no resource a still-unlaunched CTA of its own
+// grid could need (tensor memory), which lets the next kernel's CTAs set up.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // ---- launchers (return cudaError_t of the launch) ---------------------------
 struct QuantizeArgs {
   uint8_t* pool;

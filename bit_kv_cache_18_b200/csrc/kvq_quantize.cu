@@ -305,6 +305,8 @@ __global__ void __launch_bounds__(kWarps * 32)
                     const uint8_t* __restrict__ k, const uint8_t* __restrict__ v,
                     int32_t n_tokens, int64_t stride_bytes, const int32_t* __restrict__ slots, int* status) {
   extern __shared__ __align__(16) uint8_t smem[];
+  pdl_trigger();  // (the grid is persistent: every CTA is resident at once)
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const uint32_t buf0 = smem_u32(smem + warp * 2 * kTileBytes);
@@ -382,6 +384,8 @@ __global__ void __launch_bounds__(kSmallWarps * 32)
     quantize_small_kernel(uint8_t* __restrict__ pool, int32_t num_blocks, int32_t hkv,
                           const uint8_t* __restrict__ k, const uint8_t* __restrict__ v, int32_t n_tokens,
                           int64_t stride_bytes, const int32_t* __restrict__ slots, int* status) {
+  pdl_trigger();  // (the whole grid is resident at once)
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t n_vec = static_cast<int64_t>(n_tokens) * hkv;
   const int64_t w = static_cast<int64_t>(blockIdx.x) * kSmallWarps + (threadIdx.x >> 5);
@@ -492,13 +496,13 @@ cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream) {
   if (n_vec <= kSmallMaxVecs) {
     const unsigned grid = static_cast<unsigned>((2 * n_vec + kSmallWarps - 1) / kSmallWarps);
     if (a.in_dtype == KVQ_BF16)
-      quantize_small_kernel<true><<<grid, kSmallWarps * 32, 0, stream>>>(
-          a.pool, a.num_blocks, a.num_kv_heads, static_cast<const uint8_t*>(a.k),
-          static_cast<const uint8_t*>(a.v), a.n_tokens, stride_bytes, a.slots, a.status);
+      return launch_pdl(quantize_small_kernel<true>, dim3(grid), dim3(kSmallWarps * 32), 0, stream, a.pool,
+                        a.num_blocks, a.num_kv_heads, static_cast<const uint8_t*>(a.k),
+                        static_cast<const uint8_t*>(a.v), a.n_tokens, stride_bytes, a.slots, a.status);
     else
-      quantize_small_kernel<false><<<grid, kSmallWarps * 32, 0, stream>>>(
-          a.pool, a.num_blocks, a.num_kv_heads, static_cast<const uint8_t*>(a.k),
-          static_cast<const uint8_t*>(a.v), a.n_tokens, stride_bytes, a.slots, a.status);
+      return launch_pdl(quantize_small_kernel<false>, dim3(grid), dim3(kSmallWarps * 32), 0, stream, a.pool,
+                        a.num_blocks, a.num_kv_heads, static_cast<const uint8_t*>(a.k),
+                        static_cast<const uint8_t*>(a.v), a.n_tokens, stride_bytes, a.slots, a.status);
     return cudaGetLastError();
   }
   const int64_t tiles = 2 * ((n_vec + kRows - 1) / kRows);
@@ -510,15 +514,15 @@ cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream) {
   if (a.in_dtype == KVQ_BF16) {
     const cudaError_t e = ensure_smem_limit<quantize_kernel<true>>(smem);
     if (e != cudaSuccess) return e;
-    quantize_kernel<true><<<static_cast<unsigned>(grid), kWarps * 32, smem, stream>>>(
-        a.pool, a.num_blocks, a.num_kv_heads, static_cast<const uint8_t*>(a.k),
-        static_cast<const uint8_t*>(a.v), a.n_tokens, stride_bytes, a.slots, a.status);
+    return launch_pdl(quantize_kernel<true>, dim3(static_cast<unsigned>(grid)), dim3(kWarps * 32), smem, stream,
+                      a.pool, a.num_blocks, a.num_kv_heads, static_cast<const uint8_t*>(a.k),
+                      static_cast<const uint8_t*>(a.v), a.n_tokens, stride_bytes, a.slots, a.status);
   } else {
     const cudaError_t e = ensure_smem_limit<quantize_kernel<false>>(smem);
     if (e != cudaSuccess) return e;
-    quantize_kernel<false><<<static_cast<unsigned>(grid), kWarps * 32, smem, stream>>>(
-        a.pool, a.num_blocks, a.num_kv_heads, static_cast<const uint8_t*>(a.k),
-        static_cast<const uint8_t*>(a.v), a.n_tokens, stride_bytes, a.slots, a.status);
+    return launch_pdl(quantize_kernel<false>, dim3(static_cast<unsigned>(grid)), dim3(kWarps * 32), smem, stream,
+                      a.pool, a.num_blocks, a.num_kv_heads, static_cast<const uint8_t*>(a.k),
+                      static_cast<const uint8_t*>(a.v), a.n_tokens, stride_bytes, a.slots, a.status);
   }
   return cudaGetLastError();
 }
