@@ -73,6 +73,9 @@ def lib():
                                                            vp, ctypes.c_int, vp, sz, i32, vp]),
                 "kvq_decode_attention_noalloc": (ctypes.c_int, [dp, vp, ctypes.c_int, i32, i32, vp, i32, vp, i32, f32,
                                                                 vp, ctypes.c_int, vp]),
+                "kvq_append_decode_attention": (ctypes.c_int, [dp, vp, vp, ctypes.c_int, i64, vp, ctypes.c_int, i32,
+                                                               i32, vp, i32, vp, i32, f32, vp, ctypes.c_int, vp, sz,
+                                                               vp]),
                 "kvq_last_device_status": (ctypes.c_int, [vp]),
                 "kvq_error_string": (ctypes.c_char_p, [ctypes.c_int]),
             }
@@ -199,6 +202,22 @@ def kvq_decode_attention(pool, num_blocks, num_kv_heads, q, block_table, seq_len
                                        _dtype_code(out), _ptr(workspace), workspace.numel(), blocks_per_split,
                                        _stream_ptr(stream))
     _check(rc, "kvq_decode_attention")
+
+
+def kvq_append_decode_attention(pool, num_blocks, num_kv_heads, k_new, v_new, q, block_table, seq_lens, max_seq_len,
+                                out, workspace, softmax_scale=0.0, stream=None, token_stride=None):
+    """One fused decode step: the new token of each sequence (k_new, v_new:
+    [batch, ..., Hkv*128] fp16/bf16 rows) is quantized into position
+    seq_lens[b] - 1, then decode attention runs over the grown cache."""
+    desc = make_desc(num_blocks, num_kv_heads, pool)
+    batch, hq, _ = q.shape
+    ts = k_new.stride(0) if token_stride is None else token_stride
+    rc = lib().kvq_append_decode_attention(ctypes.byref(desc), _ptr(k_new), _ptr(v_new), _dtype_code(k_new), ts,
+                                           _ptr(q), _dtype_code(q), batch, hq, _ptr(block_table),
+                                           block_table.shape[1], _ptr(seq_lens), max_seq_len, softmax_scale,
+                                           _ptr(out), _dtype_code(out), _ptr(workspace), workspace.numel(),
+                                           _stream_ptr(stream))
+    _check(rc, "kvq_append_decode_attention")
 
 
 def kvq_decode_attention_noalloc(pool, num_blocks, num_kv_heads, q, block_table, seq_lens, max_seq_len, out,

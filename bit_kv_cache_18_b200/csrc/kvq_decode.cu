@@ -410,10 +410,32 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
 #pragma unroll
     for (int i = 0; i < 6; ++i) bq[i] = bid_of(kNV + i);
   } else if (is_soft) {
-    // rotate the G query heads (warp sw: heads sw, sw + 4), then write their
-    // digits with one c1 for all heads
     const int sw = warp - kLoadWarps;
     const int stok = tid - 32 * kLoadWarps;
+    // fused one-token append: the split holding position L-1 first writes the
+    // new token's K (warp 4) and V (warp 5) of kv head h into that position,
+    // before any loader reads the block (the proxy fence and the set-up
+    // barrier below order the writes before the bulk copies)
+    if (a.k_new != nullptr && sw < 2 && L > 0) {
+      const int blk_new = (L - 1) / kBlockSize;
+      if (blk_new >= blk0 && blk_new < blk1) {
+        const int32_t p = bt_row[blk_new];
+        if (p >= 0 && p < a.num_blocks) {
+          uint8_t* seg = const_cast<uint8_t*>(pool_h) + static_cast<int64_t>(p) * pstride;
+          const uint8_t* src = (sw ? a.v_new : a.k_new) + static_cast<int64_t>(b) * a.new_stride_bytes +
+                               static_cast<int64_t>(h) * (kHeadDim * 2);
+          if (a.new_bf16)
+            quantize_vector_warp<true>(src, seg, (L - 1) % kBlockSize, sw == 1, lane);
+          else
+            quantize_vector_warp<false>(src, seg, (L - 1) % kBlockSize, sw == 1, lane);
+          asm volatile("fence.proxy.async.global;" ::: "memory");
+        } else if (lane == 0) {
+          record_status(a.status, KVQ_ERR_OUT_OF_RANGE);
+        }
+      }
+    }
+    // rotate the G query heads (warp sw: heads sw, sw + 4), then write their
+    // digits with one c1 for all heads
     reinterpret_cast<uint4*>(sm.qb)[stok] = make_uint4(0, 0, 0, 0);
     reinterpret_cast<uint4*>(sm.qb)[stok + 128] = make_uint4(0, 0, 0, 0);
     float x[2][4];

@@ -288,12 +288,19 @@ size_t kvq_decode_workspace_bytes(const kvq_cache_desc* desc, int32_t batch, int
   return kvq_decode_workspace_bytes_ex(desc, batch, num_q_heads, max_seq_len, 0);
 }
 
-int kvq_decode_attention_ex(const kvq_cache_desc* desc, const void* q, kvq_dtype q_dtype,
-                            int32_t batch, int32_t num_q_heads, const int32_t* block_table,
-                            int32_t max_blocks_per_seq, const int32_t* seq_lens,
-                            int32_t max_seq_len, float softmax_scale, void* out,
-                            kvq_dtype out_dtype, void* workspace, size_t ws_bytes,
-                            int32_t blocks_per_split, void* stream) {
+namespace {
+// The new-token rows of a fused append + decode call.
+struct AppendRows {
+  const void* k;
+  const void* v;
+  kvq_dtype dtype;
+  int64_t token_stride;
+};
+
+int decode_impl(const kvq_cache_desc* desc, const void* q, kvq_dtype q_dtype, int32_t batch, int32_t num_q_heads,
+                const int32_t* block_table, int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                int32_t max_seq_len, float softmax_scale, void* out, kvq_dtype out_dtype, void* workspace,
+                size_t ws_bytes, int32_t blocks_per_split, void* stream, const AppendRows* app) {
   int rc = check_desc(desc);
   if (rc != KVQ_OK) return rc;
   if (batch < 0 || num_q_heads <= 0 || max_blocks_per_seq < 0 || max_seq_len < 0 ||
@@ -333,8 +340,41 @@ int kvq_decode_attention_ex(const kvq_cache_desc* desc, const void* q, kvq_dtype
   a.blocks_per_split = plan.blocks_per_split;
   a.nsplit = plan.nsplit;
   a.status = device_status_ptr();
+  a.k_new = app ? static_cast<const uint8_t*>(app->k) : nullptr;
+  a.v_new = app ? static_cast<const uint8_t*>(app->v) : nullptr;
+  a.new_bf16 = app && app->dtype == KVQ_BF16 ? 1 : 0;
+  a.new_stride_bytes = app ? app->token_stride * 2 : 0;
   if (!a.status) return KVQ_ERR_CUDA;
   return launch_decode(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+}  // namespace
+
+int kvq_decode_attention_ex(const kvq_cache_desc* desc, const void* q, kvq_dtype q_dtype,
+                            int32_t batch, int32_t num_q_heads, const int32_t* block_table,
+                            int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                            int32_t max_seq_len, float softmax_scale, void* out,
+                            kvq_dtype out_dtype, void* workspace, size_t ws_bytes,
+                            int32_t blocks_per_split, void* stream) {
+  return decode_impl(desc, q, q_dtype, batch, num_q_heads, block_table, max_blocks_per_seq, seq_lens, max_seq_len,
+                     softmax_scale, out, out_dtype, workspace, ws_bytes, blocks_per_split, stream, nullptr);
+}
+
+int kvq_append_decode_attention(const kvq_cache_desc* desc, const void* k_new, const void* v_new,
+                                kvq_dtype in_dtype, int64_t token_stride, const void* q,
+                                kvq_dtype q_dtype, int32_t batch, int32_t num_q_heads,
+                                const int32_t* block_table, int32_t max_blocks_per_seq,
+                                const int32_t* seq_lens, int32_t max_seq_len, float softmax_scale,
+                                void* out, kvq_dtype out_dtype, void* workspace, size_t ws_bytes,
+                                void* stream) {
+  const int rc = check_desc(desc);
+  if (rc != KVQ_OK) return rc;
+  if (in_dtype != KVQ_F16 && in_dtype != KVQ_BF16) return KVQ_ERR_INVALID;
+  if (batch > 0 && (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new))) return KVQ_ERR_INVALID;
+  if (token_stride < static_cast<int64_t>(desc->num_kv_heads) * kHeadDim || token_stride % 8 != 0)
+    return KVQ_ERR_INVALID;
+  const AppendRows app{k_new, v_new, in_dtype, token_stride};
+  return decode_impl(desc, q, q_dtype, batch, num_q_heads, block_table, max_blocks_per_seq, seq_lens, max_seq_len,
+                     softmax_scale, out, out_dtype, workspace, ws_bytes, 0, stream, &app);
 }
 
 int kvq_decode_attention(const kvq_cache_desc* desc, const void* q, kvq_dtype q_dtype, int32_t batch,

@@ -369,13 +369,7 @@ __global__ void __launch_bounds__(kWarps * 32)
 
 
 // ---- small appends (a few tokens per call, as in decode) --------------------
-// One warp per 128-element vector: lane l holds elements 4l .. 4l+3, so the
-// two lowest butterfly stages run in registers and the five others by
-// shuffles; the statistics are warp reductions.  The arithmetic is that of
-// quantize_store (moments of y = sqrt(128) r, fp16 S and Z, codes from the
-// stored S and Z), only the summation order differs.  Each lane then owns
-// whole bytes of the packed row: two bytes of 4-bit key codes or one byte of
-// 2-bit value codes.
+// One warp per head vector (quantize_vector_warp in kvq_internal.cuh).
 constexpr int kSmallWarps = 4;
 constexpr int64_t kSmallMaxVecs = 1024;  // at most this many head vectors per tensor
 
@@ -404,87 +398,8 @@ __global__ void __launch_bounds__(kSmallWarps * 32)
   const int row_in_block = slot % kBlockSize;
   uint8_t* seg = pool + (static_cast<int64_t>(p) * hkv + h) * kSegBytes;
 
-  // elements 4 lane .. 4 lane + 3 (8 bytes)
-  const uint8_t* src = (is_v ? v : k) + tok * stride_bytes + static_cast<int64_t>(h) * (kHeadDim * 2);
-  const uint2 raw = *reinterpret_cast<const uint2*>(src + 8 * lane);
-  float y[4];
-  if (kBF16) {
-    y[0] = bf16lo_to_f32(raw.x);
-    y[1] = bf16hi_to_f32(raw.x);
-    y[2] = bf16lo_to_f32(raw.y);
-    y[3] = bf16hi_to_f32(raw.y);
-  } else {
-    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
-    const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
-    y[0] = a.x;
-    y[1] = a.y;
-    y[2] = b.x;
-    y[3] = b.y;
-  }
-  // Walsh-Hadamard butterflies (unnormalised): strides 1, 2 in registers,
-  // strides 4 .. 64 across lanes (the lower index keeps u + v)
-  {
-    const float a0 = y[0] + y[1], a1 = y[0] - y[1], a2 = y[2] + y[3], a3 = y[2] - y[3];
-    y[0] = a0 + a2;
-    y[1] = a1 + a3;
-    y[2] = a0 - a2;
-    y[3] = a1 - a3;
-  }
-#pragma unroll
-  for (int st = 1; st < 32; st <<= 1) {
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float o = __shfl_xor_sync(0xffffffffu, y[j], st);
-      y[j] = (lane & st) ? o - y[j] : y[j] + o;
-    }
-  }
-  float sum = (y[0] + y[1]) + (y[2] + y[3]);
-  float sq = fmaf(y[0], y[0], fmaf(y[1], y[1], fmaf(y[2], y[2], y[3] * y[3])));
-  float ymin = fminf(fminf(y[0], y[1]), fminf(y[2], y[3]));
-  float ymax = fmaxf(fmaxf(y[0], y[1]), fmaxf(y[2], y[3]));
-#pragma unroll
-  for (int o = 16; o; o >>= 1) {
-    sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    sq += __shfl_xor_sync(0xffffffffu, sq, o);
-    ymin = fminf(ymin, __shfl_xor_sync(0xffffffffu, ymin, o));
-    ymax = fmaxf(ymax, __shfl_xor_sync(0xffffffffu, ymax, o));
-  }
-  const float levels = is_v ? static_cast<float>((1 << kVBits) - 1) : static_cast<float>((1 << kKBits) - 1);
-  constexpr float kInvSqrtD = 0.088388347648318440550f;
-  const float mean = sum * (1.0f / kHeadDim);
-  const float var = fmaxf(sq * (1.0f / kHeadDim) - mean * mean, 0.0f);
-  float sigma = sqrtf(var);
-  if (sigma == 0.0f) sigma = 1.0f;
-  const float lo = (ymin - mean) / sigma;
-  const float hi = (ymax - mean) / sigma;
-  const __half Sh = __float2half_rn(kInvSqrtD * (sigma * (hi - lo)) / levels);
-  const __half Zh = __float2half_rn(kInvSqrtD * (mean + sigma * lo));
-  const float Sf = __half2float(Sh);
-  const float Zf = __half2float(Zh);
-  uint32_t c[4] = {0u, 0u, 0u, 0u};
-  if (Sf != 0.0f) {
-    const float a = kInvSqrtD / Sf;
-    const float b = -Zf / Sf;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float t = fminf(fmaxf(fmaf(y[j], a, b), 0.0f), levels);
-      c[j] = __float_as_uint(t + kMagic) & 0xFFu;
-    }
-  }
-  if (is_v) {
-    seg[kOffV + row_in_block * kVRowBytes + lane] = static_cast<uint8_t>(c[0] | c[1] << 2 | c[2] << 4 | c[3] << 6);
-    if (lane == 0) {
-      reinterpret_cast<__half*>(seg + kOffSV)[row_in_block] = Sh;
-      reinterpret_cast<__half*>(seg + kOffZV)[row_in_block] = Zh;
-    }
-  } else {
-    reinterpret_cast<uint16_t*>(seg + kOffK + row_in_block * kKRowBytes)[lane] =
-        static_cast<uint16_t>(c[0] | c[1] << 4 | c[2] << 8 | c[3] << 12);
-    if (lane == 0) {
-      reinterpret_cast<__half*>(seg + kOffSK)[row_in_block] = Sh;
-      reinterpret_cast<__half*>(seg + kOffZK)[row_in_block] = Zh;
-    }
-  }
+  quantize_vector_warp<kBF16>((is_v ? v : k) + tok * stride_bytes + static_cast<int64_t>(h) * (kHeadDim * 2), seg,
+                              row_in_block, is_v, lane);
 }
 
 }  // namespace

@@ -179,6 +179,28 @@ int kvq_decode_attention_ex(const kvq_cache_desc* desc, const void* q, kvq_dtype
                             kvq_dtype out_dtype, void* workspace, size_t ws_bytes,
                             int32_t blocks_per_split, void* stream);
 
+/* One decode step of a cache that grows by one token per sequence: for each
+ * sequence b with L = seq_lens[b] > 0, the new token's K and V rows (k_new,
+ * v_new: device, row b at element b*token_stride, [num_kv_heads, 128] of
+ * in_dtype F16 or BF16, 16-byte aligned, token_stride a multiple of 8 and
+ * >= num_kv_heads*128) are quantized into position L-1, i.e. slot
+ * block_table[b][(L-1)/16]*16 + (L-1)%16 -- the bytes kvq_quantize_append
+ * writes for that slot -- and then the decode attention of
+ * kvq_decode_attention runs over positions 0 .. L-1, the new token included.
+ * One kernel launch: the CTA whose split holds position L-1 writes the new
+ * row before it reads that block.  The same arguments, workspace and status
+ * rules as kvq_decode_attention; the new token's block must not be read by
+ * another sequence of the same call.  Follows the KVarN write path (Hadamard
+ * rotation, variance normalisation, asymmetric RTN) and read path (scale
+ * folding at read time) of "KVarN vs TurboQuant" (dothoosh.com). */
+int kvq_append_decode_attention(const kvq_cache_desc* desc, const void* k_new, const void* v_new,
+                                kvq_dtype in_dtype, int64_t token_stride, const void* q,
+                                kvq_dtype q_dtype, int32_t batch, int32_t num_q_heads,
+                                const int32_t* block_table, int32_t max_blocks_per_seq,
+                                const int32_t* seq_lens, int32_t max_seq_len, float softmax_scale,
+                                void* out, kvq_dtype out_dtype, void* workspace, size_t ws_bytes,
+                                void* stream);
+
 /* kvq_decode_attention without a caller-provided workspace, for callers that
  * cannot allocate device memory at call time: code that runs inside a memory
  * pool or allocator that forbids runtime allocations, embedded or plugin

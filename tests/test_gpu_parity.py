@@ -183,6 +183,19 @@ def test_decode_ragged_gqa8(kvq, cuda, bps):
     assert not got[5].any()  # length 0 -> zeros
 
 
+@pytest.mark.parametrize("bps", [1, 2])
+def test_decode_many_splits(kvq, cuda, bps):
+    """More splits than one thread-block cluster holds (clusters of 16 merge
+    through distributed shared memory, then across clusters through the
+    workspace), with empty splits and whole empty clusters."""
+    wl = synth.Workload("m", 3, 16, 2, 128, [400, 33, 0], 16, synth.BF16, 3, 10.0, 30.0, seed=23, extra_blocks=2)
+    g, pool, _, _ = _oracle_pool(wl)
+    q = wl.query()
+    got, _ = _gpu_decode(kvq, wl, pool, q, wl.dtype, bps=bps)
+    _check_decode(wl, g, pool, q, wl.dtype, got)
+    assert not got[2].any()
+
+
 @pytest.mark.parametrize("G", [1, 2, 4])
 def test_decode_group_sizes(kvq, cuda, G):
     wl = synth.Workload("g", 2, 4 * G, 4, 128, [129, 47], 16, synth.F16, 4, 20.0, 20.0, seed=30 + G)
@@ -201,6 +214,60 @@ def test_decode_dtypes(kvq, cuda, q_dtype, out_dtype, rel):
     got, _ = _gpu_decode(kvq, wl, pool, q, q_dtype, out_dtype=out_dtype)
     # bf16/f16 outputs carry their own rounding on top of the 2e-3 kernel bound
     _check_decode(wl, g, pool, q, q_dtype, got, rel=rel)
+
+
+def test_append_decode_matches_append_then_decode(kvq, cuda):
+    """The fused one-step call writes the same pool bytes as the write path
+    followed by the read path, gives the same outputs, and both agree with
+    the oracle (codes: near-tie rules; outputs: 2e-3 on the same codes)."""
+    torch = _torch()
+    wl = synth.Workload("ad", 4, 16, 2, 128, [70, 1, 33, 0], 16, synth.BF16, 3, 10.0, 30.0, seed=25,
+                        extra_blocks=2)
+    T = wl.total_tokens
+    k = wl.kv_rows(synth.TID_K, 0, T)
+    v = wl.kv_rows(synth.TID_V, 0, T)
+    slots = wl.slots()
+    last = np.array([int(wl.token_offsets[b]) + int(wl.seq_lens[b]) - 1 for b in range(wl.batch)
+                     if wl.seq_lens[b] > 0])
+    keep = np.setdiff1d(np.arange(T), last)
+    g = oracle.geom(num_blocks=wl.num_blocks, num_kv_heads=wl.hkv)
+    base = oracle.new_pool(g, fill=0x5A)
+    assert oracle.quantize_append(g, base, np.ascontiguousarray(k[keep]), np.ascontiguousarray(v[keep]), wl.dtype,
+                                  slots[keep]) == 0
+    # new rows per sequence (zeros for the empty sequence, which appends nothing)
+    kn = np.zeros((wl.batch, wl.hkv, 128), np.uint16)
+    vn = np.zeros((wl.batch, wl.hkv, 128), np.uint16)
+    for b in range(wl.batch):
+        if wl.seq_lens[b] > 0:
+            t = int(wl.token_offsets[b]) + int(wl.seq_lens[b]) - 1
+            kn[b], vn[b] = k[t], v[t]
+    q = wl.query()
+    qd = _dev_u16(q, wl.dtype)
+    bt = torch.from_numpy(wl.block_table).cuda()
+    sl = torch.from_numpy(wl.seq_lens).cuda()
+    msl = int(wl.seq_lens.max())
+    ws = kvq.new_workspace(wl.num_blocks, wl.hkv, wl.batch, wl.hq, msl)
+    # two calls: write path, then read path
+    pool1 = torch.from_numpy(base.copy()).cuda()
+    kvq.kvq_quantize_append(pool1, wl.num_blocks, wl.hkv, _dev_u16(k[last], wl.dtype).reshape(len(last), -1),
+                            _dev_u16(v[last], wl.dtype).reshape(len(last), -1),
+                            torch.from_numpy(slots[last].copy()).cuda())
+    out1 = torch.empty((wl.batch, wl.hq, 128), dtype=torch.float32, device="cuda")
+    kvq.kvq_decode_attention(pool1, wl.num_blocks, wl.hkv, qd, bt, sl, msl, out1, ws)
+    # one fused call
+    pool2 = torch.from_numpy(base.copy()).cuda()
+    out2 = torch.empty_like(out1)
+    kvq.kvq_append_decode_attention(pool2, wl.num_blocks, wl.hkv, _dev_u16(kn, wl.dtype).reshape(wl.batch, -1),
+                                    _dev_u16(vn, wl.dtype).reshape(wl.batch, -1), qd, bt, sl, msl, out2, ws)
+    assert kvq.kvq_last_device_status() == 0
+    p1, p2 = pool1.cpu().numpy(), pool2.cpu().numpy()
+    assert np.array_equal(p1, p2)
+    assert torch.equal(out1, out2)
+    rep = helpers.QuantReport()
+    helpers.check_pool_tokens(rep, p2, wl.num_blocks, wl.hkv, k, v, wl.dtype, slots, last)
+    assert rep.ok(), rep
+    _check_decode(wl, g, p2, q, wl.dtype, out2.cpu().numpy().astype(np.float64))
+    assert not out2[3].any()
 
 
 def test_decode_workspace_is_reusable(kvq, cuda):
