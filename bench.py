@@ -51,18 +51,26 @@ BYTES_PER_TOKEN_HEAD = 104
 # DRAM bytes (read + write) of one decode launch on the Qwen3-32B layer
 # workload, from `ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum`
 # (cache control on: every replay starts cold, as every launch of the step
-# does), with the SHA-256 of the kernel source it was taken on.  Reported as
-# roofline.traffic only while the source still has that hash.
-DECODE_TRAFFIC = {"sha256": "84ff6e79ccd98272e68268f7313411d19e224ec13df74fe51ee03b70445368f4",
+# does), with the SHA-256 of the kernel code it was taken on (decode_code_sha256:
+# comments stripped).  Reported as roofline.traffic only while the code still
+# has that hash.
+DECODE_TRAFFIC = {"sha256": "3ba1317c4c2f07495b25bdddda1b3b934a72b4edec1735d8791ced7af0389c9d",
                   "bytes": 13764096}
 
 
-def decode_traffic():
+def decode_code_sha256():
+    """SHA-256 of the decode kernel source with // comments and blank lines
+    removed (a comment edit does not change the kernel)."""
     import hashlib
+    import re
     path = os.path.join(ROOT, "bit_kv_cache_18_b200", "csrc", "kvq_decode.cu")
-    with open(path, "rb") as f:
-        sha = hashlib.sha256(f.read()).hexdigest()
-    return DECODE_TRAFFIC["bytes"] if sha == DECODE_TRAFFIC["sha256"] else None
+    with open(path) as f:
+        lines = [re.sub(r"\s*//.*$", "", ln).rstrip() for ln in f]
+    return hashlib.sha256("\n".join(ln for ln in lines if ln).encode()).hexdigest()
+
+
+def decode_traffic():
+    return DECODE_TRAFFIC["bytes"] if decode_code_sha256() == DECODE_TRAFFIC["sha256"] else None
 
 
 def measured_peaks():

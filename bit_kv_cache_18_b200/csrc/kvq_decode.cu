@@ -3,27 +3,30 @@
 // integer arithmetic.
 //
 // One CTA owns one (sequence b, kv head h, split of the context) and walks
-// the split in chunks of 8 blocks = 128 tokens.  Two kinds of warps work on
+// the split in chunks of 8 blocks = 128 tokens.  Three kinds of warps work on
 // different chunks at the same time and hand buffers to each other through
-// mbarrier rings:
+// mbarrier rings of depth kNV:
 //   * loader warps 0-3 (thread t <-> token t of a chunk <-> TMEM lane t):
-//     bring their two segments of each chunk into a private three-slot
+//     bring their two segments of each chunk into a private kNV-slot
 //     shared-memory ring with bulk copies (TMA, one instruction per segment)
-//     three chunks ahead, after an L2 prefetch six chunks ahead;
-//     spread the 4-bit key codes to one byte each into tensor memory (A of
-//     QK) and the 2-bit value codes to one byte each into shared memory (A of
-//     PV), and publish the per-token factors;
+//     kNV chunks ahead, after an L2 prefetch six chunks ahead; read them
+//     with conflict-free 16-byte loads; spread the 4-bit key codes to one
+//     byte each into tensor memory (A of QK, 16x256b stores whose fragment
+//     layout matches the 16-byte pieces) and the 2-bit value codes to one
+//     byte each into shared memory (A of PV), and publish the per-token
+//     factors;
+//   * one MMA warp (tensor-memory owner) whose lane 0 issues, in order,
+//     QK(0), QK(1), PV(0), QK(2), PV(1), ... as tcgen05.mma (M = 128, N = 32):
+//       QK:  S  = codes_K (128 tok x 128) . digits(q~)^T  (u8 x s8 -> s32)
+//       PV:  O += codes_V^T (128 pos x 128 tok) . digits(P') (u8 x u8 -> s32)
 //   * softmax warps 4-7 (thread t <-> token t of S, value position t of O):
 //     read a token's row of S, form the base-2 score of each of the G heads
 //       s_g = S_K,t c1 (S0 + S1/254 + S2/254^2) + Z_K,t sum(q~_g),
 //     the probability p = 2^(s_g - m_g) and P'_g = p S_V,t as a 30-bit fixed
 //     point whose four bytes are four u8 digit columns of the PV operand,
-//     and keep l_g = sum p and zeta_g = sum p Z_V in registers.  One lane of
-//     warp 4 issues every tensor-core instruction:
-//       QK:  S  = codes_K (128 tok x 128) . digits(q~)^T  (u8 x s8 -> s32)
-//       PV:  O += codes_V^T (128 pos x 128 tok) . digits(P') (u8 x u8 -> s32)
-//     (tcgen05.mma, M = 128, N = 32): the QK of chunk c+2 as soon as the four
-//     warps have read S of chunk c, the PV of chunk c once its P' is written.
+//     and keep l_g = sum p and zeta_g = sum p Z_V in registers.
+// For the fused decode step the softmax warps of the CTA whose split holds
+// position L-1 first quantize the new token's K and V into that position.
 // Before the scan the softmax warps rotate the G query heads once (warp
 // FWHT, softmax scale times log2(e) folded in) and write q~ as three signed
 // 8-bit digits, q~/c1 = Q0 + Q1/254 + Q2/254^2 with c1 = max|q~|/127.  After
@@ -54,8 +57,8 @@
 // chunks, which keeps every s32 sum below 2^31.
 //
 // Code order.  The byte spreading permutes the 128 positions of a row
-// (keys: position 8i + 4h + j holds dim 8i + 2j + h; values: position
-// 16i + 4k + j holds dim 16i + 4j + k, times 4^k).  The query digits are
+// (keys: position 32j + 8m + 4h + b holds dim 32m + 8j + 2b + h; values:
+// position 16i + 4k + j holds dim 16i + 4j + k, times 4^k).  The query digits are
 // written in the key order, so S is exact, and the output rows are put back
 // in dim order, and divided by 4^k, when O is read.
 #include <math_constants.h>
