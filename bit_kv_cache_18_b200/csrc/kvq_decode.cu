@@ -362,10 +362,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
         mbar_init(&sm.s_free[i], 32 * kSoftWarps);
       }
       mbar_init(&sm.fin, 1);
-#pragma unroll
-      for (int w = 0; w < kLoadWarps; ++w)
-#pragma unroll
-        for (int i = 0; i < kNV; ++i) mbar_init(&sm.full[w][i], 1);
       sm.abort = 0;
       asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -373,6 +369,21 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
   pdl_wait();
 
   // ---- the split: blocks [blk0, blk1) of sequence b, in chunks of 8 -------
+  // Loader warp w owns blocks 2w and 2w+1 of every chunk (tokens 32w ..
+  // 32w + 31 = TMEM lanes of its quarter); its lanes read the block ids of
+  // segment lane & 1 of chunks 0 .. 8 at once, before the sequence length
+  // is known (every entry of the row is in bounds), and cut them to the
+  // split below.
+  const int blk0 = split * a.blocks_per_split;
+  const int32_t* bt_row = a.block_table + static_cast<int64_t>(b) * a.max_blocks_per_seq;
+  int32_t braw[kNV + 6];
+  if (is_loader) {
+#pragma unroll
+    for (int i = 0; i < kNV + 6; ++i) {
+      const int blk = blk0 + kChunkBlocks * i + 2 * warp + (lane & 1);
+      braw[i] = blk < a.max_blocks_per_seq ? __ldg(bt_row + blk) : -1;
+    }
+  }
   int L = a.seq_lens[b];
   if (L < 0 || L > a.max_seq_len || L > a.max_blocks_per_seq * kBlockSize) {
     if (tid == 0) record_status(a.status, KVQ_ERR_OUT_OF_RANGE);
@@ -381,16 +392,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
     L = min(L, a.max_blocks_per_seq * kBlockSize);
   }
   const int nb = (L + kBlockSize - 1) / kBlockSize;
-  const int blk0 = split * a.blocks_per_split;
   const int blk1 = min(nb, blk0 + a.blocks_per_split);
   const int nchunks = blk1 > blk0 ? (blk1 - blk0 + kChunkBlocks - 1) / kChunkBlocks : 0;
   bool bad = false;      // a wait ran out: the results are void, the control flow is kept
   bool bad_blk = false;  // a block-table entry outside the pool (its tokens are skipped)
 
-  // loader warp w owns blocks 2w and 2w+1 of every chunk (tokens 32w ..
-  // 32w + 31 = TMEM lanes of its quarter); lanes 0 and 1 keep the block
-  // ids of segment lane & 1
-  const int32_t* bt_row = a.block_table + static_cast<int64_t>(b) * a.max_blocks_per_seq;
   const uint8_t* pool_h = a.pool + static_cast<int64_t>(h) * kSegBytes;
   const int64_t pstride = static_cast<int64_t>(a.num_kv_heads) * kSegBytes;
   const int mseg = lane >> 4;  // segment of my factor bytes
@@ -403,15 +409,55 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
   auto prefetch_seg = [&](int32_t p) {
     if (lane < 2 && p >= 0 && p < a.num_blocks) prefetch_l2(pool_h + static_cast<int64_t>(p) * pstride, kSegBytes);
   };
+  const uint32_t my_stg = smem_u32(sm.stg[warp < kLoadWarps ? warp : 0][0]);
+  // lanes 0 and 1: bulk copy of segment lane & 1 of chunk c (block p) into
+  // staging slot `slot`; every lane gets the pair of segment flags
+  // (bit s: segment s is inside the split and the pool)
+  auto issue = [&](int c, int32_t p, int slot) -> uint32_t {
+    const int blk = blk0 + kChunkBlocks * c + 2 * warp + (lane & 1);
+    const bool live = blk < blk1;
+    const bool ok = live && p >= 0 && p < a.num_blocks;
+    if (lane < 2) {
+      bad_blk |= live && !ok;
+      uint64_t* bar = &sm.full[warp][slot];
+      if (lane == 0) mbar_arrive_expect_tx(bar, a.num_blocks > 0 ? 2u * kSegBytes : 0u);
+      if (a.num_blocks > 0)  // (an empty pool has no block 0 to stand in)
+        bulk_g2s(my_stg + slot * (2 * kSegBytes) + lane * kSegBytes,
+                 pool_h + static_cast<int64_t>(ok ? p : 0) * pstride, kSegBytes, bar);
+    }
+    return __ballot_sync(0xffffffffu, ok && lane < 2) & 3u;
+  };
 
   // ---- 0. set-up: barriers and tensor memory; first loads; query digits ----
   int32_t bfirst[kNV];  // loaders: block ids of chunks 0 .. 2
   int32_t bq[6];        // loaders: block ids of chunks c+3 .. c+8 at the start of iteration c
+  uint32_t okq[kNV] = {0u, 0u, 0u};  // loaders: segment flags of chunks c .. c+2
+  // the chunk holding the block that the fused append writes is copied only
+  // after the set-up barrier (-1: none)
+  int c_defer = -1;
+  if (a.k_new != nullptr && L > 0) {
+    const int bn = (L - 1) / kBlockSize;
+    if (bn >= blk0 && bn < blk1) c_defer = (bn - blk0) / kChunkBlocks;
+  }
   if (is_loader) {
 #pragma unroll
-    for (int i = 0; i < kNV; ++i) bfirst[i] = bid_of(i);
+    for (int i = 0; i < kNV; ++i) bfirst[i] = blk0 + kChunkBlocks * i + 2 * warp + (lane & 1) < blk1 ? braw[i] : -1;
 #pragma unroll
-    for (int i = 0; i < 6; ++i) bq[i] = bid_of(kNV + i);
+    for (int i = 0; i < 6; ++i)
+      bq[i] = blk0 + kChunkBlocks * (kNV + i) + 2 * warp + (lane & 1) < blk1 ? braw[kNV + i] : -1;
+    // my staging ring's barriers, then the first three chunks' copies go out
+    // while the query is rotated
+    if (lane == 0) {
+#pragma unroll
+      for (int i = 0; i < kNV; ++i) mbar_init(&sm.full[warp][i], 1);
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < kNV; ++i)
+      if (i < nchunks && i != c_defer) okq[i] = issue(i, bfirst[i], i);
+#pragma unroll
+    for (int i = 0; i < 3; ++i) prefetch_seg(bq[i]);
   } else if (is_soft) {
     const int sw = warp - kLoadWarps;
     const int stok = tid - 32 * kLoadWarps;
@@ -501,7 +547,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
   // ---- 1. the paged scan ------------------------------------------------------
   if (is_loader) {
     const uint32_t my_lanes = tbase + (static_cast<uint32_t>(warp * 32) << 16);
-    const uint32_t my_stg = smem_u32(sm.stg[warp][0]);
     // my value rows: row lane/2 of segment s, dims 64 (lane%2) + [0, 64)
     const uint32_t my_vt = smem_u32(sm.vt[0]) + ((32 * warp + (lane >> 1)) >> 3) * 1024 + (lane & 1) * 512 +
                            (lane >> 1 & 7) * 16;  // segment 1: + 2048
@@ -510,29 +555,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
     const float mscale = mkind == 0 ? c1 : (mkind == 2 ? kFix : 1.0f);
     const float mnone = mkind == 2 ? -1.0f : 0.0f;  // the factor of an absent token
     const uint32_t my_meta = smem_u32(&sm.meta[0][mkind][32 * warp + 16 * mseg + mrow0]);
-    // lanes 0 and 1: bulk copy of segment lane & 1 of chunk c (block p) into
-    // staging slot `slot`; every lane gets the pair of segment flags
-    // (bit s: segment s is inside the split and the pool)
-    auto issue = [&](int c, int32_t p, int slot) -> uint32_t {
-      const int blk = blk0 + kChunkBlocks * c + 2 * warp + (lane & 1);
-      const bool live = blk < blk1;
-      const bool ok = live && p >= 0 && p < a.num_blocks;
-      if (lane < 2) {
-        bad_blk |= live && !ok;
-        uint64_t* bar = &sm.full[warp][slot];
-        if (lane == 0) mbar_arrive_expect_tx(bar, a.num_blocks > 0 ? 2u * kSegBytes : 0u);
-        if (a.num_blocks > 0)  // (an empty pool has no block 0 to stand in)
-          bulk_g2s(my_stg + slot * (2 * kSegBytes) + lane * kSegBytes,
-                   pool_h + static_cast<int64_t>(ok ? p : 0) * pstride, kSegBytes, bar);
-      }
-      return __ballot_sync(0xffffffffu, ok && lane < 2) & 3u;
-    };
-    uint32_t okq[kNV] = {0u, 0u, 0u};  // segment flags of chunks c .. c+2
 #pragma unroll
-    for (int i = 0; i < kNV; ++i)
-      if (i < nchunks) okq[i] = issue(i, bfirst[i], i);
-#pragma unroll
-    for (int i = 0; i < 3; ++i) prefetch_seg(bq[i]);
+    for (int i = 0; i < kNV; ++i)  // the deferred chunk, if it is one of the first three
+      if (i == c_defer) okq[i] = issue(i, bfirst[i], i);
     Ring3 r{0, 0u};  // chunk c: staging slot, key-code, value and factor buffers r.i
 #pragma unroll 1
     for (int c = 0; c < nchunks; ++c) {
@@ -841,53 +866,52 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
     if (!sm.is_last) return;
     __threadfence();
 
-    // the last CTA of (b, h) merges the splits: thread t owns four output
-    // dims of one head and reads that slice and (m, l) of every split in
-    // batches of eight, all loads of a batch in flight at once, merging
-    // online (max, rescale, weighted sum)
+    // the last CTA of (b, h) merges the splits: warp g takes head g, lane l
+    // dims 4l .. 4l+3 of every split and, in lane s, (m, l) of split s; all
+    // loads of a batch of 16 splits are in flight at once, the weights go
+    // round by shuffles, and batches merge online (max, rescale, sum)
     const int ns = a.nsplit;
     const float* base = a.partials + (static_cast<int64_t>(b) * a.num_q_heads + h * G) * ns * kPartialFloats;
-    for (int t = tid; t < G * (kHeadDim / 4); t += kThreads) {
-      const int g = t / (kHeadDim / 4), q4 = t % (kHeadDim / 4);
+    for (int g = warp; g < G; g += kThreads / 32) {
       const float* hb = base + static_cast<int64_t>(g) * ns * kPartialFloats;
       float M = -CUDART_INF_F, lsum = 0.0f;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int s0 = 0; s0 < ns; s0 += 8) {
-        float2 ml[8];
-        float4 v[8];
+      for (int s0 = 0; s0 < ns; s0 += 16) {
+        float4 v[16];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float* rec = hb + static_cast<int64_t>(min(s0 + u, ns - 1)) * kPartialFloats;
-          ml[u] = __ldcg(reinterpret_cast<const float2*>(rec + kHeadDim));
-          v[u] = __ldcg(reinterpret_cast<const float4*>(rec) + q4);
-          if (s0 + u >= ns) ml[u].y = 0.0f;  // (a repeated record, not counted)
-        }
-        float Mb = M;
+        for (int u = 0; u < 16; ++u)
+          v[u] = s0 + u < ns ? __ldcg(reinterpret_cast<const float4*>(hb + static_cast<int64_t>(s0 + u) * kPartialFloats) + lane)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float2 ml = lane < 16 && s0 + lane < ns
+                              ? __ldcg(reinterpret_cast<const float2*>(hb + static_cast<int64_t>(s0 + lane) * kPartialFloats + kHeadDim))
+                              : make_float2(0.f, 0.f);
+        const bool has = ml.y > 0.0f;  // (an empty split has l = 0)
+        float Mb = has ? ml.x : -CUDART_INF_F;
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-          if (ml[u].y > 0.0f) Mb = fmaxf(Mb, ml[u].x);
+        for (int o = 16; o; o >>= 1) Mb = fmaxf(Mb, __shfl_xor_sync(0xffffffffu, Mb, o));
+        Mb = fmaxf(Mb, M);
         const float f = M == -CUDART_INF_F ? 0.0f : ex2(M - Mb);
+        const float w = has ? ex2(ml.x - Mb) : 0.0f;  // weight of split s0 + lane
+        float lw = w * ml.y;
+#pragma unroll
+        for (int o = 16; o; o >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
+        lsum = fmaf(lsum, f, lw);
         acc.x *= f;
         acc.y *= f;
         acc.z *= f;
         acc.w *= f;
-        lsum *= f;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float w = ml[u].y > 0.0f ? ex2(ml[u].x - Mb) : 0.0f;
-          lsum = fmaf(w, ml[u].y, lsum);
-          acc.x = fmaf(w, v[u].x, acc.x);
-          acc.y = fmaf(w, v[u].y, acc.y);
-          acc.z = fmaf(w, v[u].z, acc.z);
-          acc.w = fmaf(w, v[u].w, acc.w);
+        for (int u = 0; u < 16; ++u) {
+          const float wu = __shfl_sync(0xffffffffu, w, u);
+          acc.x = fmaf(wu, v[u].x, acc.x);
+          acc.y = fmaf(wu, v[u].y, acc.y);
+          acc.z = fmaf(wu, v[u].z, acc.z);
+          acc.w = fmaf(wu, v[u].w, acc.w);
         }
         M = Mb;
       }
       const float inv = lsum > 0.0f ? 1.0f / lsum : 0.0f;
-      sm.obuf[g][4 * q4] = acc.x * inv;
-      sm.obuf[g][4 * q4 + 1] = acc.y * inv;
-      sm.obuf[g][4 * q4 + 2] = acc.z * inv;
-      sm.obuf[g][4 * q4 + 3] = acc.w * inv;
+      reinterpret_cast<float4*>(sm.obuf[g])[lane] = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
     }
     if (tid == 0) a.tickets[b * a.num_kv_heads + h] = 0;  // ready for the next call
   }

@@ -216,13 +216,25 @@ def test_decode_dtypes(kvq, cuda, q_dtype, out_dtype, rel):
     _check_decode(wl, g, pool, q, q_dtype, got, rel=rel)
 
 
-def test_append_decode_matches_append_then_decode(kvq, cuda):
+# The fused step's appended block lies in the first chunk of a split ("short",
+# many splits) or, with one split per sequence ("one_split": 80 x 8 kv heads
+# are more CTAs than the SMs hold, so the plan does not split), in chunks
+# 0 .. 5 of it: the first three chunks are copied before the append is
+# written, except the one holding the new block.
+_APPEND_LENS = {
+    "short": (4, 16, 2, [70, 1, 33, 0]),
+    "one_split": (80, 16, 8, [0, 1, 700, 384, 385, 513] + [(97 * i * i + 31 * i) % 701 for i in range(74)]),
+}
+
+
+@pytest.mark.parametrize("case", sorted(_APPEND_LENS))
+def test_append_decode_matches_append_then_decode(kvq, cuda, case):
     """The fused one-step call writes the same pool bytes as the write path
     followed by the read path, gives the same outputs, and both agree with
     the oracle (codes: near-tie rules; outputs: 2e-3 on the same codes)."""
     torch = _torch()
-    wl = synth.Workload("ad", 4, 16, 2, 128, [70, 1, 33, 0], 16, synth.BF16, 3, 10.0, 30.0, seed=25,
-                        extra_blocks=2)
+    batch, hq, hkv, lens = _APPEND_LENS[case]
+    wl = synth.Workload("ad", batch, hq, hkv, 128, lens, 16, synth.BF16, 3, 10.0, 30.0, seed=25, extra_blocks=2)
     T = wl.total_tokens
     k = wl.kv_rows(synth.TID_K, 0, T)
     v = wl.kv_rows(synth.TID_V, 0, T)
@@ -267,7 +279,9 @@ def test_append_decode_matches_append_then_decode(kvq, cuda):
     helpers.check_pool_tokens(rep, p2, wl.num_blocks, wl.hkv, k, v, wl.dtype, slots, last)
     assert rep.ok(), rep
     _check_decode(wl, g, p2, q, wl.dtype, out2.cpu().numpy().astype(np.float64))
-    assert not out2[3].any()
+    for b in range(wl.batch):
+        if wl.seq_lens[b] == 0:  # an empty sequence appends nothing and reads nothing
+            assert not out2[b].any()
 
 
 def test_decode_workspace_is_reusable(kvq, cuda):
