@@ -856,15 +856,21 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
     }
   }
   if (a.nsplit > 1) {
-    __threadfence();
+    // ticket: one acquire-release add by thread 0 between two CTA barriers
+    // publishes every thread's record stores (they happen before the add)
+    // and, in the last CTA, makes every split's record visible to every
+    // thread's loads below
     __syncthreads();
     if (tid == 0) {
-      const int t = atomicAdd(&a.tickets[b * a.num_kv_heads + h], 1);
+      int t;
+      asm volatile("atom.add.acq_rel.gpu.global.s32 %0, [%1], 1;"
+                   : "=r"(t)
+                   : "l"(a.tickets + b * a.num_kv_heads + h)
+                   : "memory");
       sm.is_last = (t == a.nsplit - 1);
     }
     __syncthreads();
     if (!sm.is_last) return;
-    __threadfence();
 
     // the last CTA of (b, h) merges the splits: warp g takes head g, lane l
     // dims 4l .. 4l+3 of every split and, in lane s, (m, l) of split s; all
