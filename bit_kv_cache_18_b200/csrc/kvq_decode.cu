@@ -368,6 +368,27 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
   }
   pdl_wait();
 
+  // The softmax warps' loads that need no sequence length go out first:
+  // warp sw's query heads sw and sw + 4 and, for warps 4 and 5 of a fused
+  // step, their lanes' 8 bytes of the new token's K or V row.
+  float x[2][4];
+  uint2 new_raw = make_uint2(0u, 0u);
+  if (is_soft) {
+    const int sw = warp - kLoadWarps;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int g = sw + 4 * i;
+      if (g < G) {
+        const int64_t q0 = (static_cast<int64_t>(b) * a.num_q_heads + h * G + g) * kHeadDim;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) x[i][k] = load_as_f32(a.q, a.q_dtype, q0 + lane + 32 * k);
+      }
+    }
+    if (a.k_new != nullptr && sw < 2)
+      new_raw = *reinterpret_cast<const uint2*>((sw ? a.v_new : a.k_new) + static_cast<int64_t>(b) * a.new_stride_bytes +
+                                                static_cast<int64_t>(h) * (kHeadDim * 2) + 8 * lane);
+  }
+
   // ---- the split: blocks [blk0, blk1) of sequence b, in chunks of 8 -------
   // Loader warp w owns blocks 2w and 2w+1 of every chunk (tokens 32w ..
   // 32w + 31 = TMEM lanes of its quarter); its lanes read the block ids of
@@ -471,30 +492,24 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
         const int32_t p = bt_row[blk_new];
         if (p >= 0 && p < a.num_blocks) {
           uint8_t* seg = const_cast<uint8_t*>(pool_h) + static_cast<int64_t>(p) * pstride;
-          const uint8_t* src = (sw ? a.v_new : a.k_new) + static_cast<int64_t>(b) * a.new_stride_bytes +
-                               static_cast<int64_t>(h) * (kHeadDim * 2);
           if (a.new_bf16)
-            quantize_vector_warp<true>(src, seg, (L - 1) % kBlockSize, sw == 1, lane);
+            quantize_vector_warp_raw<true>(new_raw, seg, (L - 1) % kBlockSize, sw == 1, lane);
           else
-            quantize_vector_warp<false>(src, seg, (L - 1) % kBlockSize, sw == 1, lane);
+            quantize_vector_warp_raw<false>(new_raw, seg, (L - 1) % kBlockSize, sw == 1, lane);
           asm volatile("fence.proxy.async.global;" ::: "memory");
         } else if (lane == 0) {
           record_status(a.status, KVQ_ERR_OUT_OF_RANGE);
         }
       }
     }
-    // rotate the G query heads (warp sw: heads sw, sw + 4), then write their
-    // digits with one c1 for all heads
+    // rotate the G query heads, then write their digits with one c1 for all
+    // heads
     reinterpret_cast<uint4*>(sm.qb)[stok] = make_uint4(0, 0, 0, 0);
     reinterpret_cast<uint4*>(sm.qb)[stok + 128] = make_uint4(0, 0, 0, 0);
-    float x[2][4];
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       const int g = sw + 4 * i;
       if (g < G) {
-        const int64_t q0 = (static_cast<int64_t>(b) * a.num_q_heads + h * G + g) * kHeadDim;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) x[i][k] = load_as_f32(a.q, a.q_dtype, q0 + lane + 32 * k);
         fwht_warp(x[i], lane, a.scale_log2);
         float s4 = (x[i][0] + x[i][1]) + (x[i][2] + x[i][3]);
         float mx = fmaxf(fmaxf(fabsf(x[i][0]), fabsf(x[i][1])), fmaxf(fabsf(x[i][2]), fabsf(x[i][3])));

@@ -73,12 +73,11 @@ __device__ __forceinline__ void store_from_f32(void* p, int dtype, int64_t i, fl
 // the packed row: two bytes of 4-bit key codes or one byte of 2-bit codes.
 // Method: "KVarN vs TurboQuant" (dothoosh.com), pipeline list: Hadamard
 // rotation, variance normalisation, asymmetric round-to-nearest.
+// quantize_vector_warp_raw takes the lane's 8 source bytes already loaded.
 template <bool kBF16>
-__device__ __forceinline__ void quantize_vector_warp(const uint8_t* src, uint8_t* seg, int row_in_block, bool is_v,
-                                                     int lane) {
+__device__ __forceinline__ void quantize_vector_warp_raw(uint2 raw, uint8_t* seg, int row_in_block, bool is_v,
+                                                         int lane) {
   constexpr float kMagicRne = 12582912.0f;  // 1.5 * 2^23: low mantissa bits hold rne of the addend
-  // elements 4 lane .. 4 lane + 3 (8 bytes)
-  const uint2 raw = *reinterpret_cast<const uint2*>(src + 8 * lane);
   float y[4];
   if (kBF16) {
     y[0] = bf16lo_to_f32(raw.x);
@@ -157,6 +156,13 @@ __device__ __forceinline__ void quantize_vector_warp(const uint8_t* src, uint8_t
       reinterpret_cast<__half*>(seg + kOffZK)[row_in_block] = Zh;
     }
   }
+}
+
+// elements 4 lane .. 4 lane + 3 (8 bytes) of the vector at src
+template <bool kBF16>
+__device__ __forceinline__ void quantize_vector_warp(const uint8_t* src, uint8_t* seg, int row_in_block, bool is_v,
+                                                     int lane) {
+  quantize_vector_warp_raw<kBF16>(*reinterpret_cast<const uint2*>(src + 8 * lane), seg, row_in_block, is_v, lane);
 }
 
 // ---- programmatic dependent launch ------------------------------------------

@@ -183,7 +183,9 @@ int kvq_decode_attention_ex(const kvq_cache_desc* desc, const void* q, kvq_dtype
  * sequence b with L = seq_lens[b] > 0, the new token's K and V rows (k_new,
  * v_new: device, row b at element b*token_stride, [num_kv_heads, 128] of
  * in_dtype F16 or BF16, 16-byte aligned, token_stride a multiple of 8 and
- * >= num_kv_heads*128) are quantized into position L-1, i.e. slot
+ * >= num_kv_heads*128; the rows of all batch sequences must be readable,
+ * an empty sequence's row is read and ignored) are quantized into position
+ * L-1, i.e. slot
  * block_table[b][(L-1)/16]*16 + (L-1)%16 -- the bytes kvq_quantize_append
  * writes for that slot -- and then the decode attention of
  * kvq_decode_attention runs over positions 0 .. L-1, the new token included.
