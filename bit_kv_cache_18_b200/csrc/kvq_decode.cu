@@ -260,6 +260,8 @@ __device__ __forceinline__ void tmem_ld8(uint32_t addr, uint32_t (&r)[8]) {
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// The 128-byte line holding p into L2.
+__device__ __forceinline__ void prefetch_line_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
 __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
@@ -466,6 +468,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
 #pragma unroll
     for (int i = 0; i < 6; ++i)
       bq[i] = blk0 + kChunkBlocks * (kNV + i) + 2 * warp + (lane & 1) < blk1 ? braw[kNV + i] : -1;
+    // the split's block-table slice into L2: the ids of later chunks are
+    // read six chunks ahead of use, and a miss would stall the ring
+    for (int ln = tid; ln * 128 < (blk1 - blk0) * 4; ln += 32 * kLoadWarps)
+      prefetch_line_l2(reinterpret_cast<const char*>(bt_row + blk0) + ln * 128);
     // my staging ring's barriers, then the first three chunks' copies go out
     // while the query is rotated
     if (lane == 0) {
