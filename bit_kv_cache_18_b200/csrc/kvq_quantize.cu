@@ -1,31 +1,31 @@
 // kvq_quantize.cu -- cache write path: rotate, normalise, quantise, pack.
 //
-// One thread owns one 128-element K or V head vector end to end, so the
-// Walsh-Hadamard transform, the mean/variance/min/max reductions and the
-// packing all stay in that thread's registers and need no shuffles.  The
-// butterflies use Blackwell's packed f32x2 add/sub: the thread keeps the
-// vector as 64 pairs (x[k], x[k+64]); the stride-64 stage is done first as
-// scalars and the six remaining stages run on whole pairs.
+// Bulk appends (prefill): the rotation of a tile of 128 head vectors is one
+// matrix product on the fifth-generation tensor cores, Y = X H with H the
+// 128 x 128 Sylvester Hadamard matrix (entries +-1, exact in bf16 and fp16,
+// accumulated in fp32).  Rows reach shared memory through 16-byte cp.async
+// copies laid out as the no-swizzle K-major operand (eight lanes write 128
+// contiguous bytes; each source row is read 64 bytes at a time), one thread
+// issues the 8-step tcgen05.mma chain into 128 fp32 tensor-memory columns,
+// and thread t then owns vector t (tensor-memory lane t): moments, range and
+// (S, Z) from one pass over its columns, the codes from a second, packed
+// with fp32x2 arithmetic and written as 16-byte stores into the paged
+// segment plus two fp16 stores.  Two operand buffers per CTA let the copies
+// of the next tiles run under the current tile's arithmetic.
 //
-// Rows reach shared memory through 16-byte cp.async copies that are coalesced
-// across the warp (two 256-byte rows per instruction) into a 272-byte pitch,
-// which makes the per-thread row reads bank-conflict free; each warp double
-// buffers its 32-row tiles.  Codes leave as 16-byte stores into the paged
-// segment (64 B of K codes or 32 B of V codes per row) plus two fp16 stores.
+// Small appends (decode steps): one warp per vector (quantize_vector_warp in
+// kvq_internal.cuh), butterflies in registers and shuffles.
 //
 // Method ("Трюк Huawei с KV-кэшем", section "Заявка, которая ломает
 // привычный компромисс"; "KVarN vs TurboQuant", pipeline list): Hadamard
 // rotation, variance normalisation, asymmetric round-to-nearest; the exact
 // definition and pool layout are stated in include/kvq.h.
+#include <math_constants.h>
+
 #include "kvq_internal.cuh"
 
 namespace kvq {
 namespace {
-
-constexpr int kWarps = 4;
-constexpr int kRows = 32;                  // vectors per warp tile, one per lane
-constexpr int kPitch = kHeadDim * 2 + 16;  // 272-byte smem pitch of a 256-byte row
-constexpr int kTileBytes = kRows * kPitch;
 
 typedef unsigned long long u64;
 
@@ -43,11 +43,6 @@ __device__ __forceinline__ void upk_u(u64 v, uint32_t& a, uint32_t& b) {
 __device__ __forceinline__ u64 add2(u64 a, u64 b) {
   u64 d;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ u64 sub2(u64 a, u64 b) {
-  u64 d;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
 __device__ __forceinline__ u64 fma2(u64 a, u64 b, u64 c) {
@@ -84,17 +79,167 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N));
 }
 
-// Stage the 32 rows of tile `tile` (vectors tile*32 .. tile*32+31 of one of
-// the two tensors) into smem.  Row r of the tile is vector n = tile*32 + r,
-// i.e. token n / Hkv, head n % Hkv.  Lane l copies chunk (16 B) l of rows
-// 2j and 2j+1 in iteration j; the row addresses are computed once per lane
-// (its own vector) and handed around with shuffles.
-__device__ __forceinline__ void stage_tile(uint32_t sbuf, const uint8_t* src, int64_t n_vec,
-                                           int hkv, int64_t stride_bytes, int64_t tile, int lane) {
-  const int64_t n = tile * kRows + lane;
-  const bool mine_valid = n < n_vec;
-  const int64_t tok = mine_valid ? n / hkv : 0;
-  const int hh = mine_valid ? static_cast<int>(n - tok * hkv) : 0;
+// ---- tensor-core pieces -------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+      : "=r"(done)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Wait for a barrier phase, at most about a second (false: it never came).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t it = 1; it < (1u << 26); ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0 && global_ns() - t0 > 1000000000ull) return false;
+  }
+  return false;
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void async_proxy_fence() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+// sm_100 shared-memory matrix descriptor: start address, leading (K) and
+// stride (M/N) byte offsets in 16-byte units, version 1, no swizzle.
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+// The 128 fp32 columns at addr of this thread's tensor-memory lane, one
+// load and one wait.
+__device__ __forceinline__ void tmem_ld128(uint32_t addr, float (&v)[128]) {
+  uint32_t r[128];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x128.b32 {"
+      "%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+      "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,"
+      "%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,"
+      "%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95,"
+      "%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,"
+      "%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127"
+      "}, [%128];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+        "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+        "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63]),
+        "=r"(r[64]), "=r"(r[65]), "=r"(r[66]), "=r"(r[67]), "=r"(r[68]), "=r"(r[69]), "=r"(r[70]), "=r"(r[71]),
+        "=r"(r[72]), "=r"(r[73]), "=r"(r[74]), "=r"(r[75]), "=r"(r[76]), "=r"(r[77]), "=r"(r[78]), "=r"(r[79]),
+        "=r"(r[80]), "=r"(r[81]), "=r"(r[82]), "=r"(r[83]), "=r"(r[84]), "=r"(r[85]), "=r"(r[86]), "=r"(r[87]),
+        "=r"(r[88]), "=r"(r[89]), "=r"(r[90]), "=r"(r[91]), "=r"(r[92]), "=r"(r[93]), "=r"(r[94]), "=r"(r[95]),
+        "=r"(r[96]), "=r"(r[97]), "=r"(r[98]), "=r"(r[99]), "=r"(r[100]), "=r"(r[101]), "=r"(r[102]), "=r"(r[103]),
+        "=r"(r[104]), "=r"(r[105]), "=r"(r[106]), "=r"(r[107]), "=r"(r[108]), "=r"(r[109]), "=r"(r[110]), "=r"(r[111]),
+        "=r"(r[112]), "=r"(r[113]), "=r"(r[114]), "=r"(r[115]), "=r"(r[116]), "=r"(r[117]), "=r"(r[118]), "=r"(r[119]),
+        "=r"(r[120]), "=r"(r[121]), "=r"(r[122]), "=r"(r[123]), "=r"(r[124]), "=r"(r[125]), "=r"(r[126]), "=r"(r[127])
+      : "r"(addr)
+      : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 128; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// ---- bulk path ------------------------------------------------------------------
+// A CTA of 128 threads walks tiles of 128 head vectors (one tensor, K or V);
+// thread t owns vector t of a tile and tensor-memory lane t.  Warp w stages
+// its 32 rows (vectors 32w .. 32w+31 of the tile) itself, two tiles ahead,
+// with coalesced 16-byte cp.async copies into a 272-byte-pitch ring; each
+// lane reads its row back (conflict free) and stores its 64 pairs of 16-bit
+// elements, unconverted, into its tensor-memory lane: the A operand.  The
+// rotation y = x H (H the 128 x 128 Sylvester Hadamard matrix,
+// unnormalised, exact in 16-bit floats) is then one tcgen05.mma chain
+// (M = 128 vectors, N = 128, K = 128 in 8 steps of 16; B = H in shared
+// memory) into 128 fp32 columns, which every thread reads back in one load
+// for the moments, range and codes of its vector.
+constexpr int kTileVecs = 128;
+constexpr int kBulkThreads = 128;
+constexpr int kWarpRows = 32;                     // rows a warp stages per tile
+constexpr int kPitch = kHeadDim * 2 + 16;         // 272-byte pitch of a 256-byte row
+constexpr int kStageBytes = kWarpRows * kPitch;   // 8.5 KB
+constexpr uint32_t kBulkTmemCols = 256;
+constexpr uint32_t kColD = 0;    // y: 128 fp32 columns
+constexpr uint32_t kColA = 128;  // x: 64 columns of 16-bit pairs
+
+// B = H in the no-swizzle K-major layout of 8-row x 16-byte core matrices:
+// element (n, k) at (k/8)*2048 + n*16 + (k%8)*2 (leading, i.e. K, offset
+// 2048; stride offset 128).
+struct __align__(1024) BulkSmem {
+  uint8_t hm[kHeadDim * kHeadDim * 2];   // 32 KB
+  uint8_t stg[4][2][kStageBytes];        // warp w: its rows of tiles i (slot i % 2) and i+1
+  uint64_t mma_done;                     // the MMA chain of the tile is complete
+  uint32_t tmem_base;
+};
+constexpr int kBulkSmemBytes = static_cast<int>(sizeof(BulkSmem));
+static_assert(kBulkSmemBytes <= 113 * 1024, "two CTAs per SM");
+
+// Instruction descriptor, kind::f16: D f32, A and B f16 or bf16, A in
+// tensor memory, B K-major, N = 128, M = 128.
+template <bool kBF16>
+__host__ __device__ constexpr uint32_t idesc_h() {
+  return (1u << 4) | ((kBF16 ? 1u : 0u) << 7) | ((kBF16 ? 1u : 0u) << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+}
+__device__ __forceinline__ void mma_f16_ta(uint32_t d, uint32_t a, uint64_t bdesc, uint32_t idesc, bool acc) {
+  asm volatile(
+      "{ .reg .pred p; setp.ne.b32 p, %3, 0;\n"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %4, p; }" ::"r"(d),
+      "r"(a), "l"(bdesc), "r"(static_cast<uint32_t>(acc)), "r"(idesc)
+      : "memory");
+}
+// 64 consecutive columns of this thread's lane from 64 registers.
+__device__ __forceinline__ void tmem_st64(uint32_t addr, const uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], {"
+      "%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,"
+      "%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,"
+      "%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64};" ::"r"(addr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+      "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+      "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]),
+      "r"(r[32]), "r"(r[33]), "r"(r[34]), "r"(r[35]), "r"(r[36]), "r"(r[37]), "r"(r[38]), "r"(r[39]),
+      "r"(r[40]), "r"(r[41]), "r"(r[42]), "r"(r[43]), "r"(r[44]), "r"(r[45]), "r"(r[46]), "r"(r[47]),
+      "r"(r[48]), "r"(r[49]), "r"(r[50]), "r"(r[51]), "r"(r[52]), "r"(r[53]), "r"(r[54]), "r"(r[55]),
+      "r"(r[56]), "r"(r[57]), "r"(r[58]), "r"(r[59]), "r"(r[60]), "r"(r[61]), "r"(r[62]), "r"(r[63])
+      : "memory");
+}
+
+// Token of vector n (n < n_vec): 32-bit division whenever the indices fit.
+__device__ __forceinline__ int64_t token_of(int64_t n, int64_t n_vec, int hkv) {
+  return n_vec <= 0xFFFFFFFFll ? static_cast<int64_t>(static_cast<uint32_t>(n) / static_cast<uint32_t>(hkv))
+                               : n / hkv;
+}
+
+// Stage rows row0 .. row0+31 (vector n = token n / Hkv, head n % Hkv) into a
+// warp's slot: in copy j lane l moves 16-byte chunk l % 16 of row 2j + l/16
+// (two whole rows per instruction); the row addresses are computed once per
+// lane (its own row) and handed round by shuffles.  Rows past the tensor are
+// zero filled.
+__device__ __forceinline__ void stage_rows(uint32_t dst, const uint8_t* src, int64_t n_vec, int hkv,
+                                           int64_t stride_bytes, int64_t row0, int lane) {
+  const int64_t n = row0 + lane;
+  const bool mine = n < n_vec;
+  const int64_t tok = mine ? token_of(n, n_vec, hkv) : 0;
+  const int hh = mine ? static_cast<int>(n - tok * hkv) : 0;
   const uint8_t* my_row = src + tok * stride_bytes + static_cast<int64_t>(hh) * (kHeadDim * 2);
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
@@ -102,55 +247,8 @@ __device__ __forceinline__ void stage_tile(uint32_t sbuf, const uint8_t* src, in
     const int col = lane & 15;
     const uint8_t* row_ptr = reinterpret_cast<const uint8_t*>(
         __shfl_sync(0xffffffffu, static_cast<unsigned long long>(reinterpret_cast<uintptr_t>(my_row)), row));
-    const bool valid = tile * kRows + row < n_vec;
-    cp_async16(sbuf + row * kPitch + col * 16, valid ? row_ptr + col * 16 : src, valid);
-  }
-}
-
-// 128 elements of the thread's row in smem -> pairs P[k] = (x[k], x[k+64])
-// after the stride-64 butterfly (x[k] + x[k+64], x[k] - x[k+64]).
-template <bool kBF16>
-__device__ __forceinline__ void load_row(const uint8_t* row, u64 (&P)[64]) {
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const uint4 lo = *reinterpret_cast<const uint4*>(row + j * 16);       // x[8j .. 8j+7]
-    const uint4 hi = *reinterpret_cast<const uint4*>(row + j * 16 + 128);  // x[64+8j ..]
-    const uint32_t wl[4] = {lo.x, lo.y, lo.z, lo.w};
-    const uint32_t wh[4] = {hi.x, hi.y, hi.z, hi.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      float a0, a1, b0, b1;
-      if (kBF16) {
-        a0 = bf16lo_to_f32(wl[e]);
-        a1 = bf16hi_to_f32(wl[e]);
-        b0 = bf16lo_to_f32(wh[e]);
-        b1 = bf16hi_to_f32(wh[e]);
-      } else {
-        const float2 fa = __half22float2(*reinterpret_cast<const __half2*>(&wl[e]));
-        const float2 fb = __half22float2(*reinterpret_cast<const __half2*>(&wh[e]));
-        a0 = fa.x;
-        a1 = fa.y;
-        b0 = fb.x;
-        b1 = fb.y;
-      }
-      P[8 * j + 2 * e] = pk(a0 + b0, a0 - b0);
-      P[8 * j + 2 * e + 1] = pk(a1 + b1, a1 - b1);
-    }
-  }
-}
-
-// The remaining six butterfly stages (strides 1..32) on whole pairs.
-__device__ __forceinline__ void fwht_pairs(u64 (&P)[64]) {
-#pragma unroll
-  for (int s = 1; s < 64; s <<= 1) {
-#pragma unroll
-    for (int k = 0; k < 64; ++k) {
-      if ((k & s) == 0) {
-        const u64 a = P[k], b = P[k + s];
-        P[k] = add2(a, b);
-        P[k + s] = sub2(a, b);
-      }
-    }
+    const bool valid = row0 + row < n_vec;
+    cp_async16(dst + row * kPitch + col * 16, valid ? row_ptr + col * 16 : src, valid);
   }
 }
 
@@ -158,64 +256,85 @@ __device__ __forceinline__ void fwht_pairs(u64 (&P)[64]) {
 // t = q + 1.5*2^23 has ulp 1, so its low bits hold rne(q) (ties to even).
 constexpr float kMagic = 12582912.0f;
 
+// Codes rne(y a + b) (clamped to [0, L] if kClamp) of the 128 elements of
+// y, packed: 8 four-bit codes or 16 two-bit codes per word, element 0 in
+// the low bits.
+template <int kBits, bool kClamp>
+__device__ __forceinline__ void codes_to_words(const float (&y)[kHeadDim], u64 a2, u64 b2,
+                                               uint32_t (&words)[kHeadDim * kBits / 32]) {
+  constexpr float kLevels = static_cast<float>((1 << kBits) - 1);
+  const u64 m2 = pk(kMagic, kMagic);
+#pragma unroll
+  for (int c0 = 0; c0 < kHeadDim; c0 += 32) {
+    uint32_t c[32];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      u64 t = fma2(pk(y[c0 + 2 * j], y[c0 + 2 * j + 1]), a2, b2);
+      if (kClamp) {
+        float ta, tb;
+        upk(t, ta, tb);
+        t = pk(fminf(fmaxf(ta, 0.0f), kLevels), fminf(fmaxf(tb, 0.0f), kLevels));
+      }
+      upk_u(add2(t, m2), c[2 * j], c[2 * j + 1]);
+    }
+    if (kBits == 4) {
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {  // word c0/8 + m = elements c0 + 8m .. +7
+        const uint32_t* e = c + 8 * m;
+        const uint32_t b0 = e[0] + 16u * e[1], b1 = e[2] + 16u * e[3];
+        const uint32_t bb2 = e[4] + 16u * e[5], b3 = e[6] + 16u * e[7];
+        words[c0 / 8 + m] = prmt(prmt(b0, b1, 0x0040u), prmt(bb2, b3, 0x0040u), 0x5410u);
+      }
+    } else {
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {  // word c0/16 + m = elements c0 + 16m .. +15
+        const uint32_t* e = c + 16 * m;
+        uint32_t by[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) by[q] = e[4 * q] + 4u * e[4 * q + 1] + 16u * e[4 * q + 2] + 64u * e[4 * q + 3];
+        words[c0 / 16 + m] = prmt(prmt(by[0], by[1], 0x0040u), prmt(by[2], by[3], 0x0040u), 0x5410u);
+      }
+    }
+  }
+}
+
+// Moments, range, (S, Z) and codes of the vector whose y = x H sits in 128
+// fp32 columns of tensor memory at taddr (read once, into registers); the
+// packed row, S and Z go to row `row_in_block` of the segment (seg ==
+// nullptr: not stored).  Every thread of the warp runs it: the
+// tensor-memory load is warp-collective.
 template <int kBits>
-__device__ __forceinline__ void quantize_store(u64 (&P)[64], uint8_t* seg, int row_in_block) {
+__device__ __forceinline__ void quantize_lane(uint32_t taddr, float x0, uint8_t* seg, int row_in_block) {
   constexpr float kLevels = static_cast<float>((1 << kBits) - 1);
   constexpr float kInvSqrtD = 0.088388347648318440550f;  // 1/sqrt(128)
-
-  // variance normalisation statistics of r = y / sqrt(128), computed on y
-  u64 s2 = 0ull, q2 = 0ull;
-  {
-    u64 acc_s[8], acc_q[8];
+  float y[kHeadDim];  // y = x H of my vector (r = y / sqrt(128))
+  tmem_ld128(taddr, y);
+  // moments and range; the mean of y is x0 (every column of H but the first
+  // sums to zero), the rest is summed here
+  u64 acc_q[4] = {0ull, 0ull, 0ull, 0ull};
+  float mn[4], mx[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      acc_s[i] = P[i];
-      acc_q[i] = fma2(P[i], P[i], 0ull);
-    }
-#pragma unroll
-    for (int k = 8; k < 64; ++k) {
-      acc_s[k & 7] = add2(acc_s[k & 7], P[k]);
-      acc_q[k & 7] = fma2(P[k], P[k], acc_q[k & 7]);
-    }
-#pragma unroll
-    for (int w = 4; w >= 1; w >>= 1)
-#pragma unroll
-      for (int i = 0; i < w; ++i) {
-        acc_s[i] = add2(acc_s[i], acc_s[i + w]);
-        acc_q[i] = add2(acc_q[i], acc_q[i + w]);
-      }
-    s2 = acc_s[0];
-    q2 = acc_q[0];
+  for (int i = 0; i < 4; ++i) {
+    mn[i] = CUDART_INF_F;
+    mx[i] = -CUDART_INF_F;
   }
-  float sa, sb, qa, qb;
-  upk(s2, sa, sb);
+#pragma unroll
+  for (int j = 0; j < kHeadDim / 2; ++j) {
+    const u64 p = pk(y[2 * j], y[2 * j + 1]);
+    acc_q[j & 3] = fma2(p, p, acc_q[j & 3]);
+    mn[j & 3] = min3(mn[j & 3], y[2 * j], y[2 * j + 1]);
+    mx[j & 3] = max3(mx[j & 3], y[2 * j], y[2 * j + 1]);
+  }
+  const u64 q2 = add2(add2(acc_q[0], acc_q[1]), add2(acc_q[2], acc_q[3]));
+  float qa, qb;
   upk(q2, qa, qb);
-  const float mean = (sa + sb) * (1.0f / kHeadDim);
+  const float ymin = fminf(fminf(mn[0], mn[1]), fminf(mn[2], mn[3]));
+  const float ymax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+  const float mean = x0;
   const float var = fmaxf((qa + qb) * (1.0f / kHeadDim) - mean * mean, 0.0f);
   float sigma = sqrtf(var);
   if (sigma == 0.0f) sigma = 1.0f;
-
-  // range of y (min/max of u = (y - mean)/sigma sit at the same elements)
-  float ymin, ymax;
-  {
-    float mn[8], mx[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      float a, b;
-      upk(P[i], a, b);
-      mn[i] = fminf(a, b);
-      mx[i] = fmaxf(a, b);
-    }
-#pragma unroll
-    for (int k = 8; k < 64; ++k) {
-      float a, b;
-      upk(P[k], a, b);
-      mn[k & 7] = min3(mn[k & 7], a, b);
-      mx[k & 7] = max3(mx[k & 7], a, b);
-    }
-    ymin = min3(min3(mn[0], mn[1], mn[2]), min3(mn[3], mn[4], mn[5]), fminf(mn[6], mn[7]));
-    ymax = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
-  }
+  // (min/max of u = (y - mean)/sigma sit at the same elements as those of y)
   const float lo = (ymin - mean) / sigma;
   const float hi = (ymax - mean) / sigma;
   const __half Sh = __float2half_rn(kInvSqrtD * (sigma * (hi - lo)) / kLevels);
@@ -223,65 +342,28 @@ __device__ __forceinline__ void quantize_store(u64 (&P)[64], uint8_t* seg, int r
   const float Sf = __half2float(Sh);
   const float Zf = __half2float(Zh);
 
-  // codes: q = (r - Z)/S = y * (c/S) - Z/S, rounded to nearest even, clamped
-  uint32_t words[16];
-  if (Sf == 0.0f) {
-#pragma unroll
-    for (int m = 0; m < 16; ++m) words[m] = 0u;
-  } else {
-    const float a = kInvSqrtD / Sf;
-    const float b = -Zf / Sf;
-    const u64 a2 = pk(a, a), b2 = pk(b, b), m2 = pk(kMagic, kMagic);
-    // q is monotone in y, so clamping is needed only if an extreme leaves range
-    const float cmin = fmaf(ymin, a, b) + kMagic;
-    const float cmax = fmaf(ymax, a, b) + kMagic;
-    const bool clamp = (cmin < kMagic) || (cmax > kMagic + kLevels);
-#pragma unroll
-    for (int k = 0; k < 64; ++k) {
-      u64 t = fma2(P[k], a2, b2);
-      if (clamp) {
-        float ta, tb;
-        upk(t, ta, tb);
-        t = pk(fminf(fmaxf(ta, 0.0f), kLevels), fminf(fmaxf(tb, 0.0f), kLevels));
-      }
-      P[k] = add2(t, m2);
-    }
-    // pack: element i < 64 is P[i].x, element i >= 64 is P[i-64].y
-    if (kBits == 4) {
-#pragma unroll
-      for (int m = 0; m < 16; ++m) {  // word m = elements 8m .. 8m+7
-        uint32_t c[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int i = 8 * m + e;
-          uint32_t lo_bits, hi_bits;
-          upk_u(P[i & 63], lo_bits, hi_bits);
-          c[e] = (i < 64) ? lo_bits : hi_bits;
-        }
-        const uint32_t b0 = c[0] + 16u * c[1], b1 = c[2] + 16u * c[3];
-        const uint32_t b2 = c[4] + 16u * c[5], b3 = c[6] + 16u * c[7];
-        words[m] = prmt(prmt(b0, b1, 0x0040u), prmt(b2, b3, 0x0040u), 0x5410u);
-      }
-    } else {
-#pragma unroll
-      for (int m = 0; m < 8; ++m) {  // word m = elements 16m .. 16m+15
-        uint32_t c[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int i = 16 * m + e;
-          uint32_t lo_bits, hi_bits;
-          upk_u(P[i & 63], lo_bits, hi_bits);
-          c[e] = (i < 64) ? lo_bits : hi_bits;
-        }
-        uint32_t by[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          by[q] = c[4 * q] + 4u * c[4 * q + 1] + 16u * c[4 * q + 2] + 64u * c[4 * q + 3];
-        words[m] = prmt(prmt(by[0], by[1], 0x0040u), prmt(by[2], by[3], 0x0040u), 0x5410u);
-      }
-    }
+  // codes: q = (r - Z)/S = y (c/S) - Z/S, rounded to nearest even, clamped
+  // (S == 0: a = b = 0 gives code 0 everywhere)
+  constexpr int kWords = kHeadDim * kBits / 32;  // 16 (K) or 8 (V)
+  uint32_t words[kWords];
+  {
+    const bool flat = Sf == 0.0f;
+    const float a = flat ? 0.0f : kInvSqrtD / Sf;
+    const float b = flat ? 0.0f : -Zf / Sf;
+    const u64 a2 = pk(a, a), b2 = pk(b, b);
+    // q is monotone in y, so clamping is needed only if the code of an
+    // extreme leaves [0, L]: rne(q) < 0 iff q < -1/2, rne(q) > L iff
+    // q >= L + 1/2 (the same fused multiply-add as below); clamping to the
+    // integers 0 and L commutes with the rounding
+    const bool clamp = (fmaf(ymin, a, b) < -0.5f) || (fmaf(ymax, a, b) >= kLevels + 0.5f);
+    // (two copies of the loop, so that the common unclamped one carries no
+    // clamping work)
+    if (clamp)
+      codes_to_words<kBits, true>(y, a2, b2, words);
+    else
+      codes_to_words<kBits, false>(y, a2, b2, words);
   }
-
+  if (seg == nullptr) return;
   if (kBits == 4) {
     uint4* dst = reinterpret_cast<uint4*>(seg + kOffK + row_in_block * kKRowBytes);
 #pragma unroll
@@ -300,71 +382,142 @@ __device__ __forceinline__ void quantize_store(u64 (&P)[64], uint8_t* seg, int r
 }
 
 template <bool kBF16>
-__global__ void __launch_bounds__(kWarps * 32)
+__global__ void __launch_bounds__(kBulkThreads, 2)
     quantize_kernel(uint8_t* __restrict__ pool, int32_t num_blocks, int32_t hkv,
                     const uint8_t* __restrict__ k, const uint8_t* __restrict__ v,
                     int32_t n_tokens, int64_t stride_bytes, const int32_t* __restrict__ slots, int* status) {
-  extern __shared__ __align__(16) uint8_t smem[];
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  BulkSmem& sm = *reinterpret_cast<BulkSmem*>(smem_raw);
   pdl_trigger();  // (the grid is persistent: every CTA is resident at once)
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+
+  // tensor memory, the barrier and H need no global memory: before the wait
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sm.tmem_base)),
+                 "n"(kBulkTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if (tid == 0) {
+    mbar_init(&sm.mma_done, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  {  // H row n = tid: entry (n, k) = (-1)^popcount(n & k), as 16-bit +-1
+    const uint32_t one = kBF16 ? 0x3F80u : 0x3C00u;
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int k0 = 8 * c + 2 * e;
+        const uint32_t h0 = one | ((__popc(tid & k0) & 1u) << 15);
+        const uint32_t h1 = one | ((__popc(tid & (k0 + 1)) & 1u) << 15);
+        w[e] = h0 | (h1 << 16);
+      }
+      *reinterpret_cast<uint4*>(sm.hm + c * 2048 + tid * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+  async_proxy_fence();  // (H is read by the tensor cores)
   pdl_wait();
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  const uint32_t buf0 = smem_u32(smem + warp * 2 * kTileBytes);
-  const uint8_t* my_buf0 = smem + warp * 2 * kTileBytes;
 
   const int64_t n_vec = static_cast<int64_t>(n_tokens) * hkv;
-  const int64_t tiles_per_tensor = (n_vec + kRows - 1) / kRows;
+  const int64_t tiles_per_tensor = (n_vec + kTileVecs - 1) / kTileVecs;
   const int64_t total_tiles = 2 * tiles_per_tensor;  // K tiles, then V tiles
-  const int64_t warp_id = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
-  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kWarps;
-
-  int64_t tile = warp_id;
-  if (tile >= total_tiles) return;
-  int stage = 0;
-  {
-    const bool isv = tile >= tiles_per_tensor;
-    stage_tile(buf0, isv ? v : k, n_vec, hkv, stride_bytes, isv ? tile - tiles_per_tensor : tile,
-               lane);
-    cp_async_commit();
-  }
-  for (; tile < total_tiles; tile += nwarps) {
-    const int64_t next = tile + nwarps;
-    if (next < total_tiles) {
-      const bool nv = next >= tiles_per_tensor;
-      stage_tile(buf0 + (stage ^ 1) * kTileBytes, nv ? v : k, n_vec, hkv, stride_bytes,
-                 nv ? next - tiles_per_tensor : next, lane);
-      cp_async_commit();
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
+  const int64_t grid = gridDim.x;
+  const uint32_t hb = smem_u32(sm.hm);
+  const uint32_t my_stg = smem_u32(sm.stg[warp][0]);
+  // my warp's rows of tile t into slot `slot` (a group is committed even when
+  // there is nothing to copy, which keeps the counting uniform)
+  auto stage = [&](int64_t t, int slot) {
+    if (t < total_tiles) {
+      const bool isv = t >= tiles_per_tensor;
+      stage_rows(my_stg + slot * kStageBytes, isv ? v : k, n_vec, hkv, stride_bytes,
+                 (isv ? t - tiles_per_tensor : t) * kTileVecs + kWarpRows * warp, lane);
     }
-    __syncwarp();
-
+    cp_async_commit();
+  };
+  int64_t tile = blockIdx.x;
+  stage(tile, 0);
+  stage(tile + grid, 1);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tlane = sm.tmem_base + (static_cast<uint32_t>(32 * warp) << 16);  // my lane
+  bool bad = false;
+  uint32_t ph = 0;
+  int slot = 0;
+  for (; tile < total_tiles; tile += grid) {
+    // my vector and its slot (the load overlaps the copies and the MMAs)
     const bool is_v = tile >= tiles_per_tensor;
-    const int64_t n = (is_v ? tile - tiles_per_tensor : tile) * kRows + lane;
-    if (n < n_vec) {
-      const int64_t tok = n / hkv;
-      const int h = static_cast<int>(n - tok * hkv);
-      const int32_t slot = slots[tok];
-      if (slot >= 0) {
-        const int32_t p = slot / kBlockSize;
-        if (p >= num_blocks) {
-          record_status(status, KVQ_ERR_OUT_OF_RANGE);
-        } else {
-          uint8_t* seg = pool + (static_cast<int64_t>(p) * hkv + h) * kSegBytes;
-          u64 P[64];
-          load_row<kBF16>(my_buf0 + stage * kTileBytes + lane * kPitch, P);
-          fwht_pairs(P);
-          if (is_v)
-            quantize_store<kVBits>(P, seg, slot % kBlockSize);
-          else
-            quantize_store<kKBits>(P, seg, slot % kBlockSize);
-        }
+    const int64_t n = (is_v ? tile - tiles_per_tensor : tile) * kTileVecs + tid;
+    const int64_t tok = n < n_vec ? token_of(n, n_vec, hkv) : 0;
+    const int32_t pslot = n < n_vec ? __ldg(slots + tok) : -1;
+
+    cp_async_wait<1>();  // my copies of this tile are done
+    __syncwarp();
+    uint32_t x[64];      // my row: 64 pairs of 16-bit elements
+    {
+      const uint8_t* row = reinterpret_cast<const uint8_t*>(sm.stg[warp][slot]) + lane * kPitch;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const uint4 q = *reinterpret_cast<const uint4*>(row + 16 * c);
+        x[4 * c] = q.x;
+        x[4 * c + 1] = q.y;
+        x[4 * c + 2] = q.z;
+        x[4 * c + 3] = q.w;
       }
     }
-    __syncwarp();
-    stage ^= 1;
+    __syncwarp();           // the slot is read
+    stage(tile + 2 * grid, slot);
+    tmem_st64(tlane + kColA, x);  // (the previous chain, which read A, is complete)
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+    tc_fence_before();
+    __syncthreads();  // A of every lane is written; y of the previous tile is read
+    tc_fence_after();
+    if (tid == 0) {
+#pragma unroll
+      for (int s = 0; s < kHeadDim / 16; ++s)
+        mma_f16_ta(sm.tmem_base + kColD, sm.tmem_base + kColA + 8 * s, sdesc(hb + 4096 * s, 2048, 128),
+                   idesc_h<kBF16>(), s > 0);
+      mma_commit(&sm.mma_done);
+    }
+    if (__syncthreads_or(!mbar_wait(&sm.mma_done, ph))) {  // (one decision for the CTA)
+      bad = true;
+      break;
+    }
+    ph ^= 1u;
+    tc_fence_after();
+
+    // every thread reads its lane (warp-collective loads); vectors without a
+    // slot in the pool are not stored
+    uint8_t* seg = nullptr;
+    if (pslot >= 0) {
+      const int32_t p = pslot / kBlockSize;
+      if (p >= num_blocks)
+        record_status(status, KVQ_ERR_OUT_OF_RANGE);
+      else
+        seg = pool + (static_cast<int64_t>(p) * hkv + static_cast<int>(n - tok * hkv)) * kSegBytes;
+    }
+    const float x0 = kBF16 ? bf16lo_to_f32(x[0]) : __half2float(__ushort_as_half(static_cast<uint16_t>(x[0])));
+    if (is_v)  // (uniform over the tile)
+      quantize_lane<kVBits>(tlane + kColD, x0, seg, pslot >= 0 ? pslot % kBlockSize : 0);
+    else
+      quantize_lane<kKBits>(tlane + kColD, x0, seg, pslot >= 0 ? pslot % kBlockSize : 0);
+    tc_fence_before();
+    slot ^= 1;
   }
+  cp_async_wait<0>();
+  if (bad) {
+    record_status(status, KVQ_ERR_DEVICE_TIMEOUT);
+    mbar_wait(&sm.mma_done, ph);  // (tensor memory is released only once the chain is complete)
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(sm.tmem_base), "n"(kBulkTmemCols));
 }
 
 
@@ -420,22 +573,21 @@ cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream) {
                         static_cast<const uint8_t*>(a.v), a.n_tokens, stride_bytes, a.slots, a.status);
     return cudaGetLastError();
   }
-  const int64_t tiles = 2 * ((n_vec + kRows - 1) / kRows);
-  const int smem = kWarps * 2 * kTileBytes;
-  const int sms = device_sm_count();
-  int64_t grid = (tiles + kWarps - 1) / kWarps;
-  const int64_t cap = static_cast<int64_t>(sms) * 3;
+  const int64_t tiles = 2 * ((n_vec + kTileVecs - 1) / kTileVecs);
+  const int smem = kBulkSmemBytes;
+  int64_t grid = tiles;
+  const int64_t cap = static_cast<int64_t>(device_sm_count()) * 2;  // two CTAs per SM, all resident
   if (grid > cap) grid = cap;
   if (a.in_dtype == KVQ_BF16) {
     const cudaError_t e = ensure_smem_limit<quantize_kernel<true>>(smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(quantize_kernel<true>, dim3(static_cast<unsigned>(grid)), dim3(kWarps * 32), smem, stream,
+    return launch_pdl(quantize_kernel<true>, dim3(static_cast<unsigned>(grid)), dim3(kBulkThreads), smem, stream,
                       a.pool, a.num_blocks, a.num_kv_heads, static_cast<const uint8_t*>(a.k),
                       static_cast<const uint8_t*>(a.v), a.n_tokens, stride_bytes, a.slots, a.status);
   } else {
     const cudaError_t e = ensure_smem_limit<quantize_kernel<false>>(smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(quantize_kernel<false>, dim3(static_cast<unsigned>(grid)), dim3(kWarps * 32), smem, stream,
+    return launch_pdl(quantize_kernel<false>, dim3(static_cast<unsigned>(grid)), dim3(kBulkThreads), smem, stream,
                       a.pool, a.num_blocks, a.num_kv_heads, static_cast<const uint8_t*>(a.k),
                       static_cast<const uint8_t*>(a.v), a.n_tokens, stride_bytes, a.slots, a.status);
   }

@@ -71,13 +71,16 @@ def _run_quantize(kvq, wl, slots, k, v, pool_fill=0x5A):
 
 
 # The write path takes a warp per head vector for small appends (at most 1024
-# head vectors per tensor) and a thread per head vector above that; both
-# paths are covered, with ragged tails.
+# head vectors per tensor) and tensor-core tiles of 128 head vectors above
+# that; both paths are covered, with ragged tails, and the tile path with
+# bf16 and fp16 inputs (the two forms of its MMA).
 @pytest.mark.parametrize("make", [lambda: synth.tiny(0),
                                   lambda: synth.Workload("q", 3, 16, 8, 128, [70, 1, 33], 16, synth.BF16, 3, 10.0,
                                                          30.0, seed=11),
                                   lambda: synth.Workload("qb", 2, 16, 8, 128, [70, 93], 16, synth.BF16, 3, 10.0,
-                                                         30.0, seed=14)])
+                                                         30.0, seed=14),
+                                  lambda: synth.Workload("qb16", 2, 16, 8, 128, [70, 93], 16, synth.F16, 3, 10.0,
+                                                         30.0, seed=16)])
 def test_quantize_matches_oracle(kvq, cuda, make):
     wl = make()
     k = wl.kv_rows(synth.TID_K, 0, wl.total_tokens)
@@ -97,6 +100,22 @@ def test_quantize_matches_oracle(kvq, cuda, make):
             if not written[p, 0, o]:
                 assert np.all(seg[p, :, o * 64:(o + 1) * 64] == 0x5A)
                 assert np.all(seg[p, :, 1024 + o * 32:1024 + (o + 1) * 32] == 0x5A)
+
+
+def test_quantize_bulk_many_tiles(kvq, cuda):
+    """More tiles than the persistent grid holds at once (two CTAs per SM):
+    every CTA walks several tiles through both operand buffers; a sample of
+    tokens (every 17th and the last eight) is checked against the oracle."""
+    wl = synth.Workload("qm", 2, 16, 8, 128, [1500, 1491], 16, synth.BF16, 3, 10.0, 30.0, seed=15)
+    T = wl.total_tokens
+    k = wl.kv_rows(synth.TID_K, 0, T)
+    v = wl.kv_rows(synth.TID_V, 0, T)
+    slots = wl.slots()
+    gpu = _run_quantize(kvq, wl, slots, k, v)
+    rep = helpers.QuantReport()
+    tokens = sorted(set(range(0, T, 17)) | set(range(T - 8, T)))
+    helpers.check_pool_tokens(rep, gpu, wl.num_blocks, wl.hkv, k, v, wl.dtype, slots, tokens)
+    assert rep.ok(), rep
 
 
 @pytest.mark.parametrize("n", [40, 600])
