@@ -16,10 +16,11 @@ figure with pinned host copies inside the timed region; and the CPU oracle's
 throughput on a bounded sample.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kvq|reference]
-                    [--profile qwen3-32b-16k|batched|long|mixed]
+                    [--profile qwen3-32b-16k|batched|long|mixed|prefill-quantize]
 
---profile times the decode kernel alone on one workload and prints its
-per-launch time; it is the command the ncu summaries are taken with.
+--profile times the decode kernel alone on one workload (or, with
+prefill-quantize, the bulk write path on 3 x 16384 fresh tokens) and prints
+its per-launch time; it is the command the ncu summaries are taken with.
 
 For N > 1 (torchrun), every rank runs an independent replica (the path has
 no cross-GPU step); the timing is the max over ranks and the value sums all
@@ -54,8 +55,8 @@ BYTES_PER_TOKEN_HEAD = 104
 # does), with the SHA-256 of the kernel code it was taken on (decode_code_sha256:
 # comments stripped).  Reported as roofline.traffic only while the code still
 # has that hash.
-DECODE_TRAFFIC = {"sha256": "3ba1317c4c2f07495b25bdddda1b3b934a72b4edec1735d8791ced7af0389c9d",
-                  "bytes": 13764096}
+DECODE_TRAFFIC = {"sha256": "eb70575cbebda52fd81531fda67b598333630517e393023daa3f9ece7e708d81",
+                  "bytes": 13764608}
 
 
 def decode_code_sha256():
@@ -497,11 +498,23 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=sorted(PROFILE_WORKLOADS), default=None,
-                    help="time decode launches alone on one workload (1 GPU; for ncu captures)")
+    ap.add_argument("--profile", choices=sorted(PROFILE_WORKLOADS) + ["prefill-quantize"], default=None,
+                    help="time decode launches alone on one workload, or the bulk quantize-append "
+                         "(1 GPU; for ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.profile == "prefill-quantize":
+        import torch
+        import bit_kv_cache_18_b200 as kvq
+        dev = torch.device("cuda", 0)
+        torch.cuda.set_device(dev)
+        r = prefill_quantize_gbs(kvq, torch, dev, seqs=3, reps=args.steps)
+        peak, kind = measured_peaks()
+        print(json.dumps({"profile": args.profile, "launches": args.steps, "us_per_launch": r["us"],
+                          "bytes_per_launch": r["bytes"], "gbs": r["gbs"], "frac": r["gbs"] / peak,
+                          "peak_kind": kind, "device_status": r["status"]}))
+        return 0
     if args.profile:
         return profile_decode(args)
     world, rank, local = dist_env()
