@@ -3,15 +3,14 @@
 // Bulk appends (prefill): the rotation of a tile of 128 head vectors is one
 // matrix product on the fifth-generation tensor cores, Y = X H with H the
 // 128 x 128 Sylvester Hadamard matrix (entries +-1, exact in bf16 and fp16,
-// accumulated in fp32).  Rows reach shared memory through 16-byte cp.async
-// copies laid out as the no-swizzle K-major operand (eight lanes write 128
-// contiguous bytes; each source row is read 64 bytes at a time), one thread
-// issues the 8-step tcgen05.mma chain into 128 fp32 tensor-memory columns,
-// and thread t then owns vector t (tensor-memory lane t): moments, range and
-// (S, Z) from one pass over its columns, the codes from a second, packed
-// with fp32x2 arithmetic and written as 16-byte stores into the paged
-// segment plus two fp16 stores.  Two operand buffers per CTA let the copies
-// of the next tiles run under the current tile's arithmetic.
+// accumulated in fp32).  Each warp stages its 32 rows two tiles ahead with
+// coalesced 16-byte cp.async copies, each lane moves its row, unconverted,
+// into its tensor-memory lane (the A operand), one thread issues the 8-step
+// tcgen05.mma chain (B = H in shared memory) into 128 fp32 columns, and
+// thread t then owns vector t (tensor-memory lane t): one read of its
+// columns gives the moments, range, (S, Z) and codes, packed with fp32x2
+// arithmetic and written as 16-byte stores into the paged segment plus two
+// fp16 stores.  Two CTAs per SM overlap each other's MMA waits.
 //
 // Small appends (decode steps): one warp per vector (quantize_vector_warp in
 // kvq_internal.cuh), butterflies in registers and shuffles.
