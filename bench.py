@@ -334,7 +334,12 @@ def time_replays(torch, g, n, barrier=None, pre=None, post=None):
     return e0.elapsed_time(e1)
 
 
-def prefill_quantize_gbs(kvq, torch, dev, seed=0, seqs=16, tokens=16384, reps=10):
+def seg_bytes(preset):
+    """Bytes of one (block, kv head) segment: 16 rows of K and V codes + 4 x 16 fp16."""
+    return 16 * 128 * (preset[0] + preset[1]) // 8 + 128
+
+
+def prefill_quantize_gbs(kvq, torch, dev, seed=0, seqs=16, tokens=16384, reps=10, preset=(4, 2)):
     """Quantize-append of 16 x 16384 fresh tokens, 8 kv heads, bf16."""
     hkv = 8
     T = seqs * tokens
@@ -348,21 +353,54 @@ def prefill_quantize_gbs(kvq, torch, dev, seed=0, seqs=16, tokens=16384, reps=10
     perm = synth.permutation(seed, synth.TID_PERM, nblocks).astype(np.int64)
     slots = (perm[np.arange(T) // 16] * 16 + np.arange(T) % 16).astype(np.int32)
     sl = torch.from_numpy(slots).to(dev)
-    pool = kvq.new_pool(nblocks, hkv, device=dev)
-    kvq.kvq_quantize_append(pool, nblocks, hkv, k, v, sl)
+    pool = kvq.new_pool(nblocks, hkv, device=dev, preset=preset)
+    kvq.kvq_quantize_append(pool, nblocks, hkv, k, v, sl, preset=preset)
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(reps):
-        kvq.kvq_quantize_append(pool, nblocks, hkv, k, v, sl)
+        kvq.kvq_quantize_append(pool, nblocks, hkv, k, v, sl, preset=preset)
     e1.record()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / reps
-    nbytes = T * hkv * (2 * 128 * 2 + BYTES_PER_TOKEN_HEAD) + T * 4
+    nbytes = T * hkv * (2 * 128 * 2 + seg_bytes(preset) // 16) + T * 4
     status = kvq.kvq_last_device_status()
     del k, v, pool, kb
     return {"us": ms * 1e3, "gbs": nbytes / (ms * 1e-3) / 1e9, "bytes": nbytes, "status": status}
+
+
+def preset_decode_gbs(kvq, torch, dev, preset, batch=32, context=8192, reps=10):
+    """Decode of batch x context tokens (64/8 heads) on a pool of the preset
+    larger than L2: random code bytes with fp16 factors 0.01 (the work does
+    not depend on the values); µs per launch and GB/s on packed bytes."""
+    wl = synth.mixed_decode(0, batch=batch, context=context)
+    seg = seg_bytes(preset)
+    pool = torch.empty(wl.num_blocks * wl.hkv * seg, dtype=torch.uint8, device=dev).random_(0, 256)
+    pool.view(wl.num_blocks * wl.hkv, seg)[:, seg - 128:].view(torch.float16).fill_(0.01)
+    q = torch.randn(wl.batch, wl.hq, 128, device=dev, dtype=torch.bfloat16)
+    bt = torch.from_numpy(wl.block_table).to(dev)
+    lens = torch.from_numpy(wl.seq_lens).to(dev)
+    out = torch.empty(wl.batch, wl.hq, 128, device=dev, dtype=torch.bfloat16)
+    ws = kvq.new_workspace(wl.num_blocks, wl.hkv, wl.batch, wl.hq, context, device=dev, preset=preset)
+
+    def launch():
+        kvq.kvq_decode_attention(pool, wl.num_blocks, wl.hkv, q, bt, lens, context, out, ws, preset=preset)
+
+    for _ in range(3):
+        launch()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        launch()
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / reps
+    nbytes = batch * context * wl.hkv * seg // 16
+    status = kvq.kvq_last_device_status()
+    del pool, ws
+    return {"us": us, "gbs": nbytes / (us * 1e-6) / 1e9, "bytes": nbytes, "status": status}
 
 
 # --------------------------------------------------------------------------- CPU oracle
@@ -563,6 +601,18 @@ def main():
     e2e_ms_max, e2e_tokens = aggregate(dist, e2e_ms, args.steps * stepper.tokens_per_step(), dev)
 
     quant = prefill_quantize_gbs(kvq, torch, dev)
+    # every preset on the same shapes: decode of 32 x 8192 tokens and the
+    # prefill append of 4 x 16384 tokens (the default preset included, for
+    # comparison)
+    presets = {}
+    for pr in kvq.PRESETS:
+        dq = preset_decode_gbs(kvq, torch, dev, pr)
+        pq = prefill_quantize_gbs(kvq, torch, dev, seqs=4, reps=5, preset=pr)
+        presets[f"kvarn_k{pr[0]}v{pr[1]}_g128"] = {
+            "segment_bytes": seg_bytes(pr),
+            "decode_32x8192": {"us": dq["us"], "gbs": dq["gbs"], "frac": dq["gbs"] / measured_peaks()[0]},
+            "quantize_4x16384": {"us": pq["us"], "gbs": pq["gbs"], "frac": pq["gbs"] / measured_peaks()[0]},
+            "device_status": dq["status"] or pq["status"]}
     status = kvq.kvq_last_device_status()
 
     cpu = None
@@ -593,6 +643,7 @@ def main():
                        "context_tokens_per_s": stepper.context * stepper.batch / (dms * 1e-3)},
             "quantize": {"workload": "prefill append 16 x 16384 tokens, 8 kv heads, bf16", "us": quant["us"],
                          "gbs": quant["gbs"], "bytes": quant["bytes"], "frac": quant["gbs"] / peak},
+            "presets": presets,
             "e2e": {"value": e2e_tokens / (e2e_ms_max * 1e-3), "unit": "tokens/s",
                     "h2d_bytes_per_step": stepper.h_in.numel() * 2, "d2h_bytes_per_step": stepper.h_out.numel() * 2},
             "gpu_launches": stepper.launches_per_step() * args.steps,

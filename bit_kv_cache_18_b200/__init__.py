@@ -126,8 +126,13 @@ def kvq_parse_dtype(s: str):
     return rc, (kb.value, vb.value, g.value)
 
 
-def make_desc(num_blocks: int, num_kv_heads: int, pool=None) -> CacheDesc:
-    return CacheDesc(num_blocks, BLOCK_SIZE, num_kv_heads, HEAD_DIM, 4, 2, HEAD_DIM,
+# The cache presets the library builds, as (key bits, value bits); the first
+# is the pages' default, kvarn_k4v2_g128.
+PRESETS = ((4, 2), (4, 4), (2, 2), (8, 4))
+
+
+def make_desc(num_blocks: int, num_kv_heads: int, pool=None, preset=(4, 2)) -> CacheDesc:
+    return CacheDesc(num_blocks, BLOCK_SIZE, num_kv_heads, HEAD_DIM, preset[0], preset[1], HEAD_DIM,
                      pool.data_ptr() if pool is not None else None)
 
 
@@ -159,17 +164,18 @@ def kvq_slot_mapping(block_table, positions, seq_ids, block_size=BLOCK_SIZE):
 
 # ---- device calls ------------------------------------------------------------
 
-def new_pool(num_blocks: int, num_kv_heads: int, device="cuda"):
+def new_pool(num_blocks: int, num_kv_heads: int, device="cuda", preset=(4, 2)):
     """A caller-owned pool tensor (uint8) sized by kvq_cache_bytes."""
     import torch
-    nbytes = kvq_cache_bytes(make_desc(num_blocks, num_kv_heads))
+    nbytes = kvq_cache_bytes(make_desc(num_blocks, num_kv_heads, preset=preset))
     return torch.zeros(nbytes, dtype=torch.uint8, device=device)
 
 
-def kvq_quantize_append(pool, num_blocks, num_kv_heads, k, v, slot_mapping, stream=None, token_stride=None):
+def kvq_quantize_append(pool, num_blocks, num_kv_heads, k, v, slot_mapping, stream=None, token_stride=None,
+                        preset=(4, 2)):
     """k, v: [n_tokens, ..., Hkv*128 elements per row] fp16/bf16 device tensors
     with stride(0) = token_stride; slot_mapping: int32 device [n_tokens]."""
-    desc = make_desc(num_blocks, num_kv_heads, pool)
+    desc = make_desc(num_blocks, num_kv_heads, pool, preset)
     n = int(slot_mapping.numel())
     ts = k.stride(0) if token_stride is None else token_stride
     rc = lib().kvq_quantize_append(ctypes.byref(desc), _ptr(k), _ptr(v), _dtype_code(k), n, ts, _ptr(slot_mapping),
@@ -177,25 +183,28 @@ def kvq_quantize_append(pool, num_blocks, num_kv_heads, k, v, slot_mapping, stre
     _check(rc, "kvq_quantize_append")
 
 
-def kvq_decode_workspace_bytes(num_blocks, num_kv_heads, batch, num_q_heads, max_seq_len, blocks_per_split=0):
-    desc = make_desc(num_blocks, num_kv_heads)
+def kvq_decode_workspace_bytes(num_blocks, num_kv_heads, batch, num_q_heads, max_seq_len, blocks_per_split=0,
+                               preset=(4, 2)):
+    desc = make_desc(num_blocks, num_kv_heads, preset=preset)
     return lib().kvq_decode_workspace_bytes_ex(ctypes.byref(desc), batch, num_q_heads, max_seq_len,
                                                blocks_per_split)
 
 
-def new_workspace(num_blocks, num_kv_heads, batch, num_q_heads, max_seq_len, blocks_per_split=0, device="cuda"):
+def new_workspace(num_blocks, num_kv_heads, batch, num_q_heads, max_seq_len, blocks_per_split=0, device="cuda",
+                  preset=(4, 2)):
     import torch
-    n = kvq_decode_workspace_bytes(num_blocks, num_kv_heads, batch, num_q_heads, max_seq_len, blocks_per_split)
+    n = kvq_decode_workspace_bytes(num_blocks, num_kv_heads, batch, num_q_heads, max_seq_len, blocks_per_split,
+                                   preset)
     if n == 0:
         raise KvqError(KVQ_ERR_UNSUPPORTED, "kvq_decode_workspace_bytes")
     return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
 def kvq_decode_attention(pool, num_blocks, num_kv_heads, q, block_table, seq_lens, max_seq_len, out, workspace,
-                         softmax_scale=0.0, blocks_per_split=0, stream=None):
+                         softmax_scale=0.0, blocks_per_split=0, stream=None, preset=(4, 2)):
     """q: [batch, Hq, 128] device; block_table int32 [batch, max_blocks]; seq_lens int32 [batch];
     out: [batch, Hq, 128] device (fp32/bf16/fp16); workspace from new_workspace()."""
-    desc = make_desc(num_blocks, num_kv_heads, pool)
+    desc = make_desc(num_blocks, num_kv_heads, pool, preset)
     batch, hq, _ = q.shape
     rc = lib().kvq_decode_attention_ex(ctypes.byref(desc), _ptr(q), _dtype_code(q), batch, hq, _ptr(block_table),
                                        block_table.shape[1], _ptr(seq_lens), max_seq_len, softmax_scale, _ptr(out),
@@ -205,11 +214,11 @@ def kvq_decode_attention(pool, num_blocks, num_kv_heads, q, block_table, seq_len
 
 
 def kvq_append_decode_attention(pool, num_blocks, num_kv_heads, k_new, v_new, q, block_table, seq_lens, max_seq_len,
-                                out, workspace, softmax_scale=0.0, stream=None, token_stride=None):
+                                out, workspace, softmax_scale=0.0, stream=None, token_stride=None, preset=(4, 2)):
     """One fused decode step: the new token of each sequence (k_new, v_new:
     [batch, ..., Hkv*128] fp16/bf16 rows) is quantized into position
     seq_lens[b] - 1, then decode attention runs over the grown cache."""
-    desc = make_desc(num_blocks, num_kv_heads, pool)
+    desc = make_desc(num_blocks, num_kv_heads, pool, preset)
     batch, hq, _ = q.shape
     ts = k_new.stride(0) if token_stride is None else token_stride
     rc = lib().kvq_append_decode_attention(ctypes.byref(desc), _ptr(k_new), _ptr(v_new), _dtype_code(k_new), ts,
@@ -221,10 +230,10 @@ def kvq_append_decode_attention(pool, num_blocks, num_kv_heads, k_new, v_new, q,
 
 
 def kvq_decode_attention_noalloc(pool, num_blocks, num_kv_heads, q, block_table, seq_lens, max_seq_len, out,
-                                 softmax_scale=0.0, stream=None):
+                                 softmax_scale=0.0, stream=None, preset=(4, 2)):
     """kvq_decode_attention with the library's fixed device scratch instead of
     a caller workspace (for callers that cannot allocate at call time)."""
-    desc = make_desc(num_blocks, num_kv_heads, pool)
+    desc = make_desc(num_blocks, num_kv_heads, pool, preset)
     batch, hq, _ = q.shape
     rc = lib().kvq_decode_attention_noalloc(ctypes.byref(desc), _ptr(q), _dtype_code(q), batch, hq,
                                             _ptr(block_table), block_table.shape[1], _ptr(seq_lens), max_seq_len,

@@ -110,13 +110,14 @@ constexpr uint32_t kIdescPV =
 //   qb (B of QK, K-major):  byte (n, pos)   at (pos/16)*512 + (n/8)*128    + (n%8)*16   + pos%16
 // S column n = 8j + g holds digit j of head g (rows 24..31 of qb are zero);
 // P' and O column n = 4g + j hold byte j of head g.
+template <int kSeg>  // segment bytes of the preset
 struct __align__(1024) Smem {
   uint8_t vt[kNV][kChunkTokens * kHeadDim];  // 3 x 16 KB
   uint8_t pm[kNV][kChunkTokens * 32];        // 3 x 4 KB
   uint8_t qb[32 * kHeadDim];                 // 4 KB
   float meta[kNV][4][kChunkTokens];          // per token: S_K c1, Z_K, S_V 2^27 (< 0: no token), Z_V
   union {
-    uint8_t stg[kLoadWarps][kNV][2 * kSegBytes];  // loader warp w: its two segments of chunk c in slot c % 3
+    uint8_t stg[kLoadWarps][kNV][2 * kSeg];  // loader warp w: its two segments of chunk c in slot c % 3
     float obuf[8][kHeadDim];                      // o~ (epilogue, after the scan)
   };
   float2 hq[8];                              // per head: sum(q~), max|q~|
@@ -134,8 +135,11 @@ struct __align__(1024) Smem {
   int is_last;
   int abort;              // a wait ran out: every other wait gives up at once
 };
-constexpr int kSmemBytes = static_cast<int>((sizeof(Smem) + 1023) / 1024 * 1024);
-static_assert(kSmemBytes <= 113 * 1024, "two CTAs per SM");
+template <int kSeg>
+constexpr int kSmemBytesOf = static_cast<int>((sizeof(Smem<kSeg>) + 1023) / 1024 * 1024);
+static_assert(kSmemBytesOf<Fmt<4, 2>::kSegBytes> <= 113 * 1024, "two CTAs per SM (k4v2)");
+static_assert(kSmemBytesOf<Fmt<2, 2>::kSegBytes> <= 113 * 1024, "two CTAs per SM (k2v2)");
+static_assert(kSmemBytesOf<Fmt<8, 4>::kSegBytes> <= 227 * 1024, "one CTA per SM (k8v4)");
 
 // Position in a ring of three buffers and the parity of its current use.
 struct Ring3 {
@@ -186,7 +190,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 // Bounded, warp-uniform wait for a barrier phase.  False if it never came or
 // another warp already gave up (then every later wait returns at once and
-// the kernel runs to its end on void data, which it reports).
+// the kernel runs to its end on void data, which it reports).  The slow loop
+// is a call, one copy per preset (kTag), which keeps the wait sites small.
+template <int kTag>
 __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort) {
   for (uint32_t it = 0; it < kWaitLimit; ++it) {
     if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
@@ -195,9 +201,10 @@ __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, vola
   *abort = 1;
   return false;
 }
+template <int kTag>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
-  return mbar_wait_slow(bar, parity, abort);
+  return mbar_wait_slow<kTag>(bar, parity, abort);
 }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -316,12 +323,106 @@ __device__ __forceinline__ void fwht_warp(float (&x)[4], int lane, float scale) 
   for (int k = 0; k < 4; ++k) x[k] *= f;
 }
 
-// Position of dim d in a spread key row, and dim of position p in a spread
-// value row (the byte-spreading orders of the file comment).
+// Position of dim d in a spread key row of KB-bit codes (with 32m + 8j + 4h
+// + b the byte b of column 8j + 2(l%4) + h written by lane l, m = l%4):
+//   KB = 4: position 32j + 8m + 4h + b holds dim 32m + 8j + 2b + h
+//   KB = 8: position 32j + 8m + e holds dim 32m + 8j + e (the raw bytes)
+//   KB = 2: position 32j + 8m + 4h + b holds dim 32m + 16(j/2) + 4b + 2(j%2) + h
+template <int KB>
 __device__ __forceinline__ int key_pos_of_dim(int d) {
-  return ((d >> 3) & 3) << 5 | (d >> 5) << 3 | (d & 1) << 2 | ((d >> 1) & 3);
+  const int m = d >> 5, r = d & 31;
+  if (KB == 4) return ((r >> 3) & 3) << 5 | m << 3 | (r & 1) << 2 | ((r >> 1) & 3);
+  if (KB == 8) return ((r >> 3) & 3) << 5 | m << 3 | (r & 7);
+  const int j = 2 * (r >> 4) + ((r >> 1) & 1);
+  return j << 5 | m << 3 | (r & 1) << 2 | ((r >> 2) & 3);
 }
-__device__ __forceinline__ int value_dim_of_pos(int p) { return (p & ~15) | ((p & 3) << 2) | ((p >> 2) & 3); }
+// Dim of position p in a spread value row and log2 of the factor the spread
+// multiplied its code by:
+//   VB = 2: position 16i + 4k + b holds dim 16i + 4b + k, times 4^k
+//   VB = 4: position 32m + 16h + 4w + b holds dim 32m + 8w + 2b + h, times 16^h
+template <int VB>
+__device__ __forceinline__ int value_dim_of_pos(int p) {
+  if (VB == 2) return (p & ~15) | ((p & 3) << 2) | ((p >> 2) & 3);
+  return (p & ~31) | (((p >> 2) & 3) << 3) | ((p & 3) << 1) | ((p >> 4) & 1);
+}
+template <int VB>
+__device__ __forceinline__ uint32_t value_scale_log2(int p) {
+  return VB == 2 ? 2u * ((p >> 2) & 3) : 4u * ((p >> 4) & 1);
+}
+
+// Raw key codes of one segment row pair for lane l (rows l/4 and 8 + l/4,
+// dims 32(l%4) .. +31 of each) and their spread into the 16 words of a
+// tcgen05.st.16x256b.x4 (registers 4j, 4j+1: row l/4, columns
+// 8j + 2(l%4) + 0/1; registers 4j+2, 4j+3: row 8 + l/4).
+template <int KB>
+struct KeyRaw;
+template <>
+struct KeyRaw<4> {
+  uint4 a, b;
+  __device__ __forceinline__ void load(uint32_t k, int lane);
+  __device__ __forceinline__ void spread(uint32_t (&w)[16]) const;
+};
+template <>
+struct KeyRaw<8> {
+  uint4 a0, a1, b0, b1;
+  __device__ __forceinline__ void load(uint32_t k, int lane);
+  __device__ __forceinline__ void spread(uint32_t (&w)[16]) const;
+};
+template <>
+struct KeyRaw<2> {
+  uint2 a, b;
+  __device__ __forceinline__ void load(uint32_t k, int lane);
+  __device__ __forceinline__ void spread(uint32_t (&w)[16]) const;
+};
+// 4-bit: 16 bytes of each row; nibbles to bytes (even dims, odd dims)
+__device__ __forceinline__ void KeyRaw<4>::load(uint32_t k, int lane) {
+  a = lds128(k + 16 * lane);
+  b = lds128(k + 512 + 16 * lane);
+}
+__device__ __forceinline__ void KeyRaw<4>::spread(uint32_t (&w)[16]) const {
+  const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    w[4 * j] = wa[j] & 0x0F0F0F0Fu;
+    w[4 * j + 1] = (wa[j] >> 4) & 0x0F0F0F0Fu;
+    w[4 * j + 2] = wb[j] & 0x0F0F0F0Fu;
+    w[4 * j + 3] = (wb[j] >> 4) & 0x0F0F0F0Fu;
+  }
+}
+// 8-bit: 32 bytes of each row, already one code per byte
+__device__ __forceinline__ void KeyRaw<8>::load(uint32_t k, int lane) {
+  a0 = lds128(k + 32 * lane);
+  a1 = lds128(k + 32 * lane + 16);
+  b0 = lds128(k + 1024 + 32 * lane);
+  b1 = lds128(k + 1024 + 32 * lane + 16);
+}
+__device__ __forceinline__ void KeyRaw<8>::spread(uint32_t (&w)[16]) const {
+  const uint32_t wa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+  const uint32_t wb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    w[4 * j] = wa[2 * j];
+    w[4 * j + 1] = wa[2 * j + 1];
+    w[4 * j + 2] = wb[2 * j];
+    w[4 * j + 3] = wb[2 * j + 1];
+  }
+}
+// 2-bit: 8 bytes of each row; word u, shift 2k -> register 4(2u + k/2) + k%2
+__device__ __forceinline__ void KeyRaw<2>::load(uint32_t k, int lane) {
+  a = lds64(k + 8 * lane);
+  b = lds64(k + 256 + 8 * lane);
+}
+__device__ __forceinline__ void KeyRaw<2>::spread(uint32_t (&w)[16]) const {
+  const uint32_t wa[2] = {a.x, a.y}, wb[2] = {b.x, b.y};
+#pragma unroll
+  for (int u = 0; u < 2; ++u)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int j = 2 * u + (k >> 1), hh = k & 1;
+      w[4 * j + hh] = (wa[u] >> (2 * k)) & 0x03030303u;
+      w[4 * j + 2 + hh] = (wb[u] >> (2 * k)) & 0x03030303u;
+    }
+}
 
 // Bounded wait that ignores the abort flag: the issuer's last wait for its
 // own MMAs, so tensor memory is never released under a running MMA.
@@ -330,10 +431,17 @@ __device__ __forceinline__ bool mbar_wait_final(uint64_t* bar, uint32_t parity) 
     if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
   return false;
 }
-template <int G>
-__global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
+// CTAs per SM the shared memory of a preset allows (two for k4v2 and k2v2).
+template <int KB, int VB>
+constexpr int kMinCtasOf = kSmemBytesOf<Fmt<KB, VB>::kSegBytes> <= 113 * 1024 ? 2 : 1;
+
+template <int G, int KB, int VB>
+__global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(DecodeArgs a) {
+  using F = Fmt<KB, VB>;
+  constexpr int kSeg = F::kSegBytes;
+  constexpr int kWaitTag = 16 * KB + VB;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
+  Smem<kSeg>& sm = *reinterpret_cast<Smem<kSeg>*>(smem_raw);
   volatile int* abort = &sm.abort;
   const int split = blockIdx.x;
   const int h = blockIdx.y;
@@ -420,8 +528,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
   bool bad = false;      // a wait ran out: the results are void, the control flow is kept
   bool bad_blk = false;  // a block-table entry outside the pool (its tokens are skipped)
 
-  const uint8_t* pool_h = a.pool + static_cast<int64_t>(h) * kSegBytes;
-  const int64_t pstride = static_cast<int64_t>(a.num_kv_heads) * kSegBytes;
+  const uint8_t* pool_h = a.pool + static_cast<int64_t>(h) * kSeg;
+  const int64_t pstride = static_cast<int64_t>(a.num_kv_heads) * kSeg;
   const int mseg = lane >> 4;  // segment of my factor bytes
 
   // physical block of segment lane & 1 of my warp in chunk c (-1: none)
@@ -430,7 +538,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
     return blk < blk1 ? __ldg(bt_row + blk) : -1;
   };
   auto prefetch_seg = [&](int32_t p) {
-    if (lane < 2 && p >= 0 && p < a.num_blocks) prefetch_l2(pool_h + static_cast<int64_t>(p) * pstride, kSegBytes);
+    if (lane < 2 && p >= 0 && p < a.num_blocks) prefetch_l2(pool_h + static_cast<int64_t>(p) * pstride, kSeg);
   };
   const uint32_t my_stg = smem_u32(sm.stg[warp < kLoadWarps ? warp : 0][0]);
   // lanes 0 and 1: bulk copy of segment lane & 1 of chunk c (block p) into
@@ -443,10 +551,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
     if (lane < 2) {
       bad_blk |= live && !ok;
       uint64_t* bar = &sm.full[warp][slot];
-      if (lane == 0) mbar_arrive_expect_tx(bar, a.num_blocks > 0 ? 2u * kSegBytes : 0u);
+      if (lane == 0) mbar_arrive_expect_tx(bar, a.num_blocks > 0 ? 2u * kSeg : 0u);
       if (a.num_blocks > 0)  // (an empty pool has no block 0 to stand in)
-        bulk_g2s(my_stg + slot * (2 * kSegBytes) + lane * kSegBytes,
-                 pool_h + static_cast<int64_t>(ok ? p : 0) * pstride, kSegBytes, bar);
+        bulk_g2s(my_stg + slot * (2 * kSeg) + lane * kSeg, pool_h + static_cast<int64_t>(ok ? p : 0) * pstride, kSeg,
+                 bar);
     }
     return __ballot_sync(0xffffffffu, ok && lane < 2) & 3u;
   };
@@ -499,9 +607,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
         if (p >= 0 && p < a.num_blocks) {
           uint8_t* seg = const_cast<uint8_t*>(pool_h) + static_cast<int64_t>(p) * pstride;
           if (a.new_bf16)
-            quantize_vector_warp_raw<true>(new_raw, seg, (L - 1) % kBlockSize, sw == 1, lane);
+            quantize_vector_warp_raw<true, KB, VB>(new_raw, seg, (L - 1) % kBlockSize, sw == 1, lane);
           else
-            quantize_vector_warp_raw<false>(new_raw, seg, (L - 1) % kBlockSize, sw == 1, lane);
+            quantize_vector_warp_raw<false, KB, VB>(new_raw, seg, (L - 1) % kBlockSize, sw == 1, lane);
           asm volatile("fence.proxy.async.global;" ::: "memory");
         } else if (lane == 0) {
           record_status(a.status, KVQ_ERR_OUT_OF_RANGE);
@@ -538,7 +646,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
       if (g < G) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const int pos = key_pos_of_dim(lane + 32 * k);
+          const int pos = key_pos_of_dim<KB>(lane + 32 * k);
           const float y = x[i][k] * inv;
           const float q1 = rintf(y);
           const float r1 = (y - q1) * 254.0f;
@@ -568,9 +676,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
   // ---- 1. the paged scan ------------------------------------------------------
   if (is_loader) {
     const uint32_t my_lanes = tbase + (static_cast<uint32_t>(warp * 32) << 16);
-    // my value rows: row lane/2 of segment s, dims 64 (lane%2) + [0, 64)
-    const uint32_t my_vt = smem_u32(sm.vt[0]) + ((32 * warp + (lane >> 1)) >> 3) * 1024 + (lane & 1) * 512 +
-                           (lane >> 1 & 7) * 16;  // segment 1: + 2048
+    // my value rows, segment 1: + 2048.  VB = 2: row lane/2 of the segment,
+    // positions 64 (lane%2) + [0, 64); VB = 4: rows lane/4 and (+ 1024)
+    // 8 + lane/4, positions 32 (lane%4) + [0, 32)
+    const uint32_t my_vt =
+        VB == 2 ? smem_u32(sm.vt[0]) + ((32 * warp + (lane >> 1)) >> 3) * 1024 + (lane & 1) * 512 +
+                      (lane >> 1 & 7) * 16
+                : smem_u32(sm.vt[0]) + 4 * warp * 1024 + (lane >> 2) * 16 + 2 * (lane & 3) * 128;
     const int mrow0 = 4 * (lane & 3);    // my factor rows mrow0 .. mrow0+3 of segment mseg
     const int mkind = (lane >> 2) & 3;  // S_K, Z_K, S_V, Z_V
     const float mscale = mkind == 0 ? c1 : (mkind == 2 ? kFix : 1.0f);
@@ -582,16 +694,17 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
     Ring3 r{0, 0u};  // chunk c: staging slot, key-code, value and factor buffers r.i
 #pragma unroll 1
     for (int c = 0; c < nchunks; ++c) {
-      if (!mbar_wait(&sm.full[warp][r.i], r.ph, abort)) bad = true;
-      const uint32_t sb = my_stg + r.i * (2 * kSegBytes);
-      uint4 kr[4], vr[2];
+      if (!mbar_wait<kWaitTag>(&sm.full[warp][r.i], r.ph, abort)) bad = true;
+      const uint32_t sb = my_stg + r.i * (2 * kSeg);
+      KeyRaw<KB> kr[2];
+      uint4 vr[2][VB / 2];  // VB = 2: one 16-byte piece per segment; VB = 4: two
 #pragma unroll
       for (int sg = 0; sg < 2; ++sg) {
-        kr[2 * sg] = lds128(sb + sg * kSegBytes + kOffK + 16 * lane);
-        kr[2 * sg + 1] = lds128(sb + sg * kSegBytes + kOffK + 512 + 16 * lane);
-        vr[sg] = lds128(sb + sg * kSegBytes + kOffV + 16 * lane);
+        kr[sg].load(sb + sg * kSeg + F::kOffK, lane);
+#pragma unroll
+        for (int i = 0; i < VB / 2; ++i) vr[sg][i] = lds128(sb + sg * kSeg + F::kOffV + 512 * i + 16 * lane);
       }
-      const uint2 mr2 = lds64(sb + mseg * kSegBytes + kOffSK + 8 * (lane & 15));
+      const uint2 mr2 = lds64(sb + mseg * kSeg + F::kOffSK + 8 * (lane & 15));
       const uint32_t ok = okq[0];
       // the slot is read: refill it with chunk c+3 (the reads above are
       // ordered before the copy's writes by the proxy fence)
@@ -606,31 +719,32 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
       bq[5] = bid_of(c + kNV + 6);
 
       if (c >= kNV) {  // buffers r.i are free once PV(c-3) (issued after QK(c-2)) is done
-        if (!mbar_wait(&sm.pv_done[r.i], r.ph ^ 1u, abort)) bad = true;
+        if (!mbar_wait<kWaitTag>(&sm.pv_done[r.i], r.ph ^ 1u, abort)) bad = true;
         tc_fence_after();
       }
 #pragma unroll
       for (int sg = 0; sg < 2; ++sg) {  // key codes of segment sg -> lanes 32 warp + 16 sg + [0, 16)
-        const uint4 ka = kr[2 * sg], kb = kr[2 * sg + 1];
-        const uint32_t wa[4] = {ka.x, ka.y, ka.z, ka.w}, wb[4] = {kb.x, kb.y, kb.z, kb.w};
         uint32_t w[16];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          w[4 * j] = wa[j] & 0x0F0F0F0Fu;
-          w[4 * j + 1] = (wa[j] >> 4) & 0x0F0F0F0Fu;
-          w[4 * j + 2] = wb[j] & 0x0F0F0F0Fu;
-          w[4 * j + 3] = (wb[j] >> 4) & 0x0F0F0F0Fu;
-        }
+        kr[sg].spread(w);
         tmem_st16x256(my_lanes + (static_cast<uint32_t>(16 * sg) << 16) + kColA + 32 * r.i, w);
       }
 #pragma unroll
       for (int sg = 0; sg < 2; ++sg) {  // value codes, one byte each
         const uint32_t va = my_vt + sg * 2048 + r.i * (kChunkTokens * kHeadDim);
-        const uint32_t vw[4] = {vr[sg].x, vr[sg].y, vr[sg].z, vr[sg].w};
+        if (VB == 2) {  // crumb k of each byte -> position 16i + 4k + b, times 4^k
+          const uint32_t vw[4] = {vr[sg][0].x, vr[sg][0].y, vr[sg][0].z, vr[sg][0].w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint32_t x = vw[i];
-          sts128(va + 128 * i, x & 0x03030303u, x & 0x0C0C0C0Cu, x & 0x30303030u, x & 0xC0C0C0C0u);
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t x = vw[i];
+            sts128(va + 128 * i, x & 0x03030303u, x & 0x0C0C0C0Cu, x & 0x30303030u, x & 0xC0C0C0C0u);
+          }
+        } else {  // nibble h of byte b of word w -> position 16h + 4w + b, times 16^h
+#pragma unroll
+          for (int i = 0; i < VB / 2; ++i) {  // rows lane/4 and 8 + lane/4
+            const uint4 x = vr[sg][i];
+            sts128(va + 1024 * i, x.x & 0x0F0F0F0Fu, x.y & 0x0F0F0F0Fu, x.z & 0x0F0F0F0Fu, x.w & 0x0F0F0F0Fu);
+            sts128(va + 1024 * i + 128, x.x & 0xF0F0F0F0u, x.y & 0xF0F0F0F0u, x.z & 0xF0F0F0F0u, x.w & 0xF0F0F0F0u);
+          }
         }
       }
       {  // factors of my four rows; absent tokens get 0 (S_V: -1)
@@ -659,8 +773,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
     for (int c = 0; c <= nchunks; ++c) {
       if (c < nchunks) {  // QK(c): its codes are in, and S buffer c % 2 was read (chunk c-2)
         const int P = c & 1;
-        if (!mbar_wait(&sm.kv_ready[rq.i], rq.ph, abort)) bad = true;
-        if (c >= kNS && !mbar_wait(&sm.s_free[P], static_cast<uint32_t>(((c - kNS) >> 1) & 1), abort)) bad = true;
+        if (!mbar_wait<kWaitTag>(&sm.kv_ready[rq.i], rq.ph, abort)) bad = true;
+        if (c >= kNS && !mbar_wait<kWaitTag>(&sm.s_free[P], static_cast<uint32_t>(((c - kNS) >> 1) & 1), abort)) bad = true;
         tc_fence_after();
         if (lane == 0) {
           const uint32_t acol = tbase + kColA + 32 * rq.i, scol = tbase + kColS + 32 * P;
@@ -672,7 +786,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
         rq.next();
       }
       if (c >= 1) {  // PV(c-1) once its P' is written
-        if (!mbar_wait(&sm.p_ready[rp.i], rp.ph, abort)) bad = true;
+        if (!mbar_wait<kWaitTag>(&sm.p_ready[rp.i], rp.ph, abort)) bad = true;
         tc_fence_after();
         if (lane == 0) {
           const bool fresh = sm.fresh[rp.i] != 0;
@@ -696,7 +810,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
     const uint32_t my_lanes = tbase + (static_cast<uint32_t>(sw * 32) << 16);
     const uint32_t my_pm = smem_u32(sm.pm[0]) + (stok >> 3) * 256 + (stok & 7) * 16;
     // output scale of my value position: the fixed point and the 4^k of the spread
-    const float oscale = kFixInv * __uint_as_float((127u - 2u * ((stok >> 2) & 3)) << 23);
+    const float oscale = kFixInv * __uint_as_float((127u - value_scale_log2<VB>(stok)) << 23);
     float qs[G], mr[G], lr[G], zr[G], oacc[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
@@ -727,12 +841,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
 #pragma unroll 1
     for (int c = 0; c < nchunks; ++c) {
       const int P = c & 1;
-      if (!mbar_wait(&sm.qk_done[P], static_cast<uint32_t>((c >> 1) & 1), abort)) bad = true;
+      if (!mbar_wait<kWaitTag>(&sm.qk_done[P], static_cast<uint32_t>((c >> 1) & 1), abort)) bad = true;
       tc_fence_after();
       uint32_t sr[16], sr2[8];
       tmem_ld16(my_lanes + kColS + 32 * P, sr);
       tmem_ld8(my_lanes + kColS + 32 * P + 16, sr2);
-      if (!mbar_wait(&sm.kv_ready[r.i], r.ph, abort)) bad = true;
+      if (!mbar_wait<kWaitTag>(&sm.kv_ready[r.i], r.ph, abort)) bad = true;
       const float4 mt = make_float4(sm.meta[r.i][0][stok], sm.meta[r.i][1][stok], sm.meta[r.i][2][stok],
                                     sm.meta[r.i][3][stok]);  // S_K c1, Z_K, S_V 2^27 (< 0: no token), Z_V
       const bool valid = mt.z >= 0.0f;
@@ -784,7 +898,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
         if (c > fresh_c) {  // PVs of chunks fresh_c .. c-1 ran into O: fold it, restart
           const int pi = r.i == 0 ? 2 : r.i - 1;
           const uint32_t pph = r.i == 0 ? r.ph ^ 1u : r.ph;
-          if (!mbar_wait(&sm.pv_done[pi], pph, abort)) bad = true;
+          if (!mbar_wait<kWaitTag>(&sm.pv_done[pi], pph, abort)) bad = true;
           tc_fence_after();
           flush_o(alpha);
         } else {
@@ -817,7 +931,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
     if (nchunks > 0) {  // the last PV, then the accumulator
       const int pi = r.i == 0 ? 2 : r.i - 1;
       const uint32_t pph = r.i == 0 ? r.ph ^ 1u : r.ph;
-      if (!mbar_wait(&sm.pv_done[pi], pph, abort)) bad = true;
+      if (!mbar_wait<kWaitTag>(&sm.pv_done[pi], pph, abort)) bad = true;
       tc_fence_after();
       float one[G];
 #pragma unroll
@@ -839,7 +953,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
       }
     }
     soft_sync();
-    const int d = value_dim_of_pos(stok);
+    const int d = value_dim_of_pos<VB>(stok);
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       const float z = (sm.red[0][g][1] + sm.red[1][g][1]) + (sm.red[2][g][1] + sm.red[3][g][1]);
@@ -956,12 +1070,24 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(DecodeArgs a) {
   }
 }
 
-template <int G>
+template <int G, int KB, int VB>
 cudaError_t launch_g(const DecodeArgs& a, cudaStream_t stream) {
-  const cudaError_t e = ensure_smem_limit<decode_kernel<G>>(kSmemBytes);
+  constexpr int kBytes = kSmemBytesOf<Fmt<KB, VB>::kSegBytes>;
+  const cudaError_t e = ensure_smem_limit<decode_kernel<G, KB, VB>>(kBytes);
   if (e != cudaSuccess) return e;
   const dim3 grid(a.nsplit, a.num_kv_heads, a.batch);
-  return launch_pdl(decode_kernel<G>, grid, dim3(kThreads), kSmemBytes, stream, a);
+  return launch_pdl(decode_kernel<G, KB, VB>, grid, dim3(kThreads), kBytes, stream, a);
+}
+
+template <int KB, int VB>
+cudaError_t launch_p(const DecodeArgs& a, cudaStream_t stream) {
+  switch (a.num_q_heads / a.num_kv_heads) {
+    case 1: return launch_g<1, KB, VB>(a, stream);
+    case 2: return launch_g<2, KB, VB>(a, stream);
+    case 4: return launch_g<4, KB, VB>(a, stream);
+    case 8: return launch_g<8, KB, VB>(a, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace
@@ -972,8 +1098,9 @@ int decode_ctas_per_sm() {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 1;
   if (cached[dev] > 0) return cached[dev];
   int n = 0;
-  if (ensure_smem_limit<decode_kernel<8>>(kSmemBytes) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<8>, kThreads, kSmemBytes) != cudaSuccess ||
+  constexpr int kBytes = kSmemBytesOf<Fmt<4, 2>::kSegBytes>;
+  if (ensure_smem_limit<decode_kernel<8, 4, 2>>(kBytes) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<8, 4, 2>, kThreads, kBytes) != cudaSuccess ||
       n < 1)
     n = 1;
   cached[dev] = n < 2 ? n : 2;  // two CTAs' tensor memory (2 x 256 columns) fills an SM
@@ -984,13 +1111,11 @@ int decode_max_splits() { return kMaxSplits; }
 int decode_chunk_blocks() { return kChunkBlocks; }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
-  switch (a.num_q_heads / a.num_kv_heads) {
-    case 1: return launch_g<1>(a, stream);
-    case 2: return launch_g<2>(a, stream);
-    case 4: return launch_g<4>(a, stream);
-    case 8: return launch_g<8>(a, stream);
-    default: return cudaErrorInvalidValue;
-  }
+  if (a.k_bits == 4 && a.v_bits == 2) return launch_p<4, 2>(a, stream);
+  if (a.k_bits == 4 && a.v_bits == 4) return launch_p<4, 4>(a, stream);
+  if (a.k_bits == 2 && a.v_bits == 2) return launch_p<2, 2>(a, stream);
+  if (a.k_bits == 8 && a.v_bits == 4) return launch_p<8, 4>(a, stream);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace kvq

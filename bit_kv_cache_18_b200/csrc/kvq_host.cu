@@ -22,7 +22,7 @@ std::mutex g_attr_mutex;
 
 bool supported_desc(const kvq_cache_desc* d) {
   return d->head_dim == kHeadDim && d->group == kHeadDim && d->block_size == kBlockSize &&
-         d->k_bits == kKBits && d->v_bits == kVBits;
+         preset_supported(d->k_bits, d->v_bits);
 }
 
 int check_desc(const kvq_cache_desc* d) {
@@ -183,12 +183,12 @@ int kvq_parse_dtype(const char* s, int32_t* k_bits, int32_t* v_bits, int32_t* gr
   *k_bits = kb;
   *v_bits = vb;
   *group = g;
-  return (kb == kKBits && vb == kVBits && g == kHeadDim) ? KVQ_OK : KVQ_ERR_UNSUPPORTED;
+  return (preset_supported(kb, vb) && g == kHeadDim) ? KVQ_OK : KVQ_ERR_UNSUPPORTED;
 }
 
 size_t kvq_cache_bytes(const kvq_cache_desc* desc) {
   if (check_desc(desc) != KVQ_OK) return 0;
-  return static_cast<size_t>(desc->num_blocks) * desc->num_kv_heads * kSegBytes;
+  return static_cast<size_t>(desc->num_blocks) * desc->num_kv_heads * seg_bytes(desc->k_bits, desc->v_bits);
 }
 
 int kvq_block_table(int32_t num_blocks, int32_t block_size, const int32_t* seq_lens, int32_t batch,
@@ -268,6 +268,8 @@ int kvq_quantize_append(const kvq_cache_desc* desc, const void* k, const void* v
   a.n_tokens = n_tokens;
   a.token_stride = token_stride;
   a.slots = slot_mapping;
+  a.k_bits = desc->k_bits;
+  a.v_bits = desc->v_bits;
   a.status = device_status_ptr();
   if (!a.status) return KVQ_ERR_CUDA;
   return launch_quantize(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
@@ -339,6 +341,8 @@ int decode_impl(const kvq_cache_desc* desc, const void* q, kvq_dtype q_dtype, in
   a.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + plan.ticket_bytes);
   a.blocks_per_split = plan.blocks_per_split;
   a.nsplit = plan.nsplit;
+  a.k_bits = desc->k_bits;
+  a.v_bits = desc->v_bits;
   a.status = device_status_ptr();
   a.k_new = app ? static_cast<const uint8_t*>(app->k) : nullptr;
   a.v_new = app ? static_cast<const uint8_t*>(app->v) : nullptr;

@@ -14,22 +14,33 @@
 
 namespace kvq {
 
-// ---- pool format (k4v2_g128, 16-token blocks) ------------------------------
+// ---- pool formats (presets k<KB>v<VB>_g128, 16-token blocks) ----------------
+// A segment (block, kv head): 16 rows of K codes, 16 rows of V codes (element
+// i of a b-bit row at bit b*i of the row, little-endian), then S_K, Z_K,
+// S_V, Z_V as 16 fp16 each.
 constexpr int kHeadDim = 128;
 constexpr int kBlockSize = 16;
-constexpr int kKBits = 4;
-constexpr int kVBits = 2;
-constexpr int kKRowBytes = kHeadDim * kKBits / 8;  // 64
-constexpr int kVRowBytes = kHeadDim * kVBits / 8;  // 32
-constexpr int kOffK = 0;
-constexpr int kOffV = kOffK + kBlockSize * kKRowBytes;  // 1024
-constexpr int kOffSK = kOffV + kBlockSize * kVRowBytes;  // 1536
-constexpr int kOffZK = kOffSK + 2 * kBlockSize;          // 1568
-constexpr int kOffSV = kOffZK + 2 * kBlockSize;          // 1600
-constexpr int kOffZV = kOffSV + 2 * kBlockSize;          // 1632
-constexpr int kSegBytes = kOffZV + 2 * kBlockSize;       // 1664
-static_assert(kSegBytes == 1664, "segment size");
-static_assert(kSegBytes % 128 == 0, "segments stay 128-byte aligned");
+template <int KB, int VB>
+struct Fmt {
+  static constexpr int kKBits = KB;
+  static constexpr int kVBits = VB;
+  static constexpr int kKRowBytes = kHeadDim * KB / 8;
+  static constexpr int kVRowBytes = kHeadDim * VB / 8;
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kOffK + kBlockSize * kKRowBytes;
+  static constexpr int kOffSK = kOffV + kBlockSize * kVRowBytes;
+  static constexpr int kOffZK = kOffSK + 2 * kBlockSize;
+  static constexpr int kOffSV = kOffZK + 2 * kBlockSize;
+  static constexpr int kOffZV = kOffSV + 2 * kBlockSize;
+  static constexpr int kSegBytes = kOffZV + 2 * kBlockSize;
+  static_assert(kSegBytes % 128 == 0, "segments stay 128-byte aligned");
+};
+static_assert(Fmt<4, 2>::kSegBytes == 1664, "the default preset's segment");
+// The presets built: k4v2 (the pages' default), k4v4, k2v2, k8v4.
+constexpr bool preset_supported(int kb, int vb) {
+  return (kb == 4 && (vb == 2 || vb == 4)) || (kb == 2 && vb == 2) || (kb == 8 && vb == 4);
+}
+constexpr int seg_bytes(int kb, int vb) { return kBlockSize * kHeadDim * (kb + vb) / 8 + 8 * kBlockSize; }
 
 // Split-K partial record in the decode workspace: o~[128], m (log2 domain), l.
 constexpr int kPartialFloats = kHeadDim + 4;
@@ -63,20 +74,31 @@ __device__ __forceinline__ void store_from_f32(void* p, int dtype, int64_t i, fl
 }
 
 // ---- write path, one warp per head vector ------------------------------------
-// Rotate, normalise, quantise and pack one 128-element K (is_v false: 4-bit)
-// or V (2-bit) head vector (bf16 or fp16, 16-byte aligned at src) into row
-// row_in_block of segment seg, lane l holding elements 4l .. 4l+3: the two
-// lowest butterfly stages in registers, the five others by shuffles, the
-// statistics as warp reductions.  The arithmetic is that of the bulk write
-// path (moments of y = sqrt(128) r, fp16 S and Z, codes from the stored S and
-// Z); only the summation order differs.  Each lane then owns whole bytes of
-// the packed row: two bytes of 4-bit key codes or one byte of 2-bit codes.
+// Rotate, normalise, quantise and pack one 128-element K (is_v false: KB
+// bits) or V (VB bits) head vector (bf16 or fp16, 16-byte aligned at src)
+// into row row_in_block of segment seg, lane l holding elements 4l .. 4l+3:
+// the two lowest butterfly stages in registers, the five others by shuffles,
+// the statistics as warp reductions.  The arithmetic is that of the bulk
+// write path (moments of y = sqrt(128) r, fp16 S and Z, codes from the stored
+// S and Z); only the summation order differs.  Each lane then owns whole
+// bytes of the packed row: the 4 b bits of its four codes.
 // Method: "KVarN vs TurboQuant" (dothoosh.com), pipeline list: Hadamard
 // rotation, variance normalisation, asymmetric round-to-nearest.
 // quantize_vector_warp_raw takes the lane's 8 source bytes already loaded.
-template <bool kBF16>
+// Lane's four codes (c[j] = element 4 lane + j) into a packed B-bit row.
+template <int B>
+__device__ __forceinline__ void store_lane_codes(uint8_t* row, const uint32_t (&c)[4], int lane) {
+  if (B == 2)
+    row[lane] = static_cast<uint8_t>(c[0] | c[1] << 2 | c[2] << 4 | c[3] << 6);
+  else if (B == 4)
+    reinterpret_cast<uint16_t*>(row)[lane] = static_cast<uint16_t>(c[0] | c[1] << 4 | c[2] << 8 | c[3] << 12);
+  else
+    reinterpret_cast<uint32_t*>(row)[lane] = c[0] | c[1] << 8 | c[2] << 16 | c[3] << 24;
+}
+template <bool kBF16, int KB, int VB>
 __device__ __forceinline__ void quantize_vector_warp_raw(uint2 raw, uint8_t* seg, int row_in_block, bool is_v,
                                                          int lane) {
+  using F = Fmt<KB, VB>;
   constexpr float kMagicRne = 12582912.0f;  // 1.5 * 2^23: low mantissa bits hold rne of the addend
   float y[4];
   if (kBF16) {
@@ -120,7 +142,7 @@ __device__ __forceinline__ void quantize_vector_warp_raw(uint2 raw, uint8_t* seg
     ymin = fminf(ymin, __shfl_xor_sync(0xffffffffu, ymin, o));
     ymax = fmaxf(ymax, __shfl_xor_sync(0xffffffffu, ymax, o));
   }
-  const float levels = is_v ? static_cast<float>((1 << kVBits) - 1) : static_cast<float>((1 << kKBits) - 1);
+  const float levels = is_v ? static_cast<float>((1 << VB) - 1) : static_cast<float>((1 << KB) - 1);
   constexpr float kInvSqrtD = 0.088388347648318440550f;
   const float mean = sum * (1.0f / kHeadDim);
   const float var = fmaxf(sq * (1.0f / kHeadDim) - mean * mean, 0.0f);
@@ -143,26 +165,26 @@ __device__ __forceinline__ void quantize_vector_warp_raw(uint2 raw, uint8_t* seg
     }
   }
   if (is_v) {
-    seg[kOffV + row_in_block * kVRowBytes + lane] = static_cast<uint8_t>(c[0] | c[1] << 2 | c[2] << 4 | c[3] << 6);
+    store_lane_codes<VB>(seg + F::kOffV + row_in_block * F::kVRowBytes, c, lane);
     if (lane == 0) {
-      reinterpret_cast<__half*>(seg + kOffSV)[row_in_block] = Sh;
-      reinterpret_cast<__half*>(seg + kOffZV)[row_in_block] = Zh;
+      reinterpret_cast<__half*>(seg + F::kOffSV)[row_in_block] = Sh;
+      reinterpret_cast<__half*>(seg + F::kOffZV)[row_in_block] = Zh;
     }
   } else {
-    reinterpret_cast<uint16_t*>(seg + kOffK + row_in_block * kKRowBytes)[lane] =
-        static_cast<uint16_t>(c[0] | c[1] << 4 | c[2] << 8 | c[3] << 12);
+    store_lane_codes<KB>(seg + F::kOffK + row_in_block * F::kKRowBytes, c, lane);
     if (lane == 0) {
-      reinterpret_cast<__half*>(seg + kOffSK)[row_in_block] = Sh;
-      reinterpret_cast<__half*>(seg + kOffZK)[row_in_block] = Zh;
+      reinterpret_cast<__half*>(seg + F::kOffSK)[row_in_block] = Sh;
+      reinterpret_cast<__half*>(seg + F::kOffZK)[row_in_block] = Zh;
     }
   }
 }
 
 // elements 4 lane .. 4 lane + 3 (8 bytes) of the vector at src
-template <bool kBF16>
+template <bool kBF16, int KB, int VB>
 __device__ __forceinline__ void quantize_vector_warp(const uint8_t* src, uint8_t* seg, int row_in_block, bool is_v,
                                                      int lane) {
-  quantize_vector_warp_raw<kBF16>(*reinterpret_cast<const uint2*>(src + 8 * lane), seg, row_in_block, is_v, lane);
+  quantize_vector_warp_raw<kBF16, KB, VB>(*reinterpret_cast<const uint2*>(src + 8 * lane), seg, row_in_block, is_v,
+                                          lane);
 }
 
 // ---- programmatic dependent launch ------------------------------------------
@@ -203,6 +225,7 @@ struct QuantizeArgs {
   int64_t token_stride;
   const int32_t* slots;
   int* status;
+  int32_t k_bits, v_bits;  // preset
 };
 cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream);
 
@@ -231,6 +254,7 @@ struct DecodeArgs {
   const uint8_t* v_new;
   int32_t new_bf16;
   int64_t new_stride_bytes;
+  int32_t k_bits, v_bits;  // preset
 };
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 

@@ -276,7 +276,13 @@ __device__ __forceinline__ void codes_to_words(const float (&y)[kHeadDim], u64 a
       }
       upk_u(add2(t, m2), c[2 * j], c[2 * j + 1]);
     }
-    if (kBits == 4) {
+    if (kBits == 8) {
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {  // word c0/4 + m = elements c0 + 4m .. +3
+        const uint32_t* e = c + 4 * m;
+        words[c0 / 4 + m] = prmt(prmt(e[0], e[1], 0x0040u), prmt(e[2], e[3], 0x0040u), 0x5410u);
+      }
+    } else if (kBits == 4) {
 #pragma unroll
       for (int m = 0; m < 4; ++m) {  // word c0/8 + m = elements c0 + 8m .. +7
         const uint32_t* e = c + 8 * m;
@@ -302,7 +308,7 @@ __device__ __forceinline__ void codes_to_words(const float (&y)[kHeadDim], u64 a
 // packed row, S and Z go to row `row_in_block` of the segment (seg ==
 // nullptr: not stored).  Every thread of the warp runs it: the
 // tensor-memory load is warp-collective.
-template <int kBits>
+template <int kBits, bool kIsV, class F>
 __device__ __forceinline__ void quantize_lane(uint32_t taddr, float x0, uint8_t* seg, int row_in_block) {
   constexpr float kLevels = static_cast<float>((1 << kBits) - 1);
   constexpr float kInvSqrtD = 0.088388347648318440550f;  // 1/sqrt(128)
@@ -363,24 +369,16 @@ __device__ __forceinline__ void quantize_lane(uint32_t taddr, float x0, uint8_t*
       codes_to_words<kBits, false>(y, a2, b2, words);
   }
   if (seg == nullptr) return;
-  if (kBits == 4) {
-    uint4* dst = reinterpret_cast<uint4*>(seg + kOffK + row_in_block * kKRowBytes);
+  uint4* dst = reinterpret_cast<uint4*>(
+      seg + (kIsV ? F::kOffV + row_in_block * F::kVRowBytes : F::kOffK + row_in_block * F::kKRowBytes));
 #pragma unroll
-    for (int m = 0; m < 4; ++m)
-      dst[m] = make_uint4(words[4 * m], words[4 * m + 1], words[4 * m + 2], words[4 * m + 3]);
-    reinterpret_cast<__half*>(seg + kOffSK)[row_in_block] = Sh;
-    reinterpret_cast<__half*>(seg + kOffZK)[row_in_block] = Zh;
-  } else {
-    uint4* dst = reinterpret_cast<uint4*>(seg + kOffV + row_in_block * kVRowBytes);
-#pragma unroll
-    for (int m = 0; m < 2; ++m)
-      dst[m] = make_uint4(words[4 * m], words[4 * m + 1], words[4 * m + 2], words[4 * m + 3]);
-    reinterpret_cast<__half*>(seg + kOffSV)[row_in_block] = Sh;
-    reinterpret_cast<__half*>(seg + kOffZV)[row_in_block] = Zh;
-  }
+  for (int m = 0; m < kBits; ++m)  // (a row is 16 kBits bytes)
+    dst[m] = make_uint4(words[4 * m], words[4 * m + 1], words[4 * m + 2], words[4 * m + 3]);
+  reinterpret_cast<__half*>(seg + (kIsV ? F::kOffSV : F::kOffSK))[row_in_block] = Sh;
+  reinterpret_cast<__half*>(seg + (kIsV ? F::kOffZV : F::kOffZK))[row_in_block] = Zh;
 }
 
-template <bool kBF16>
+template <bool kBF16, int KB, int VB>
 __global__ void __launch_bounds__(kBulkThreads, 2)
     quantize_kernel(uint8_t* __restrict__ pool, int32_t num_blocks, int32_t hkv,
                     const uint8_t* __restrict__ k, const uint8_t* __restrict__ v,
@@ -497,13 +495,13 @@ __global__ void __launch_bounds__(kBulkThreads, 2)
       if (p >= num_blocks)
         record_status(status, KVQ_ERR_OUT_OF_RANGE);
       else
-        seg = pool + (static_cast<int64_t>(p) * hkv + static_cast<int>(n - tok * hkv)) * kSegBytes;
+        seg = pool + (static_cast<int64_t>(p) * hkv + static_cast<int>(n - tok * hkv)) * Fmt<KB, VB>::kSegBytes;
     }
     const float x0 = kBF16 ? bf16lo_to_f32(x[0]) : __half2float(__ushort_as_half(static_cast<uint16_t>(x[0])));
     if (is_v)  // (uniform over the tile)
-      quantize_lane<kVBits>(tlane + kColD, x0, seg, pslot >= 0 ? pslot % kBlockSize : 0);
+      quantize_lane<VB, true, Fmt<KB, VB>>(tlane + kColD, x0, seg, pslot >= 0 ? pslot % kBlockSize : 0);
     else
-      quantize_lane<kKBits>(tlane + kColD, x0, seg, pslot >= 0 ? pslot % kBlockSize : 0);
+      quantize_lane<KB, false, Fmt<KB, VB>>(tlane + kColD, x0, seg, pslot >= 0 ? pslot % kBlockSize : 0);
     tc_fence_before();
     slot ^= 1;
   }
@@ -525,7 +523,7 @@ __global__ void __launch_bounds__(kBulkThreads, 2)
 constexpr int kSmallWarps = 4;
 constexpr int64_t kSmallMaxVecs = 1024;  // at most this many head vectors per tensor
 
-template <bool kBF16>
+template <bool kBF16, int KB, int VB>
 __global__ void __launch_bounds__(kSmallWarps * 32)
     quantize_small_kernel(uint8_t* __restrict__ pool, int32_t num_blocks, int32_t hkv,
                           const uint8_t* __restrict__ k, const uint8_t* __restrict__ v, int32_t n_tokens,
@@ -548,49 +546,49 @@ __global__ void __launch_bounds__(kSmallWarps * 32)
     return;
   }
   const int row_in_block = slot % kBlockSize;
-  uint8_t* seg = pool + (static_cast<int64_t>(p) * hkv + h) * kSegBytes;
+  uint8_t* seg = pool + (static_cast<int64_t>(p) * hkv + h) * Fmt<KB, VB>::kSegBytes;
 
-  quantize_vector_warp<kBF16>((is_v ? v : k) + tok * stride_bytes + static_cast<int64_t>(h) * (kHeadDim * 2), seg,
-                              row_in_block, is_v, lane);
+  quantize_vector_warp<kBF16, KB, VB>((is_v ? v : k) + tok * stride_bytes + static_cast<int64_t>(h) * (kHeadDim * 2),
+                                      seg, row_in_block, is_v, lane);
 }
 
-}  // namespace
-
-cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream) {
-  if (a.n_tokens == 0) return cudaSuccess;
+template <bool kBF16, int KB, int VB>
+cudaError_t launch_quantize_t(const QuantizeArgs& a, cudaStream_t stream) {
   const int64_t n_vec = static_cast<int64_t>(a.n_tokens) * a.num_kv_heads;
   const int64_t stride_bytes = a.token_stride * 2;
+  const uint8_t* k = static_cast<const uint8_t*>(a.k);
+  const uint8_t* v = static_cast<const uint8_t*>(a.v);
   if (n_vec <= kSmallMaxVecs) {
     const unsigned grid = static_cast<unsigned>((2 * n_vec + kSmallWarps - 1) / kSmallWarps);
-    if (a.in_dtype == KVQ_BF16)
-      return launch_pdl(quantize_small_kernel<true>, dim3(grid), dim3(kSmallWarps * 32), 0, stream, a.pool,
-                        a.num_blocks, a.num_kv_heads, static_cast<const uint8_t*>(a.k),
-                        static_cast<const uint8_t*>(a.v), a.n_tokens, stride_bytes, a.slots, a.status);
-    else
-      return launch_pdl(quantize_small_kernel<false>, dim3(grid), dim3(kSmallWarps * 32), 0, stream, a.pool,
-                        a.num_blocks, a.num_kv_heads, static_cast<const uint8_t*>(a.k),
-                        static_cast<const uint8_t*>(a.v), a.n_tokens, stride_bytes, a.slots, a.status);
-    return cudaGetLastError();
+    return launch_pdl(quantize_small_kernel<kBF16, KB, VB>, dim3(grid), dim3(kSmallWarps * 32), 0, stream, a.pool,
+                      a.num_blocks, a.num_kv_heads, k, v, a.n_tokens, stride_bytes, a.slots, a.status);
   }
   const int64_t tiles = 2 * ((n_vec + kTileVecs - 1) / kTileVecs);
   const int smem = kBulkSmemBytes;
   int64_t grid = tiles;
   const int64_t cap = static_cast<int64_t>(device_sm_count()) * 2;  // two CTAs per SM, all resident
   if (grid > cap) grid = cap;
-  if (a.in_dtype == KVQ_BF16) {
-    const cudaError_t e = ensure_smem_limit<quantize_kernel<true>>(smem);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(quantize_kernel<true>, dim3(static_cast<unsigned>(grid)), dim3(kBulkThreads), smem, stream,
-                      a.pool, a.num_blocks, a.num_kv_heads, static_cast<const uint8_t*>(a.k),
-                      static_cast<const uint8_t*>(a.v), a.n_tokens, stride_bytes, a.slots, a.status);
-  } else {
-    const cudaError_t e = ensure_smem_limit<quantize_kernel<false>>(smem);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(quantize_kernel<false>, dim3(static_cast<unsigned>(grid)), dim3(kBulkThreads), smem, stream,
-                      a.pool, a.num_blocks, a.num_kv_heads, static_cast<const uint8_t*>(a.k),
-                      static_cast<const uint8_t*>(a.v), a.n_tokens, stride_bytes, a.slots, a.status);
-  }
-  return cudaGetLastError();
+  const cudaError_t e = ensure_smem_limit<quantize_kernel<kBF16, KB, VB>>(smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(quantize_kernel<kBF16, KB, VB>, dim3(static_cast<unsigned>(grid)), dim3(kBulkThreads), smem,
+                    stream, a.pool, a.num_blocks, a.num_kv_heads, k, v, a.n_tokens, stride_bytes, a.slots, a.status);
+}
+
+template <int KB, int VB>
+cudaError_t launch_quantize_p(const QuantizeArgs& a, cudaStream_t stream) {
+  return a.in_dtype == KVQ_BF16 ? launch_quantize_t<true, KB, VB>(a, stream)
+                                : launch_quantize_t<false, KB, VB>(a, stream);
+}
+
+}  // namespace
+
+cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t stream) {
+  if (a.n_tokens == 0) return cudaSuccess;
+  if (a.k_bits == 4 && a.v_bits == 2) return launch_quantize_p<4, 2>(a, stream);
+  if (a.k_bits == 4 && a.v_bits == 4) return launch_quantize_p<4, 4>(a, stream);
+  if (a.k_bits == 2 && a.v_bits == 2) return launch_quantize_p<2, 2>(a, stream);
+  if (a.k_bits == 8 && a.v_bits == 4) return launch_quantize_p<8, 4>(a, stream);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace kvq

@@ -17,8 +17,9 @@
  *   mu, sigma = mean and population standard deviation of r (sigma = 0 -> 1);
  *   u = (r - mu)/sigma, lo = min u, hi = max u;
  *   S = fp16(sigma (hi - lo)/(2^b - 1)), Z = fp16(mu + sigma lo)   [g128]
- *   c_i = clamp(rne((r_i - Z)/S), 0, 2^b - 1) (all 0 when S == 0), b = 4 for
- *   keys and 2 for values.  Dequantized vector: x^ = R (S c + Z).
+ *   c_i = clamp(rne((r_i - Z)/S), 0, 2^b - 1) (all 0 when S == 0), b = k_bits
+ *   for keys and v_bits for values (4 and 2 by default).  Dequantized
+ *   vector: x^ = R (S c + Z).
  *
  * Read path (decode), for query head j of sequence b, kv head h = j / G,
  * G = Hq/Hkv, tau = softmax_scale (<= 0 means 1/sqrt(128)):
@@ -29,7 +30,8 @@
  *
  * Pool layout (the ABI; the pages leave it open).  A pool is num_blocks
  * physical blocks of block_size (16) token slots for each of num_kv_heads
- * heads.  Segment (p, h) starts at byte (p*num_kv_heads + h) * 1664 and holds
+ * heads.  Segment (p, h) starts at byte (p*num_kv_heads + h) * SEG and holds,
+ * for the default k4v2_g128 (SEG = 1664):
  *   [0,1024)    K codes, 16 rows of 64 B; element i at byte i/2, low nibble
  *               for even i
  *   [1024,1536) V codes, 16 rows of 32 B; element i at byte i/4, bits 2(i%4)
@@ -37,6 +39,10 @@
  *   [1600,1632) S_V[16]  [1632,1664) Z_V[16]          (fp16, little endian)
  * Slot s of the pool is block s/16, row s%16 (vLLM slot mapping).  That is
  * 104 bytes per token per kv head against 512 for an fp16 cache (4.92x).
+ * The other presets (k4v4, k2v2, k8v4, all g128) keep the same order: 16 K
+ * rows of 16*k_bits B, 16 V rows of 16*v_bits B, then S_K, Z_K, S_V, Z_V;
+ * a b-bit element i sits at bits [b*i, b*i+b) of its row, little endian.
+ * SEG = 16*128*(k_bits+v_bits)/8 + 128: 2176, 1152 and 3200 bytes.
  *
  * Conventions.
  *   - The caller owns every buffer.  Device pointers are CUDA device memory
@@ -85,8 +91,8 @@ typedef struct {
   int32_t block_size;   /* token slots per block: 16                      */
   int32_t num_kv_heads; /* Hkv >= 1                                       */
   int32_t head_dim;     /* 128                                            */
-  int32_t k_bits;       /* 4                                              */
-  int32_t v_bits;       /* 2                                              */
+  int32_t k_bits;       /* 4 (or 2, 8: see kvq_parse_dtype)               */
+  int32_t v_bits;       /* 2 (or 4)                                       */
   int32_t group;        /* elements per scale/zero group: 128 (= head_dim) */
   void* pool;           /* device pointer                                 */
 } kvq_cache_desc;
@@ -94,12 +100,14 @@ typedef struct {
 /* Parse a cache dtype string of the form "kvarn_k<kb>v<vb>_g<g>", the vLLM
  * flag named on the KVarN pages ("KVarN vs TurboQuant", flag paragraph).
  * Host only.  Writes the three numbers and returns KVQ_OK for a well-formed
- * string (KVQ_ERR_UNSUPPORTED if it is well formed but not k4v2_g128),
+ * string (KVQ_ERR_UNSUPPORTED if it is well formed but not one of the
+ * presets the kernels cover: k4v2_g128, k4v4_g128, k2v2_g128, k8v4_g128),
  * KVQ_ERR_INVALID otherwise.  Output pointers may not be NULL. */
 int kvq_parse_dtype(const char* s, int32_t* k_bits, int32_t* v_bits, int32_t* group);
 
-/* Bytes of the pool described by desc (num_blocks * num_kv_heads * 1664 for
- * k4v2_g128), or 0 if desc is NULL or unsupported.  Host only. */
+/* Bytes of the pool described by desc (num_blocks * num_kv_heads * SEG, SEG
+ * = 1664 for k4v2_g128, 2176 for k4v4, 1152 for k2v2, 3200 for k8v4), or 0
+ * if desc is NULL or unsupported.  Host only. */
 size_t kvq_cache_bytes(const kvq_cache_desc* desc);
 
 /* Assign physical blocks to sequences, host only (no device work).

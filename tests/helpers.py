@@ -77,9 +77,10 @@ def check_vector(rep: QuantReport, x: np.ndarray, bits: int, gpu_codes, gpu_S: i
 
 
 def check_pool_tokens(rep: QuantReport, gpu_pool: np.ndarray, num_blocks: int, hkv: int, k_rows, v_rows,
-                      in_dtype: int, slots, tokens, heads=None):
-    """Check (token, head) groups: k_rows/v_rows hold [n, Hkv, 128] raw input rows."""
-    g = oracle.geom(num_blocks=num_blocks, num_kv_heads=hkv)
+                      in_dtype: int, slots, tokens, heads=None, preset=(4, 2)):
+    """Check (token, head) groups: k_rows/v_rows hold [n, Hkv, 128] raw input rows;
+    preset = (key bits, value bits) of the pool."""
+    g = oracle.geom(num_blocks=num_blocks, num_kv_heads=hkv, k_bits=preset[0], v_bits=preset[1])
     heads = range(hkv) if heads is None else heads
     for t in tokens:
         s = int(slots[t])
@@ -88,5 +89,5 @@ def check_pool_tokens(rep: QuantReport, gpu_pool: np.ndarray, num_blocks: int, h
         p, o = divmod(s, 16)
         for h in heads:
             kc, Sk, Zk, vc, Sv, Zv = oracle.unpack_token(g, gpu_pool, p, o, h)
-            check_vector(rep, to_f64(k_rows[t, h], in_dtype), 4, kc, Sk, Zk, f"t{t} h{h} K")
-            check_vector(rep, to_f64(v_rows[t, h], in_dtype), 2, vc, Sv, Zv, f"t{t} h{h} V")
+            check_vector(rep, to_f64(k_rows[t, h], in_dtype), preset[0], kc, Sk, Zk, f"t{t} h{h} K")
+            check_vector(rep, to_f64(v_rows[t, h], in_dtype), preset[1], vc, Sv, Zv, f"t{t} h{h} V")

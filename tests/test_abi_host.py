@@ -17,8 +17,14 @@ def test_every_declared_symbol_is_exported(kvq):
 
 def test_parse_dtype(kvq):
     assert kvq.kvq_parse_dtype("kvarn_k4v2_g128") == (0, (4, 2, 128))
-    rc, parsed = kvq.kvq_parse_dtype("kvarn_k4v4_g128")
-    assert rc == kvq.KVQ_ERR_UNSUPPORTED and parsed == (4, 4, 128)
+    # the other presets built (SURVEY: the same kernels at other bit widths)
+    for kb, vb in ((4, 4), (2, 2), (8, 4)):
+        assert kvq.kvq_parse_dtype(f"kvarn_k{kb}v{vb}_g128") == (0, (kb, vb, 128))
+    # well formed but not built: other widths, other groups
+    for s, parsed in (("kvarn_k8v8_g128", (8, 8, 128)), ("kvarn_k4v2_g64", (4, 2, 64)),
+                      ("kvarn_k3v2_g128", (3, 2, 128))):
+        rc, got = kvq.kvq_parse_dtype(s)
+        assert rc == kvq.KVQ_ERR_UNSUPPORTED and got == parsed
     for bad in ("fp8", "kvarn_k4v2_g128x", "kvarn_k4v2", "kvarn_kv2_g128", ""):
         assert kvq.kvq_parse_dtype(bad)[0] == kvq.KVQ_ERR_INVALID
 
@@ -31,6 +37,11 @@ def test_error_strings(kvq):
 
 def test_cache_bytes(kvq):
     assert kvq.kvq_cache_bytes(kvq.make_desc(1024, 8)) == 1024 * 8 * 1664
+    # segment = 16 rows of K and V codes + 4 x 16 fp16 factors
+    for (kb, vb), seg in (((4, 4), 2176), ((2, 2), 1152), ((8, 4), 3200)):
+        assert seg == 16 * 128 * (kb + vb) // 8 + 128
+        assert kvq.kvq_cache_bytes(kvq.make_desc(10, 3, preset=(kb, vb))) == 10 * 3 * seg
+    assert kvq.kvq_cache_bytes(kvq.make_desc(10, 3, preset=(8, 8))) == 0
     d = kvq.make_desc(4, 2)
     d.head_dim = 64
     assert kvq.kvq_cache_bytes(d) == 0

@@ -104,7 +104,7 @@ def test_worked_example_d4(orc):
         assert np.array_equal(rh, np.array(g["rhat"], float))
 
 
-@pytest.mark.parametrize("bits", [4, 2])
+@pytest.mark.parametrize("bits", [4, 2, 8])
 @pytest.mark.parametrize("normalize", [False, True])
 def test_grid_exact_groups_are_recovered(orc, bits, normalize):
     rng = np.random.default_rng(10 + bits)
@@ -124,7 +124,7 @@ def test_grid_exact_groups_are_recovered(orc, bits, normalize):
 
 def test_code_ranges_and_error_bound(orc, syn):
     x16 = syn.kv(5, syn.TID_K, 0, 64, 4, 128, 3, 10.0, 30.0, syn.F16)
-    for bits in (4, 2):
+    for bits in (4, 2, 8):
         top = (1 << bits) - 1
         for t in range(64):
             for h in range(4):
@@ -148,7 +148,7 @@ def test_normalisation_on_off_invariant(orc, syn):
     for t in range(200):
         for h in range(2):
             x = (x16[t, h].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-            for bits in (4, 2):
+            for bits in (4, 2, 8):
                 c1, S1, Z1, r = orc.quantize_vector(x, bits, True)
                 c0, S0, Z0, _ = orc.quantize_vector(x, bits, False)
                 if (S1, Z1) != (S0, Z0):
@@ -216,6 +216,44 @@ def test_segment_size_and_byte_layout(orc):
     assert np.array_equal(back[0], kc) and np.array_equal(back[3], vc)
     assert back[1:3] == (0x1234, 0x5678) and back[4:] == (0x9ABC, 0xDEF0)
     assert orc.pack_token(g, pool, 3, 0, 0, kc, 0, 0, vc, 0, 0) == -5
+
+
+@pytest.mark.parametrize("kb,vb", [(4, 4), (2, 2), (8, 4)])
+def test_segment_layout_of_the_other_presets(orc, kb, vb):
+    """Segment = 16 rows of kb-bit K codes, 16 rows of vb-bit V codes (element
+    i of a b-bit row at bit b*i of the row, little-endian), then S_K, Z_K,
+    S_V, Z_V as 16 fp16 each."""
+    g = orc.geom(num_blocks=2, num_kv_heads=3, k_bits=kb, v_bits=vb)
+    kr, vr = 128 * kb // 8, 128 * vb // 8
+    seg_n = 16 * (kr + vr) + 4 * 32
+    assert orc.segment_bytes(g) == seg_n and orc.pool_bytes(g) == 2 * 3 * seg_n
+    pool = orc.new_pool(g, fill=0xFF)
+    kc = (np.arange(128) * 7) % (1 << kb)
+    vc = (np.arange(128) * 3) % (1 << vb)
+    assert orc.pack_token(g, pool, 1, 9, 2, kc, 0x1111, 0x2222, vc, 0x3333, 0x4444) == 0
+    seg = pool[(1 * 3 + 2) * seg_n:(1 * 3 + 3) * seg_n]
+
+    def packed(codes, b):  # written out from the layout rule, one byte at a time
+        out = []
+        for byte in range(128 * b // 8):
+            val = 0
+            for i in range(128):
+                bit0 = b * i
+                for t in range(b):
+                    if (bit0 + t) // 8 == byte and (codes[i] >> t) & 1:
+                        val |= 1 << ((bit0 + t) % 8)
+            out.append(val)
+        return out
+
+    assert list(seg[9 * kr:10 * kr]) == packed(kc, kb)
+    assert list(seg[16 * kr + 9 * vr:16 * kr + 10 * vr]) == packed(vc, vb)
+    meta = 16 * (kr + vr)
+    for a, val in enumerate((0x1111, 0x2222, 0x3333, 0x4444)):
+        assert list(seg[meta + 32 * a + 18:meta + 32 * a + 20]) == [val & 0xFF, val >> 8]
+    assert np.all(seg[8 * kr:9 * kr] == 0xFF)
+    back = orc.unpack_token(g, pool, 1, 9, 2)
+    assert np.array_equal(back[0], kc) and np.array_equal(back[3], vc)
+    assert back[1:3] == (0x1111, 0x2222) and back[4:] == (0x3333, 0x4444)
 
 
 def test_append_skips_negative_slots_and_rejects_outside(orc, syn):
