@@ -55,7 +55,7 @@ BYTES_PER_TOKEN_HEAD = 104
 # does), with the SHA-256 of the kernel code it was taken on (decode_code_sha256:
 # comments stripped).  Reported as roofline.traffic only while the code still
 # has that hash.
-DECODE_TRAFFIC = {"sha256": "30b4b7d15d5ca436c09b64fe8821ca50bb2f79b135b2f1158532133f9db9e1e2",
+DECODE_TRAFFIC = {"sha256": "93b50dd095d7bec7682b7febc315ba2e622b2c6d982bbd0351024dda468a6b2a",
                   "bytes": 13766400}
 
 

@@ -22,7 +22,7 @@
 //   * softmax warps 4-7 (thread t <-> token t of S, value position t of O):
 //     read a token's row of S, form the base-2 score of each of the G heads
 //       s_g = S_K,t c1 (S0 + S1/254 + S2/254^2) + Z_K,t sum(q~_g),
-//     the probability p = 2^(s_g - m_g) and P'_g = p S_V,t as a 30-bit fixed
+//     the probability p = 2^(s_g - m_g) and P'_g = p S_V,t as a 32-bit fixed
 //     point whose four bytes are four u8 digit columns of the PV operand,
 //     and keep l_g = sum p and zeta_g = sum p Z_V in registers.
 // For the fused decode step the softmax warps of the CTA whose split holds
@@ -44,17 +44,22 @@
 // packed word to bytes is one or two logic operations per four codes, and
 // every product and sum is exact.  The only roundings are the digit
 // expansion of q~ (about 2^-22 of max|q~|) and the fixed point of P'
-// (a step of 2^-27, with P' < 2^3).  The step must be that fine: tokens
+// (a step of 2^-29, with P' < 2^3).  The step must be that fine: tokens
 // whose P' rounds to zero drop their S_V c_V but keep their p Z_V and p, and
 // since codes are never negative that loss is a bias, not noise.
 //
-// Lazy running max.  m_g tracks the largest s_g + E_t, E_t the exponent
-// bound of S_V,t (S_V,t < 2^E_t, floored at -24), and only moves when some
-// token has s_g + E_t > m_g + 2.9: then P' < 2^3 always fits the fixed
-// point.  A move is decided by one vote of the softmax warps per chunk and is
-// rare; the integer accumulator is then folded into fp32 registers with the
-// factor 2^(m_old - m_new) and restarted.  It is also restarted every 128
-// chunks, which keeps every s32 sum below 2^31.
+// Lazy running max.  m_g bounds s_g + E_t, E_t the exponent bound of
+// S_V,t (S_V,t < 2^E_t, floored at -24), loosely: it only moves when some
+// token has s_g + E_t > m_g + 2.9 (so P' < 2^3 always fits the fixed point),
+// and then to the chunk's max of s_g + E_t plus a headroom of 2, which
+// makes later moves rarer at the price of two bits of P' (the fixed point
+// has them to spare).  A move is decided by one vote of the softmax warps
+// per chunk (the scores are formed again from S for it, exactly).  The PVs
+// then switch to the second integer accumulator, and the first is folded
+// into fp32 registers with the factor 2^(m_old - m_new) one chunk later,
+// when the PVs that ran into it are complete, so no warp waits for a PV.
+// The accumulator is also restarted every 128 chunks, which keeps every s32
+// sum below 2^31.
 //
 // Code order.  The byte spreading permutes the 128 positions of a row
 // (keys: position 32j + 8m + 4h + b holds dim 32m + 8j + 2b + h; values:
@@ -80,18 +85,20 @@ constexpr int kMaxSplits = 64;     // the plan never cuts a sequence finer
 constexpr int kNS = 2;             // score buffers in tensor memory
 constexpr int kNV = 3;             // key-code buffers in tensor memory; value / P' / factor buffers in smem
 constexpr int kFlushChunks = 128;  // integer accumulator restarted at least this often
-constexpr float kFix = 134217728.0f;  // P'_int = rne(P' 2^27) < 2^30
-constexpr float kFixInv = 1.0f / 134217728.0f;
+constexpr float kFix = 536870912.0f;  // P'_int = rne(P' 2^29) < 2^32
+constexpr float kFixInv = 1.0f / 536870912.0f;
+constexpr int kFixExp = 29;
 constexpr float kTrigger = 2.9f;    // move the max when s + E > m + kTrigger
 // The running max before any token: far below every score (|s| stays far
 // below 2^20 for fp16 factors), so the first token moves it and
 // 2^(kNoMax - m) = 0, yet finite, so that s - m + m loses only the bits that
 // the lazy max can spare.
 constexpr float kNoMax = -1048576.0f;
+constexpr float kHeadroom = 2.0f;  // a move sets m to the chunk's max of s + E plus this
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColA = 0;    // key codes of chunk c: kColA + 32 (c % 3)
 constexpr uint32_t kColS = 96;   // S of chunk c: kColS + 32 (c % 2)
-constexpr uint32_t kColO = 160;  // O accumulator
+constexpr uint32_t kColO = 160;  // O accumulators: kColO + 32 k, k = 0, 1
 constexpr uint32_t kWaitLimit = 1u << 22;
 constexpr int kBarSoftSync = 1;  // named barrier of the 128 softmax threads
 constexpr int kBarSoftVote = 2;  // named barrier for their vote
@@ -115,13 +122,14 @@ struct __align__(1024) Smem {
   uint8_t vt[kNV][kChunkTokens * kHeadDim];  // 3 x 16 KB
   uint8_t pm[kNV][kChunkTokens * 32];        // 3 x 4 KB
   uint8_t qb[32 * kHeadDim];                 // 4 KB
-  float meta[kNV][4][kChunkTokens];          // per token: S_K c1, Z_K, S_V 2^27 (< 0: no token), Z_V
+  float meta[kNV][4][kChunkTokens];          // per token: S_K c1, Z_K, S_V 2^29 (< 0: no token), Z_V
   union {
     uint8_t stg[kLoadWarps][kNV][2 * kSeg];  // loader warp w: its two segments of chunk c in slot c % 3
     float obuf[8][kHeadDim];                      // o~ (epilogue, after the scan)
   };
   float2 hq[8];                              // per head: sum(q~), max|q~|
   float red[kSoftWarps][8][2];               // cross-warp reductions
+  float palpha[kSoftWarps][8];               // per softmax warp: factor of the pending O buffer
   float hm[8], hl[8], hz[8];
   uint64_t kv_ready[kNV];  // loaders -> MMA warp, softmax: codes and factors of chunk c written
   uint64_t qk_done[kNS];   // QK(c) complete -> softmax: S of chunk c ready (and PV(c-3) complete)
@@ -131,7 +139,7 @@ struct __align__(1024) Smem {
   uint64_t full[kLoadWarps][kNV];  // TMA -> loader warp w: segments of chunk c in slot c % 3
   uint64_t fin;            // every MMA issued is complete
   uint32_t tmem_base;
-  int fresh[kNV];          // the PV of chunk c starts the accumulator afresh
+  int fresh[kNV];          // PV of chunk c: bit 0 starts the accumulator afresh, bit 1 its O buffer
   int is_last;
   int abort;              // a wait ran out: every other wait gives up at once
 };
@@ -685,7 +693,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
                 : smem_u32(sm.vt[0]) + 4 * warp * 1024 + (lane >> 2) * 16 + 2 * (lane & 3) * 128;
     const int mrow0 = 4 * (lane & 3);    // my factor rows mrow0 .. mrow0+3 of segment mseg
     const int mkind = (lane >> 2) & 3;  // S_K, Z_K, S_V, Z_V
-    const float mscale = mkind == 0 ? c1 : (mkind == 2 ? kFix : 1.0f);
+    const float mscale = mkind == 0 ? c1 : (mkind == 2 ? kFix : 1.0f);  // S_V -> S_V 2^29
     const float mnone = mkind == 2 ? -1.0f : 0.0f;  // the factor of an absent token
     const uint32_t my_meta = smem_u32(&sm.meta[0][mkind][32 * warp + 16 * mseg + mrow0]);
 #pragma unroll
@@ -789,11 +797,13 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
         if (!mbar_wait<kWaitTag>(&sm.p_ready[rp.i], rp.ph, abort)) bad = true;
         tc_fence_after();
         if (lane == 0) {
-          const bool fresh = sm.fresh[rp.i] != 0;
+          const int fr = sm.fresh[rp.i];
+          const bool fresh = (fr & 1) != 0;
+          const uint32_t ocol = tbase + kColO + 16 * (fr & 2);
           const uint32_t va = vt0 + rp.i * (kChunkTokens * kHeadDim), pa = pm0 + rp.i * (kChunkTokens * 32);
 #pragma unroll
           for (int s = 0; s < 4; ++s)
-            mma_pv(tbase + kColO, sdesc(va + 4096 * s, 1024, 128), sdesc(pa + 1024 * s, 256, 128), !fresh || s > 0);
+            mma_pv(ocol, sdesc(va + 4096 * s, 1024, 128), sdesc(pa + 1024 * s, 256, 128), !fresh || s > 0);
           mma_commit(&sm.pv_done[rp.i]);
         }
         __syncwarp();
@@ -809,9 +819,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
     const int stok = tid - 32 * kLoadWarps;
     const uint32_t my_lanes = tbase + (static_cast<uint32_t>(sw * 32) << 16);
     const uint32_t my_pm = smem_u32(sm.pm[0]) + (stok >> 3) * 256 + (stok & 7) * 16;
-    // output scale of my value position: the fixed point and the 4^k of the spread
-    const float oscale = kFixInv * __uint_as_float((127u - value_scale_log2<VB>(stok)) << 23);
-    float qs[G], mr[G], lr[G], zr[G], oacc[G];
+    float qs[G], mr[G], lr[G], zr[G], oacc[G];  // oacc: in units of the output scale below
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       qs[g] = sm.hq[g].x;
@@ -819,12 +827,19 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
       lr[g] = zr[g] = oacc[g] = 0.0f;
     }
     int fresh_c = 0;  // the chunk whose PV started the integer accumulator
+    int ob = 0;       // the O buffer the PVs of chunks fresh_c .. run into
+    // A max move switches the PVs to the other O buffer and leaves the old
+    // one (chunks up to c-1, in units of the old max) pending with the factor
+    // palpha: it is folded at the next chunk, when QK(c+1) is done and so are
+    // the PVs issued before it; nothing waits for a PV at the move.
+    bool pend = false;  // (its per-head factor is in sm.palpha[sw], one copy per warp)
 
-    // fold the integer accumulator (my lane = value position stok) into oacc
-    auto flush_o = [&](const float (&alpha)[G]) {
+    // fold O buffer k (my lane = value position stok) into oacc, with the
+    // pending factor of each head (scaled) or 1
+    auto fold_o = [&](int k, bool scaled) {
       uint32_t r[16], r2[16];
-      tmem_ld16(my_lanes + kColO, r);
-      tmem_ld16(my_lanes + kColO + 16, r2);
+      tmem_ld16(my_lanes + kColO + 32 * k, r);
+      tmem_ld16(my_lanes + kColO + 32 * k + 16, r2);
       tmem_wait_ld();
 #pragma unroll
       for (int g = 0; g < G; ++g) {
@@ -833,7 +848,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
                              fmaf(static_cast<float>(static_cast<int>(q[2])), 65536.0f,
                                   fmaf(static_cast<float>(static_cast<int>(q[1])), 256.0f,
                                        static_cast<float>(static_cast<int>(q[0])))));
-        oacc[g] = alpha[g] * fmaf(v, oscale, oacc[g]);
+        oacc[g] = scaled ? fmaf(v, sm.palpha[sw][g], oacc[g]) : oacc[g] + v;
       }
     };
 
@@ -843,15 +858,19 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
       const int P = c & 1;
       if (!mbar_wait<kWaitTag>(&sm.qk_done[P], static_cast<uint32_t>((c >> 1) & 1), abort)) bad = true;
       tc_fence_after();
+      if (pend) {  // the PVs into the pending buffer (up to chunk c-2) are done
+        fold_o(ob ^ 1, true);
+        pend = false;
+      }
       uint32_t sr[16], sr2[8];
       tmem_ld16(my_lanes + kColS + 32 * P, sr);
       tmem_ld8(my_lanes + kColS + 32 * P + 16, sr2);
       if (!mbar_wait<kWaitTag>(&sm.kv_ready[r.i], r.ph, abort)) bad = true;
       const float4 mt = make_float4(sm.meta[r.i][0][stok], sm.meta[r.i][1][stok], sm.meta[r.i][2][stok],
-                                    sm.meta[r.i][3][stok]);  // S_K c1, Z_K, S_V 2^27 (< 0: no token), Z_V
+                                    sm.meta[r.i][3][stok]);  // S_K c1, Z_K, S_V 2^29 (< 0: no token), Z_V
       const bool valid = mt.z >= 0.0f;
-      // E with S_V < 2^E, from the exponent of S_V 2^27; floored at -24
-      const int ex = static_cast<int>((__float_as_uint(mt.z) >> 23) & 0xFFu) - 153;
+      // E with S_V < 2^E, from the exponent of S_V 2^29; floored at -24
+      const int ex = static_cast<int>((__float_as_uint(mt.z) >> 23) & 0xFFu) - (126 + kFixExp);
       const float e = static_cast<float>(max(ex, -24));
       tmem_wait_ld();
       float dg[G];
@@ -866,9 +885,10 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
       const bool flag = valid && (dmax + e > kTrigger);
       const bool any = soft_vote_any(flag) || c - fresh_c >= kFlushChunks;
       if (any) {
-        // rare: move the running max of the heads to the chunk's max of s + E;
-        // the scores are formed again from S (still in tensor memory: it is
-        // released below), exactly, without the running max
+        // rare: move the running max of each head to the chunk's max of
+        // s + E plus the headroom; the scores are formed again from S (still
+        // in tensor memory: it is released below), exactly, without the
+        // running max
         tmem_ld16(my_lanes + kColS + 32 * P, sr);
         tmem_ld8(my_lanes + kColS + 32 * P + 16, sr2);
         tmem_wait_ld();
@@ -888,28 +908,29 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
 #pragma unroll
         for (int g = 0; g < G; ++g) {
           const float M = fmaxf(fmaxf(sm.red[0][g][0], sm.red[1][g][0]), fmaxf(sm.red[2][g][0], sm.red[3][g][0]));
-          const float mn = fmaxf(mr[g], M);
+          const float mn = fmaxf(mr[g], M + kHeadroom);
           alpha[g] = ex2(mr[g] - mn);
           lr[g] *= alpha[g];
           zr[g] *= alpha[g];
           dg[g] = sg[g] - mn;
           mr[g] = mn;
         }
-        if (c > fresh_c) {  // PVs of chunks fresh_c .. c-1 ran into O: fold it, restart
-          const int pi = r.i == 0 ? 2 : r.i - 1;
-          const uint32_t pph = r.i == 0 ? r.ph ^ 1u : r.ph;
-          if (!mbar_wait<kWaitTag>(&sm.pv_done[pi], pph, abort)) bad = true;
-          tc_fence_after();
-          flush_o(alpha);
-        } else {
 #pragma unroll
-          for (int g = 0; g < G; ++g) oacc[g] *= alpha[g];
+        for (int g = 0; g < G; ++g) oacc[g] *= alpha[g];
+        if (c > fresh_c) {  // PVs of chunks fresh_c .. c-1 ran into buffer ob: pending
+          if (lane == 0) {
+#pragma unroll
+            for (int g = 0; g < G; ++g) sm.palpha[sw][g] = alpha[g];
+          }
+          __syncwarp();
+          pend = true;
+          ob ^= 1;
         }
         fresh_c = c;
         // the reductions above read sm.red: none writes it again before the next vote
       }
       tc_fence_before();
-      mbar_arrive(&sm.s_free[P]);  // S of chunk c is read
+      mbar_arrive(&sm.s_free[P]);
       // P' of chunk c -> pm[r.i] (free: PV(c-3) was issued before QK(c), which is done)
       uint32_t pw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
 #pragma unroll
@@ -917,12 +938,12 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
         const float p = valid ? ex2(dg[g]) : 0.0f;
         lr[g] += p;
         zr[g] = fmaf(p, mt.w, zr[g]);
-        pw[g] = __float2uint_rn(p * mt.z);  // rne(P' 2^27) < 2^30
+        pw[g] = __float2uint_rn(p * mt.z);  // rne(P' 2^29) < 2^32
       }
       const uint32_t pa = my_pm + r.i * (kChunkTokens * 32);
       sts128(pa, pw[0], pw[1], pw[2], pw[3]);
       sts128(pa + 128, pw[4], pw[5], pw[6], pw[7]);
-      if (stok == 0) sm.fresh[r.i] = fresh_c == c;
+      if (stok == 0) sm.fresh[r.i] = (fresh_c == c ? 1 : 0) | (ob << 1);
       async_proxy_fence();
       tc_fence_before();
       mbar_arrive(&sm.p_ready[r.i]);
@@ -933,10 +954,8 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
       const uint32_t pph = r.i == 0 ? r.ph ^ 1u : r.ph;
       if (!mbar_wait<kWaitTag>(&sm.pv_done[pi], pph, abort)) bad = true;
       tc_fence_after();
-      float one[G];
-#pragma unroll
-      for (int g = 0; g < G; ++g) one[g] = 1.0f;
-      flush_o(one);
+      if (pend) fold_o(ob ^ 1, true);
+      fold_o(ob, false);
     }
     // l and zeta over the 128 tokens' threads; o~ in dim order
 #pragma unroll
@@ -954,10 +973,12 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
     }
     soft_sync();
     const int d = value_dim_of_pos<VB>(stok);
+    // output scale of my value position: the fixed point and the factor of the spread
+    const float oscale = kFixInv * __uint_as_float((127u - value_scale_log2<VB>(stok)) << 23);
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       const float z = (sm.red[0][g][1] + sm.red[1][g][1]) + (sm.red[2][g][1] + sm.red[3][g][1]);
-      sm.obuf[g][d] = oacc[g] + z;
+      sm.obuf[g][d] = fmaf(oacc[g], oscale, z);
       if (stok == g) {
         sm.hl[g] = (sm.red[0][g][0] + sm.red[1][g][0]) + (sm.red[2][g][0] + sm.red[3][g][0]);
         sm.hm[g] = mr[g];
