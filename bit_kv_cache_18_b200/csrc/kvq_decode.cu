@@ -25,8 +25,9 @@
 //     the probability p = 2^(s_g - m_g) and P'_g = p S_V,t as a 32-bit fixed
 //     point whose four bytes are four u8 digit columns of the PV operand,
 //     and keep l_g = sum p and zeta_g = sum p Z_V in registers.
-// For the fused decode step the softmax warps of the CTA whose split holds
-// position L-1 first quantize the new token's K and V into that position.
+// For the fused decode step two softmax warps of the CTA whose split holds
+// position L-1 quantize the new token's K and V into that position while
+// the first chunks are in flight; the loaders copy that block after them.
 // Before the scan the softmax warps rotate the G query heads once (warp
 // FWHT, softmax scale times log2(e) folded in) and write q~ as three signed
 // 8-bit digits, q~/c1 = Q0 + Q1/254 + Q2/254^2 with c1 = max|q~|/127.  After
@@ -87,7 +88,6 @@ constexpr int kNV = 3;             // key-code buffers in tensor memory; value /
 constexpr int kFlushChunks = 128;  // integer accumulator restarted at least this often
 constexpr float kFix = 536870912.0f;  // P'_int = rne(P' 2^29) < 2^32
 constexpr float kFixInv = 1.0f / 536870912.0f;
-constexpr int kFixExp = 29;
 constexpr float kTrigger = 2.9f;    // move the max when s + E > m + kTrigger
 // The running max before any token: far below every score (|s| stays far
 // below 2^20 for fp16 factors), so the first token moves it and
@@ -122,7 +122,7 @@ struct __align__(1024) Smem {
   uint8_t vt[kNV][kChunkTokens * kHeadDim];  // 3 x 16 KB
   uint8_t pm[kNV][kChunkTokens * 32];        // 3 x 4 KB
   uint8_t qb[32 * kHeadDim];                 // 4 KB
-  float meta[kNV][4][kChunkTokens];          // per token: S_K c1, Z_K, S_V 2^29 (< 0: no token), Z_V
+  uint16_t meta[kNV][4][kChunkTokens];       // per token, fp16 bits: S_K, Z_K, S_V (-1: segment absent), Z_V
   union {
     uint8_t stg[kLoadWarps][kNV][2 * kSeg];  // loader warp w: its two segments of chunk c in slot c % 3
     float obuf[8][kHeadDim];                      // o~ (epilogue, after the scan)
@@ -130,7 +130,8 @@ struct __align__(1024) Smem {
   float2 hq[8];                              // per head: sum(q~), max|q~|
   float red[kSoftWarps][8][2];               // cross-warp reductions
   float palpha[kSoftWarps][8];               // per softmax warp: factor of the pending O buffer
-  float hm[8], hl[8], hz[8];
+  float hm[8], hl[8];
+  float c1;                                  // max|q~| / 127: the unit of the query digits
   uint64_t kv_ready[kNV];  // loaders -> MMA warp, softmax: codes and factors of chunk c written
   uint64_t qk_done[kNS];   // QK(c) complete -> softmax: S of chunk c ready (and PV(c-3) complete)
   uint64_t s_free[kNS];    // softmax -> MMA warp: S of chunk c read
@@ -138,6 +139,7 @@ struct __align__(1024) Smem {
   uint64_t pv_done[kNV];   // PV(c) complete -> loaders, softmax (and QK(c+1) complete)
   uint64_t full[kLoadWarps][kNV];  // TMA -> loader warp w: segments of chunk c in slot c % 3
   uint64_t fin;            // every MMA issued is complete
+  uint64_t app_done;       // fused step: the new token's row is written (softmax warps 4, 5 -> loaders)
   uint32_t tmem_base;
   int fresh[kNV];          // PV of chunk c: bit 0 starts the accumulator afresh, bit 1 its O buffer
   int is_last;
@@ -289,6 +291,14 @@ __device__ __forceinline__ uint2 lds64(uint32_t addr) {
   uint2 r;
   asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(addr));
   return r;
+}
+__device__ __forceinline__ float lds_f32(uint32_t addr) {  // not hoisted out of loops
+  float r;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(r) : "r"(addr));
+  return r;
+}
+__device__ __forceinline__ void sts64(uint32_t addr, uint32_t a, uint32_t b) {
+  asm volatile("st.shared.v2.b32 [%0], {%1,%2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
 }
 __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
@@ -480,6 +490,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
         mbar_init(&sm.s_free[i], 32 * kSoftWarps);
       }
       mbar_init(&sm.fin, 1);
+      mbar_init(&sm.app_done, 64);
       sm.abort = 0;
       asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -572,7 +583,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
   int32_t bq[6];        // loaders: block ids of chunks c+3 .. c+8 at the start of iteration c
   uint32_t okq[kNV] = {0u, 0u, 0u};  // loaders: segment flags of chunks c .. c+2
   // the chunk holding the block that the fused append writes is copied only
-  // after the set-up barrier (-1: none)
+  // after the append (app_done; -1: none)
   int c_defer = -1;
   if (a.k_new != nullptr && L > 0) {
     const int bn = (L - 1) / kBlockSize;
@@ -604,26 +615,6 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
   } else if (is_soft) {
     const int sw = warp - kLoadWarps;
     const int stok = tid - 32 * kLoadWarps;
-    // fused one-token append: the split holding position L-1 first writes the
-    // new token's K (warp 4) and V (warp 5) of kv head h into that position,
-    // before any loader reads the block (the proxy fence and the set-up
-    // barrier below order the writes before the bulk copies)
-    if (a.k_new != nullptr && sw < 2 && L > 0) {
-      const int blk_new = (L - 1) / kBlockSize;
-      if (blk_new >= blk0 && blk_new < blk1) {
-        const int32_t p = bt_row[blk_new];
-        if (p >= 0 && p < a.num_blocks) {
-          uint8_t* seg = const_cast<uint8_t*>(pool_h) + static_cast<int64_t>(p) * pstride;
-          if (a.new_bf16)
-            quantize_vector_warp_raw<true, KB, VB>(new_raw, seg, (L - 1) % kBlockSize, sw == 1, lane);
-          else
-            quantize_vector_warp_raw<false, KB, VB>(new_raw, seg, (L - 1) % kBlockSize, sw == 1, lane);
-          asm volatile("fence.proxy.async.global;" ::: "memory");
-        } else if (lane == 0) {
-          record_status(a.status, KVQ_ERR_OUT_OF_RANGE);
-        }
-      }
-    }
     // rotate the G query heads, then write their digits with one c1 for all
     // heads
     reinterpret_cast<uint4*>(sm.qb)[stok] = make_uint4(0, 0, 0, 0);
@@ -648,6 +639,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
 #pragma unroll
     for (int g = 0; g < G; ++g) mx = fmaxf(mx, sm.hq[g].y);
     const float inv = mx > 0.0f ? 127.0f / mx : 0.0f;
+    if (stok == 0) sm.c1 = mx * (1.0f / 127.0f);
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       const int g = sw + 4 * i;
@@ -676,10 +668,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = sm.tmem_base;
-  float c1 = 0.0f;
-#pragma unroll
-  for (int g = 0; g < G; ++g) c1 = fmaxf(c1, sm.hq[g].y);
-  c1 *= 1.0f / 127.0f;
+  const float c1 = sm.c1;
 
   // ---- 1. the paged scan ------------------------------------------------------
   if (is_loader) {
@@ -693,12 +682,16 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
                 : smem_u32(sm.vt[0]) + 4 * warp * 1024 + (lane >> 2) * 16 + 2 * (lane & 3) * 128;
     const int mrow0 = 4 * (lane & 3);    // my factor rows mrow0 .. mrow0+3 of segment mseg
     const int mkind = (lane >> 2) & 3;  // S_K, Z_K, S_V, Z_V
-    const float mscale = mkind == 0 ? c1 : (mkind == 2 ? kFix : 1.0f);  // S_V -> S_V 2^29
-    const float mnone = mkind == 2 ? -1.0f : 0.0f;  // the factor of an absent token
+    const uint32_t mnone = mkind == 2 ? 0xBC00BC00u : 0u;  // the factors of an absent segment (S_V = -1)
+    // the block holding position L-1, for the lanes holding S_V (-2: none)
+    const int blk_last = mkind == 2 ? (L - 1) / kBlockSize : -2;
     const uint32_t my_meta = smem_u32(&sm.meta[0][mkind][32 * warp + 16 * mseg + mrow0]);
 #pragma unroll
     for (int i = 0; i < kNV; ++i)  // the deferred chunk, if it is one of the first three
-      if (i == c_defer) okq[i] = issue(i, bfirst[i], i);
+      if (i == c_defer) {
+        if (!mbar_wait<kWaitTag>(&sm.app_done, 0u, abort)) bad = true;
+        okq[i] = issue(i, bfirst[i], i);
+      }
     Ring3 r{0, 0u};  // chunk c: staging slot, key-code, value and factor buffers r.i
 #pragma unroll 1
     for (int c = 0; c < nchunks; ++c) {
@@ -720,6 +713,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
       __syncwarp();
       okq[0] = okq[1];
       okq[1] = okq[2];
+      if (c + kNV == c_defer && !mbar_wait<kWaitTag>(&sm.app_done, 0u, abort)) bad = true;
       okq[2] = c + kNV < nchunks ? issue(c + kNV, bq[0], r.i) : 0u;
       prefetch_seg(bq[3]);
 #pragma unroll
@@ -755,14 +749,20 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
           }
         }
       }
-      {  // factors of my four rows; absent tokens get 0 (S_V: -1)
+      {  // factors of my four rows, as stored; S_V = -1 marks an absent token
+         // (a segment outside the split or the pool, a row past the end of
+         // the sequence: only in the block holding position L-1)
+        const bool seg_ok = ((ok >> mseg) & 1u) != 0;
+        uint32_t m0 = seg_ok ? mr2.x : mnone, m1 = seg_ok ? mr2.y : mnone;
         const int blk = blk0 + kChunkBlocks * c + 2 * warp + mseg;
-        const int nv = ((ok >> mseg) & 1u) ? min(4, max(0, L - blk * kBlockSize - mrow0)) : 0;
-        sts128(my_meta + r.i * (4 * kChunkTokens * 4),
-               __float_as_uint(nv > 0 ? h2f(mr2.x) * mscale : mnone),
-               __float_as_uint(nv > 1 ? h2f(mr2.x >> 16) * mscale : mnone),
-               __float_as_uint(nv > 2 ? h2f(mr2.y) * mscale : mnone),
-               __float_as_uint(nv > 3 ? h2f(mr2.y >> 16) * mscale : mnone));
+        if (blk == blk_last) {
+          const int nv = L - blk * kBlockSize - mrow0;  // my rows inside the sequence (may be <= 0 or > 4)
+          if (nv < 1) m0 = (m0 & 0xFFFF0000u) | 0xBC00u;
+          if (nv < 2) m0 = (m0 & 0x0000FFFFu) | 0xBC000000u;
+          if (nv < 3) m1 = (m1 & 0xFFFF0000u) | 0xBC00u;
+          if (nv < 4) m1 = (m1 & 0x0000FFFFu) | 0xBC000000u;
+        }
+        sts64(my_meta + r.i * (4 * kChunkTokens * 2), m0, m1);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -817,6 +817,25 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
     // softmax warps: thread stok <-> token stok of S, value position stok of O
     const int sw = warp - kLoadWarps;
     const int stok = tid - 32 * kLoadWarps;
+    // fused one-token append: in the split holding position L-1, warps 4 and
+    // 5 write the new token's K and V of kv head h into that position while
+    // the first chunks are in flight (they would wait for the first QK
+    // anyway); the loaders copy the chunk holding it only after app_done
+    // (the proxy fence orders the writes before the bulk copy)
+    if (c_defer >= 0 && sw < 2) {
+      const int32_t p = bt_row[(L - 1) / kBlockSize];
+      if (p >= 0 && p < a.num_blocks) {
+        uint8_t* seg = const_cast<uint8_t*>(pool_h) + static_cast<int64_t>(p) * pstride;
+        if (a.new_bf16)
+          quantize_vector_warp_raw<true, KB, VB>(new_raw, seg, (L - 1) % kBlockSize, sw == 1, lane);
+        else
+          quantize_vector_warp_raw<false, KB, VB>(new_raw, seg, (L - 1) % kBlockSize, sw == 1, lane);
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+      } else if (lane == 0 && sw == 0) {
+        record_status(a.status, KVQ_ERR_OUT_OF_RANGE);
+      }
+      mbar_arrive(&sm.app_done);
+    }
     const uint32_t my_lanes = tbase + (static_cast<uint32_t>(sw * 32) << 16);
     const uint32_t my_pm = smem_u32(sm.pm[0]) + (stok >> 3) * 256 + (stok & 7) * 16;
     float qs[G], mr[G], lr[G], zr[G], oacc[G];  // oacc: in units of the output scale below
@@ -866,12 +885,16 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
       tmem_ld16(my_lanes + kColS + 32 * P, sr);
       tmem_ld8(my_lanes + kColS + 32 * P + 16, sr2);
       if (!mbar_wait<kWaitTag>(&sm.kv_ready[r.i], r.ph, abort)) bad = true;
-      const float4 mt = make_float4(sm.meta[r.i][0][stok], sm.meta[r.i][1][stok], sm.meta[r.i][2][stok],
-                                    sm.meta[r.i][3][stok]);  // S_K c1, Z_K, S_V 2^29 (< 0: no token), Z_V
-      const bool valid = mt.z >= 0.0f;
-      // E with S_V < 2^E, from the exponent of S_V 2^29; floored at -24
-      const int ex = static_cast<int>((__float_as_uint(mt.z) >> 23) & 0xFFu) - (126 + kFixExp);
-      const float e = static_cast<float>(max(ex, -24));
+      const uint32_t hsv = sm.meta[r.i][2][stok];
+      const bool valid = (hsv & 0x8000u) == 0;  // a token (not marked absent by the loaders)
+      // S_K c1, Z_K, S_V 2^29, Z_V (0 for an absent token)
+      // (c1 is read again each chunk: keeping it in a register made the
+      // kernel spill)
+      const float4 mt = make_float4(h2f(sm.meta[r.i][0][stok]) * lds_f32(smem_u32(&sm.c1)), h2f(sm.meta[r.i][1][stok]),
+                                    h2f(hsv) * kFix,
+                                    valid ? h2f(sm.meta[r.i][3][stok]) : 0.0f);
+      // E with S_V < 2^E, from the fp16 exponent of S_V (-14 for subnormals and 0)
+      const float e = static_cast<float>(static_cast<int>((hsv >> 10) & 31u) - 14);
       tmem_wait_ld();
       float dg[G];
       float dmax = -CUDART_INF_F;
