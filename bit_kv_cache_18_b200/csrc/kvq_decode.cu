@@ -25,9 +25,10 @@
 //     the probability p = 2^(s_g - m_g) and P'_g = p S_V,t as a 32-bit fixed
 //     point whose four bytes are four u8 digit columns of the PV operand,
 //     and keep l_g = sum p and zeta_g = sum p Z_V in registers.
-// For the fused decode step two softmax warps of the CTA whose split holds
-// position L-1 quantize the new token's K and V into that position while
-// the first chunks are in flight; the loaders copy that block after them.
+// For the fused decode step the MMA warp of the CTA whose split holds
+// position L-1 quantizes the new token's K and V into that position during
+// the set-up, while the query is rotated; the loaders copy that block after
+// the set-up barrier.
 // Before the scan the softmax warps rotate the G query heads once (warp
 // FWHT, softmax scale times log2(e) folded in) and write q~ as three signed
 // 8-bit digits, q~/c1 = Q0 + Q1/254 + Q2/254^2 with c1 = max|q~|/127.  After
@@ -139,7 +140,6 @@ struct __align__(1024) Smem {
   uint64_t pv_done[kNV];   // PV(c) complete -> loaders, softmax (and QK(c+1) complete)
   uint64_t full[kLoadWarps][kNV];  // TMA -> loader warp w: segments of chunk c in slot c % 3
   uint64_t fin;            // every MMA issued is complete
-  uint64_t app_done;       // fused step: the new token's row is written (softmax warps 4, 5 -> loaders)
   uint32_t tmem_base;
   int fresh[kNV];          // PV of chunk c: bit 0 starts the accumulator afresh, bit 1 its O buffer
   int is_last;
@@ -490,18 +490,17 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
         mbar_init(&sm.s_free[i], 32 * kSoftWarps);
       }
       mbar_init(&sm.fin, 1);
-      mbar_init(&sm.app_done, 64);
       sm.abort = 0;
       asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
   }
   pdl_wait();
 
-  // The softmax warps' loads that need no sequence length go out first:
-  // warp sw's query heads sw and sw + 4 and, for warps 4 and 5 of a fused
-  // step, their lanes' 8 bytes of the new token's K or V row.
+  // The loads that need no sequence length go out first: softmax warp sw's
+  // query heads sw and sw + 4 and, in a fused step, the MMA warp's lanes' 8
+  // bytes of the new token's K and V rows.
   float x[2][4];
-  uint2 new_raw = make_uint2(0u, 0u);
+  uint2 new_k = make_uint2(0u, 0u), new_v = make_uint2(0u, 0u);
   if (is_soft) {
     const int sw = warp - kLoadWarps;
 #pragma unroll
@@ -513,9 +512,10 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
         for (int k = 0; k < 4; ++k) x[i][k] = load_as_f32(a.q, a.q_dtype, q0 + lane + 32 * k);
       }
     }
-    if (a.k_new != nullptr && sw < 2)
-      new_raw = *reinterpret_cast<const uint2*>((sw ? a.v_new : a.k_new) + static_cast<int64_t>(b) * a.new_stride_bytes +
-                                                static_cast<int64_t>(h) * (kHeadDim * 2) + 8 * lane);
+  } else if (warp == kMmaWarp && a.k_new != nullptr) {
+    const int64_t off = static_cast<int64_t>(b) * a.new_stride_bytes + static_cast<int64_t>(h) * (kHeadDim * 2) + 8 * lane;
+    new_k = *reinterpret_cast<const uint2*>(a.k_new + off);
+    new_v = *reinterpret_cast<const uint2*>(a.v_new + off);
   }
 
   // ---- the split: blocks [blk0, blk1) of sequence b, in chunks of 8 -------
@@ -583,12 +583,13 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
   int32_t bq[6];        // loaders: block ids of chunks c+3 .. c+8 at the start of iteration c
   uint32_t okq[kNV] = {0u, 0u, 0u};  // loaders: segment flags of chunks c .. c+2
   // the chunk holding the block that the fused append writes is copied only
-  // after the append (app_done; -1: none)
+  // after the set-up barrier (-1: none)
   int c_defer = -1;
   if (a.k_new != nullptr && L > 0) {
     const int bn = (L - 1) / kBlockSize;
     if (bn >= blk0 && bn < blk1) c_defer = (bn - blk0) / kChunkBlocks;
   }
+
   if (is_loader) {
 #pragma unroll
     for (int i = 0; i < kNV; ++i) bfirst[i] = blk0 + kChunkBlocks * i + 2 * warp + (lane & 1) < blk1 ? braw[i] : -1;
@@ -663,6 +664,27 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
       }
     }
     async_proxy_fence();
+  } else if (c_defer >= 0) {
+    // fused one-token append: the MMA warp (idle until the first chunk
+    // lands) of the split holding position L-1 writes the new token's K and
+    // V of kv head h into that position, in parallel with the query
+    // rotation; the proxy fence and the set-up barrier order the writes
+    // before the loaders' bulk copy of that block
+    const int32_t p = __ldg(bt_row + (L - 1) / kBlockSize);
+    if (p >= 0 && p < a.num_blocks) {
+      uint8_t* seg = const_cast<uint8_t*>(pool_h) + static_cast<int64_t>(p) * pstride;
+      const int row = (L - 1) % kBlockSize;
+      if (a.new_bf16) {
+        quantize_vector_warp_raw<true, KB, VB>(new_k, seg, row, false, lane);
+        quantize_vector_warp_raw<true, KB, VB>(new_v, seg, row, true, lane);
+      } else {
+        quantize_vector_warp_raw<false, KB, VB>(new_k, seg, row, false, lane);
+        quantize_vector_warp_raw<false, KB, VB>(new_v, seg, row, true, lane);
+      }
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+    } else if (lane == 0) {
+      record_status(a.status, KVQ_ERR_OUT_OF_RANGE);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -688,10 +710,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
     const uint32_t my_meta = smem_u32(&sm.meta[0][mkind][32 * warp + 16 * mseg + mrow0]);
 #pragma unroll
     for (int i = 0; i < kNV; ++i)  // the deferred chunk, if it is one of the first three
-      if (i == c_defer) {
-        if (!mbar_wait<kWaitTag>(&sm.app_done, 0u, abort)) bad = true;
-        okq[i] = issue(i, bfirst[i], i);
-      }
+      if (i == c_defer) okq[i] = issue(i, bfirst[i], i);
     Ring3 r{0, 0u};  // chunk c: staging slot, key-code, value and factor buffers r.i
 #pragma unroll 1
     for (int c = 0; c < nchunks; ++c) {
@@ -713,7 +732,6 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
       __syncwarp();
       okq[0] = okq[1];
       okq[1] = okq[2];
-      if (c + kNV == c_defer && !mbar_wait<kWaitTag>(&sm.app_done, 0u, abort)) bad = true;
       okq[2] = c + kNV < nchunks ? issue(c + kNV, bq[0], r.i) : 0u;
       prefetch_seg(bq[3]);
 #pragma unroll
@@ -817,25 +835,6 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
     // softmax warps: thread stok <-> token stok of S, value position stok of O
     const int sw = warp - kLoadWarps;
     const int stok = tid - 32 * kLoadWarps;
-    // fused one-token append: in the split holding position L-1, warps 4 and
-    // 5 write the new token's K and V of kv head h into that position while
-    // the first chunks are in flight (they would wait for the first QK
-    // anyway); the loaders copy the chunk holding it only after app_done
-    // (the proxy fence orders the writes before the bulk copy)
-    if (c_defer >= 0 && sw < 2) {
-      const int32_t p = bt_row[(L - 1) / kBlockSize];
-      if (p >= 0 && p < a.num_blocks) {
-        uint8_t* seg = const_cast<uint8_t*>(pool_h) + static_cast<int64_t>(p) * pstride;
-        if (a.new_bf16)
-          quantize_vector_warp_raw<true, KB, VB>(new_raw, seg, (L - 1) % kBlockSize, sw == 1, lane);
-        else
-          quantize_vector_warp_raw<false, KB, VB>(new_raw, seg, (L - 1) % kBlockSize, sw == 1, lane);
-        asm volatile("fence.proxy.async.global;" ::: "memory");
-      } else if (lane == 0 && sw == 0) {
-        record_status(a.status, KVQ_ERR_OUT_OF_RANGE);
-      }
-      mbar_arrive(&sm.app_done);
-    }
     const uint32_t my_lanes = tbase + (static_cast<uint32_t>(sw * 32) << 16);
     const uint32_t my_pm = smem_u32(sm.pm[0]) + (stok >> 3) * 256 + (stok & 7) * 16;
     float qs[G], mr[G], lr[G], zr[G], oacc[G];  // oacc: in units of the output scale below
