@@ -55,8 +55,8 @@ BYTES_PER_TOKEN_HEAD = 104
 # does), with the SHA-256 of the kernel code it was taken on (decode_code_sha256:
 # comments stripped).  Reported as roofline.traffic only while the code still
 # has that hash.
-DECODE_TRAFFIC = {"sha256": "93b50dd095d7bec7682b7febc315ba2e622b2c6d982bbd0351024dda468a6b2a",
-                  "bytes": 13766400}
+DECODE_TRAFFIC = {"sha256": "89b58e05a9664ebd7312c6653dabae911e1136d8fdfbd40679ffde1fc8a754fe",
+                  "bytes": 13773568}
 
 
 def decode_code_sha256():
