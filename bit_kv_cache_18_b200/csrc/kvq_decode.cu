@@ -292,11 +292,6 @@ __device__ __forceinline__ uint2 lds64(uint32_t addr) {
   asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(addr));
   return r;
 }
-__device__ __forceinline__ float lds_f32(uint32_t addr) {  // not hoisted out of loops
-  float r;
-  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(r) : "r"(addr));
-  return r;
-}
 __device__ __forceinline__ void sts64(uint32_t addr, uint32_t a, uint32_t b) {
   asm volatile("st.shared.v2.b32 [%0], {%1,%2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
 }
@@ -887,10 +882,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
       const uint32_t hsv = sm.meta[r.i][2][stok];
       const bool valid = (hsv & 0x8000u) == 0;  // a token (not marked absent by the loaders)
       // S_K c1, Z_K, S_V 2^29, Z_V (0 for an absent token)
-      // (c1 is read again each chunk: keeping it in a register made the
-      // kernel spill)
-      const float4 mt = make_float4(h2f(sm.meta[r.i][0][stok]) * lds_f32(smem_u32(&sm.c1)), h2f(sm.meta[r.i][1][stok]),
-                                    h2f(hsv) * kFix,
+      const float4 mt = make_float4(h2f(sm.meta[r.i][0][stok]) * c1, h2f(sm.meta[r.i][1][stok]), h2f(hsv) * kFix,
                                     valid ? h2f(sm.meta[r.i][3][stok]) : 0.0f);
       // E with S_V < 2^E, from the fp16 exponent of S_V (-14 for subnormals and 0)
       const float e = static_cast<float>(static_cast<int>((hsv >> 10) & 31u) - 14);
