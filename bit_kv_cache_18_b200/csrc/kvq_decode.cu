@@ -10,11 +10,12 @@
 //     bring their two segments of each chunk into a private kNV-slot
 //     shared-memory ring with bulk copies (TMA, one instruction per segment)
 //     kNV chunks ahead, after an L2 prefetch six chunks ahead; read them
-//     with conflict-free 16-byte loads; spread the 4-bit key codes to one
-//     byte each into tensor memory (A of QK, 16x256b stores whose fragment
-//     layout matches the 16-byte pieces) and the 2-bit value codes to one
-//     byte each into shared memory (A of PV), and publish the per-token
-//     factors;
+//     with conflict-free 16-byte loads; spread the key codes (4 bits in the
+//     default k4v2 preset, 2 or 8 in others) to one byte each into tensor
+//     memory (A of QK, 16x256b stores whose fragment layout matches the
+//     16-byte pieces) and the value codes (2 or 4 bits) to one byte each
+//     into shared memory (A of PV), and publish the per-token factors as
+//     stored (fp16; the softmax warps convert them);
 //   * one MMA warp (tensor-memory owner) whose lane 0 issues, in order,
 //     QK(0), QK(1), PV(0), QK(2), PV(1), ... as tcgen05.mma (M = 128, N = 32):
 //       QK:  S  = codes_K (128 tok x 128) . digits(q~)^T  (u8 x s8 -> s32)
@@ -63,11 +64,13 @@
 // The accumulator is also restarted every 128 chunks, which keeps every s32
 // sum below 2^31.
 //
-// Code order.  The byte spreading permutes the 128 positions of a row
-// (keys: position 32j + 8m + 4h + b holds dim 32m + 8j + 2b + h; values:
-// position 16i + 4k + j holds dim 16i + 4j + k, times 4^k).  The query digits are
-// written in the key order, so S is exact, and the output rows are put back
-// in dim order, and divided by 4^k, when O is read.
+// Code order.  The byte spreading permutes the 128 positions of a row (for
+// k4v2 keys: position 32j + 8m + 4h + b holds dim 32m + 8j + 2b + h; values:
+// position 16i + 4k + j holds dim 16i + 4j + k, times 4^k; the other
+// presets' maps are given with key_pos_of_dim and value_dim_of_pos).  The
+// query digits are written in the key order, so S is exact, and the output
+// rows are put back in dim order, and divided by the spread's factor, when
+// O is read.
 #include <math_constants.h>
 
 #include <type_traits>
