@@ -112,6 +112,56 @@ def test_argument_checks_need_no_device(kvq):
                                   None) == kvq.KVQ_ERR_UNSUPPORTED
 
 
+def test_fused_and_noalloc_argument_checks_need_no_device(kvq):
+    L = kvq.lib()
+    d = kvq.make_desc(4, 2)
+    d.pool = 0x1000
+    one = ctypes.c_void_p(0x4000)
+    k_new, v_new = ctypes.c_void_p(0x5000), ctypes.c_void_p(0x6000)
+
+    def fused(k, v, in_dtype, stride, batch):
+        return L.kvq_append_decode_attention(ctypes.byref(d), k, v, in_dtype, stride, one, kvq.KVQ_BF16, batch, 16,
+                                             one, 1, one, 16, 0.0, one, kvq.KVQ_F32, None, 0, None)
+
+    # the new rows: fp16/bf16 only, present, 16-byte aligned, a stride that holds a row
+    assert fused(k_new, v_new, kvq.KVQ_F32, 256, 1) == kvq.KVQ_ERR_INVALID
+    assert fused(None, v_new, kvq.KVQ_BF16, 256, 1) == kvq.KVQ_ERR_INVALID
+    assert fused(ctypes.c_void_p(0x5008), v_new, kvq.KVQ_BF16, 256, 1) == kvq.KVQ_ERR_INVALID
+    assert fused(k_new, v_new, kvq.KVQ_BF16, 128, 1) == kvq.KVQ_ERR_INVALID
+    assert fused(k_new, v_new, kvq.KVQ_BF16, 260, 1) == kvq.KVQ_ERR_INVALID
+    # then the decode rules: here the missing workspace
+    assert fused(k_new, v_new, kvq.KVQ_BF16, 256, 1) == kvq.KVQ_ERR_WORKSPACE
+    # an empty batch launches nothing
+    assert fused(None, None, kvq.KVQ_BF16, 256, 0) == kvq.KVQ_OK
+    # no-allocation entry point: an empty batch is a no-op, a bad head count is rejected
+    assert L.kvq_decode_attention_noalloc(ctypes.byref(d), one, kvq.KVQ_BF16, 0, 16, one, 1, one, 16, 0.0, one,
+                                          kvq.KVQ_F32, None) == kvq.KVQ_OK
+    assert L.kvq_decode_attention_noalloc(ctypes.byref(d), one, kvq.KVQ_BF16, 1, 15, one, 1, one, 16, 0.0, one,
+                                          kvq.KVQ_F32, None) == kvq.KVQ_ERR_INVALID
+
+
+@pytest.mark.parametrize("kb,vb", [(8, 8), (3, 2), (4, 1)])
+def test_unsupported_presets_are_rejected_before_any_launch(kvq, kb, vb):
+    L = kvq.lib()
+    d = kvq.make_desc(4, 2)
+    d.k_bits, d.v_bits = kb, vb
+    d.pool = 0x1000
+    one = ctypes.c_void_p(0x4000)
+    assert L.kvq_cache_bytes(ctypes.byref(d)) == 0
+    assert L.kvq_quantize_append(ctypes.byref(d), one, one, kvq.KVQ_BF16, 1, 256, one, None) == kvq.KVQ_ERR_UNSUPPORTED
+    assert L.kvq_decode_attention(ctypes.byref(d), one, kvq.KVQ_BF16, 1, 16, one, 1, one, 16, 0.0, one, kvq.KVQ_F32,
+                                  one, 1 << 20, None) == kvq.KVQ_ERR_UNSUPPORTED
+    assert L.kvq_decode_workspace_bytes(ctypes.byref(d), 1, 16, 16) == 0
+
+
+@pytest.mark.parametrize("preset", [(4, 2), (4, 4), (2, 2), (8, 4)])
+def test_workspace_bytes_do_not_depend_on_the_preset(kvq, preset):
+    """The split-K partials hold fp32 (o~, m, l) per query head and split,
+    whatever the code widths."""
+    assert kvq.kvq_decode_workspace_bytes(1024, 8, 1, 64, 16384, blocks_per_split=1024, preset=preset) == \
+        256 + 64 * 1 * 132 * 4
+
+
 def test_workspace_bytes(kvq):
     n = kvq.kvq_decode_workspace_bytes(1024, 8, 1, 64, 16384)
     assert n > 0 and n % 4 == 0
