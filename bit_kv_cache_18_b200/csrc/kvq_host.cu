@@ -1,6 +1,7 @@
 // kvq_host.cu -- the extern "C" entry points declared in include/kvq.h:
 // argument validation, the split-K plan, host-only block-table helpers, the
 // device status word, and the kernel launches.
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstdlib>
@@ -99,7 +100,14 @@ int device_sm_count() {
 // start-up worth about two chunks (the first loads, the query rotation, the
 // partial record), and every extra split adds a tenth of a chunk of merge
 // work.  Default splits are whole chunks.  A requested blocks_per_split is
-// raised if it would need more splits than the cap.
+// raised if it would need more splits than the cap.  No split is longer
+// than kMaxSplitBlocks blocks unless the split cap forces it: the kernel's
+// fixed-point probabilities drop tokens more than about 2^30 below the
+// split's running max, a bias that grows with the tokens of one split (an
+// emulation of the arithmetic on a 131072-token sequence: 1.9e-3 in one
+// split, 2.5e-4 in splits of 2048 blocks, 1.1e-4 in splits of 512).
+constexpr int64_t kMaxSplitBlocks = 2048;
+
 int plan_decode(int32_t batch, int32_t num_kv_heads, int32_t num_q_heads, int32_t max_seq_len,
                 int32_t bps_request, DecodePlan* plan) {
   if (batch < 0 || num_kv_heads <= 0 || num_q_heads <= 0 || max_seq_len < 0 || bps_request < 0)
@@ -107,19 +115,21 @@ int plan_decode(int32_t batch, int32_t num_kv_heads, int32_t num_q_heads, int32_
   const int64_t nb = (static_cast<int64_t>(max_seq_len) + kBlockSize - 1) / kBlockSize;
   const int64_t cap = decode_max_splits();
   const int64_t cb = decode_chunk_blocks();
+  const int64_t bmax = nb > kMaxSplitBlocks * cap ? (nb + cap - 1) / cap : kMaxSplitBlocks;
   int64_t bps = bps_request;
   if (nb == 0) {
     bps = 1;
   } else if (bps == 0) {
     const int64_t units = static_cast<int64_t>(batch) * num_kv_heads;
     const int64_t slots = static_cast<int64_t>(device_sm_count()) * decode_ctas_per_sm();
+    const int64_t bmax_c = (bmax + cb - 1) / cb * cb;  // in whole chunks
     double best = 1e300;
-    bps = (nb + cb - 1) / cb * cb;
+    bps = std::min((nb + cb - 1) / cb * cb, bmax_c);
     int64_t last = -1;
     for (int64_t n = 1; n <= cap && n <= nb; ++n) {
       const int64_t b = ((nb + n - 1) / n + cb - 1) / cb * cb;  // whole chunks
       const int64_t ns = (nb + b - 1) / b;
-      if (ns > cap || b == last) continue;
+      if (ns > cap || b == last || b > bmax_c) continue;
       last = b;
       const int64_t waves = (units * ns + slots - 1) / slots;
       const double cost = static_cast<double>(waves) * (static_cast<double>(b) / cb + 2.0) + 0.1 * ns;
@@ -128,8 +138,9 @@ int plan_decode(int32_t batch, int32_t num_kv_heads, int32_t num_q_heads, int32_
         bps = b;
       }
     }
-  } else if ((nb + bps - 1) / bps > cap) {
-    bps = (nb + cap - 1) / cap;
+  } else {
+    if ((nb + bps - 1) / bps > cap) bps = (nb + cap - 1) / cap;
+    if (bps > bmax) bps = bmax;
   }
   const int64_t nsplit = nb > 0 ? (nb + bps - 1) / bps : 1;
   plan->blocks_per_split = static_cast<int32_t>(bps);

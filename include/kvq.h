@@ -175,8 +175,11 @@ int kvq_decode_attention(const kvq_cache_desc* desc, const void* q, kvq_dtype q_
 /* As kvq_decode_attention / kvq_decode_workspace_bytes, with the split-K
  * granularity chosen by the caller: blocks_per_split physical blocks (of 16
  * tokens) per CTA; 0 picks the default.  A value that would cut a sequence
- * into more than 64 splits is raised to ceil(blocks / 64).  The workspace
- * size depends on it. */
+ * into more than 64 splits is raised to ceil(blocks / 64); a value above
+ * 2048 blocks (32768 tokens) is lowered to 2048, or to that 64-split minimum
+ * if it is larger, since a longer split loses accuracy in the kernel's
+ * fixed-point probabilities (the default plan obeys the same bound).  The
+ * workspace size depends on it. */
 size_t kvq_decode_workspace_bytes_ex(const kvq_cache_desc* desc, int32_t batch,
                                      int32_t num_q_heads, int32_t max_seq_len,
                                      int32_t blocks_per_split);

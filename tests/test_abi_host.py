@@ -162,6 +162,24 @@ def test_workspace_bytes_do_not_depend_on_the_preset(kvq, preset):
         256 + 64 * 1 * 132 * 4
 
 
+def test_split_length_is_capped(kvq):
+    """A requested split longer than 2048 blocks (32768 tokens) is cut
+    further, unless 64 splits could not cover the sequence then; the
+    workspace holds one partial record per query head and split."""
+    rec = 64 * 132 * 4
+    assert kvq.kvq_decode_workspace_bytes(8192, 8, 1, 64, 131072, blocks_per_split=8192) == 256 + 4 * rec
+    assert kvq.kvq_decode_workspace_bytes(8192, 8, 1, 64, 131072, blocks_per_split=2048) == 256 + 4 * rec
+    assert kvq.kvq_decode_workspace_bytes(8192, 8, 1, 64, 131072, blocks_per_split=1024) == 256 + 8 * rec
+    # 16549 tokens = 1035 blocks still fit in one split
+    assert kvq.kvq_decode_workspace_bytes(1035, 8, 1, 64, 16549, blocks_per_split=1035) == 256 + 1 * rec
+    # beyond 64 x 2048 blocks the split cap wins: 64 splits of ceil(blocks / 64)
+    big = 64 * 2048 * 16 + 80
+    assert kvq.kvq_decode_workspace_bytes(1, 8, 1, 64, big, blocks_per_split=100000) == 256 + 64 * rec
+    # the default plan obeys the same bound
+    n_default = (kvq.kvq_decode_workspace_bytes(8192, 8, 1, 64, 131072) - 256) // rec
+    assert n_default >= 4
+
+
 def test_workspace_bytes(kvq):
     n = kvq.kvq_decode_workspace_bytes(1024, 8, 1, 64, 16384)
     assert n > 0 and n % 4 == 0
