@@ -121,13 +121,14 @@ class ClockSampler:
 
     Reads NVML from a background thread every ~2 ms (read-only queries; the
     timed regions here last tens of milliseconds, too short for
-    nvidia-smi's 200 ms loop), falling back to `nvidia-smi -lms 200`.  The
-    samples are written to gpurun_out/clocks_rank<i>.csv."""
+    nvidia-smi's 200 ms loop), falling back to `nvidia-smi -lms 200` into a
+    temporary file.  The samples are written as CSV to `log_path` when one is
+    given (bench.py --clock-log)."""
 
     REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
                ("sw_power_cap", 0x4), ("hw_power_brake_slowdown", 0x80))
 
-    def __init__(self, index: int, uuid: str | None = None, period_s: float = 0.002):
+    def __init__(self, index: int, uuid: str | None = None, period_s: float = 0.002, log_path: str | None = None):
         self.index = index
         self.uuid = uuid
         self.period = period_s
@@ -135,7 +136,8 @@ class ClockSampler:
         self.proc = None
         self.thread = None
         self.nvml = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        self.log_path = log_path
+        self.path = None  # nvidia-smi fallback output (a temporary file)
 
     def _poll(self):
         nv, h = self.nvml, self.handle
@@ -169,8 +171,9 @@ class ClockSampler:
         except Exception:  # noqa: BLE001
             self.nvml = None
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.f = open(self.path, "w")
+            import tempfile
+            fd, self.path = tempfile.mkstemp(prefix="kvq_clocks_", suffix=".csv")
+            self.f = os.fdopen(fd, "w")
             fields = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active")
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={fields}", "--format=csv,noheader,nounits",
                                           "-i", str(self.index), "-lms", "200"], stdout=self.f,
@@ -183,14 +186,6 @@ class ClockSampler:
         if self.thread is not None:
             self.stop.set()
             self.thread.join(timeout=5)
-            try:
-                os.makedirs(os.path.dirname(self.path), exist_ok=True)
-                with open(self.path, "w") as f:
-                    f.write("t_s,sm_mhz,max_sm_mhz,power_w,reasons_hex\n")
-                    for t, sm, mx, pw, rs in self.rows:
-                        f.write(f"{t:.4f},{sm},{mx},{pw:.1f},{rs:#x}\n")
-            except OSError:
-                pass
             self.nvml.nvmlShutdown()
         if self.proc is not None:
             self.proc.terminate()
@@ -205,6 +200,15 @@ class ClockSampler:
                     if len(p) >= 4 and p[0].replace(".", "").isdigit():
                         rs = int(p[3], 16) if p[3].lower().startswith("0x") else 0
                         self.rows.append((0.0, float(p[0]), float(p[1]), float(p[2] or 0), rs))
+            os.unlink(self.path)
+        if self.log_path:
+            try:
+                with open(self.log_path, "w") as f:
+                    f.write("t_s,sm_mhz,max_sm_mhz,power_w,reasons_hex\n")
+                    for t, sm, mx, pw, rs in self.rows:
+                        f.write(f"{t:.4f},{sm},{mx},{pw:.1f},{int(rs):#x}\n")
+            except OSError:
+                pass
 
     def summary(self):
         if not self.rows:

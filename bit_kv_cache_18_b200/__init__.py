@@ -76,6 +76,7 @@ def lib():
                 "kvq_append_decode_attention": (ctypes.c_int, [dp, vp, vp, ctypes.c_int, i64, vp, ctypes.c_int, i32,
                                                                i32, vp, i32, vp, i32, f32, vp, ctypes.c_int, vp, sz,
                                                                vp]),
+                "kvq_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_uint32, vp, vp]),
                 "kvq_last_device_status": (ctypes.c_int, [vp]),
                 "kvq_error_string": (ctypes.c_char_p, [ctypes.c_int]),
             }
@@ -239,6 +240,13 @@ def kvq_decode_attention_noalloc(pool, num_blocks, num_kv_heads, q, block_table,
                                             _ptr(block_table), block_table.shape[1], _ptr(seq_lens), max_seq_len,
                                             softmax_scale, _ptr(out), _dtype_code(out), _stream_ptr(stream))
     _check(rc, "kvq_decode_attention_noalloc")
+
+
+def kvq_selftest_wait_timeout(polls: int, elapsed_ns=None, stream=None):
+    """Launch the bounded-wait self-test (a wait that must give up after
+    `polls` polls); elapsed_ns: optional int64 device tensor of one element."""
+    rc = lib().kvq_selftest_wait_timeout(polls, _ptr(elapsed_ns), _stream_ptr(stream))
+    _check(rc, "kvq_selftest_wait_timeout")
 
 
 def kvq_last_device_status(stream=None) -> int:

@@ -153,6 +153,10 @@ constexpr int kSmemBytesOf = static_cast<int>((sizeof(Smem<kSeg>) + 1023) / 1024
 static_assert(kSmemBytesOf<Fmt<4, 2>::kSegBytes> <= 113 * 1024, "two CTAs per SM (k4v2)");
 static_assert(kSmemBytesOf<Fmt<2, 2>::kSegBytes> <= 113 * 1024, "two CTAs per SM (k2v2)");
 static_assert(kSmemBytesOf<Fmt<8, 4>::kSegBytes> <= 227 * 1024, "one CTA per SM (k8v4)");
+// The tensor-memory rule of kvq_internal.cuh: no SM holds three of these
+// CTAs (each allocates 256 of the 512 columns), since three never fit in the
+// SM's 228 KB of shared memory (1 KB per CTA is reserved by the hardware).
+static_assert(3 * (kSmemBytesOf<Fmt<2, 2>::kSegBytes> + 1024) > 228 * 1024, "at most two decode CTAs per SM");
 
 // Position in a ring of three buffers and the parity of its current use.
 struct Ring3 {
@@ -201,13 +205,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return done != 0;
 }
-// Bounded, warp-uniform wait for a barrier phase.  False if it never came or
-// another warp already gave up (then every later wait returns at once and
-// the kernel runs to its end on void data, which it reports).  The slow loop
-// is a call, one copy per preset (kTag), which keeps the wait sites small.
+// Bounded, warp-uniform wait for a barrier phase.  False if it never came
+// within `limit` polls or another warp already gave up (then every later
+// wait returns at once and the kernel runs to its end on void data, which it
+// reports; the loaders stop issuing copies and wait for those in flight
+// before the CTA exits).  The slow loop is a call, one copy per preset
+// (kTag), which keeps the wait sites small.
 template <int kTag>
-__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  for (uint32_t it = 0; it < kWaitLimit; ++it) {
+__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t limit) {
+  for (uint32_t it = 0; it < limit; ++it) {
     if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
     if ((it & 15u) == 15u && __any_sync(0xffffffffu, *abort != 0)) return false;
   }
@@ -217,7 +223,7 @@ __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, vola
 template <int kTag>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
-  return mbar_wait_slow<kTag>(bar, parity, abort);
+  return mbar_wait_slow<kTag>(bar, parity, abort, kWaitLimit);
 }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -533,7 +539,11 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
     }
   }
   int L = a.seq_lens[b];
-  if (L < 0 || L > a.max_seq_len || L > a.max_blocks_per_seq * kBlockSize) {
+  // a length outside [0, max_seq_len] or beyond the table row is recorded
+  // and the read is truncated to what the row covers; the fused append is
+  // then skipped (its position would be a clamped one, not seq_lens[b] - 1)
+  const bool l_bad = L < 0 || L > a.max_seq_len || L > a.max_blocks_per_seq * kBlockSize;
+  if (l_bad) {
     if (tid == 0) record_status(a.status, KVQ_ERR_OUT_OF_RANGE);
     L = max(L, 0);
     L = min(L, a.max_seq_len);
@@ -583,7 +593,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
   // the chunk holding the block that the fused append writes is copied only
   // after the set-up barrier (-1: none)
   int c_defer = -1;
-  if (a.k_new != nullptr && L > 0) {
+  if (a.k_new != nullptr && L > 0 && !l_bad) {
     const int bn = (L - 1) / kBlockSize;
     if (bn >= blk0 && bn < blk1) c_defer = (bn - blk0) / kChunkBlocks;
   }
@@ -710,9 +720,15 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
     for (int i = 0; i < kNV; ++i)  // the deferred chunk, if it is one of the first three
       if (i == c_defer) okq[i] = issue(i, bfirst[i], i);
     Ring3 r{0, 0u};  // chunk c: staging slot, key-code, value and factor buffers r.i
+    // staging slots whose bulk copy is still in flight after a failed wait:
+    // bit i, and its phase parity in bit 4 + i
+    uint32_t pend = 0u;
 #pragma unroll 1
     for (int c = 0; c < nchunks; ++c) {
-      if (!mbar_wait<kWaitTag>(&sm.full[warp][r.i], r.ph, abort)) bad = true;
+      if (!mbar_wait<kWaitTag>(&sm.full[warp][r.i], r.ph, abort)) {
+        bad = true;
+        pend |= (1u << r.i) | (r.ph << (4 + r.i));
+      }
       const uint32_t sb = my_stg + r.i * (2 * kSeg);
       KeyRaw<KB> kr[2];
       uint4 vr[2][VB / 2];  // VB = 2: one 16-byte piece per segment; VB = 4: two
@@ -730,7 +746,8 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
       __syncwarp();
       okq[0] = okq[1];
       okq[1] = okq[2];
-      okq[2] = c + kNV < nchunks ? issue(c + kNV, bq[0], r.i) : 0u;
+      // (after a failed wait no copy is issued any more: see the drain below)
+      okq[2] = c + kNV < nchunks && !bad ? issue(c + kNV, bq[0], r.i) : 0u;
       prefetch_seg(bq[3]);
 #pragma unroll
       for (int i = 0; i < 5; ++i) bq[i] = bq[i + 1];
@@ -786,6 +803,14 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
       mbar_arrive(&sm.kv_ready[r.i]);
       r.next();
     }
+    // Exit ordering after a wait gave up: this warp issued no copy since, and
+    // every copy it issued before lands in its own staging ring, so it waits
+    // (bounded, ignoring the abort flag) for the ones still in flight; the
+    // CTA barrier below then orders this before the CTA releases its shared
+    // memory.
+#pragma unroll
+    for (int i = 0; i < kNV; ++i)
+      if ((pend >> i) & 1u) mbar_wait_final(&sm.full[warp][i], (pend >> (4 + i)) & 1u);
   } else if (warp == kMmaWarp) {
     // one lane issues, in this order: QK(0), QK(1), PV(0), QK(2), PV(1), ...
     const uint32_t qb0 = smem_u32(sm.qb);
@@ -1128,7 +1153,38 @@ cudaError_t launch_p(const DecodeArgs& a, cudaStream_t stream) {
   }
 }
 
+// Failure-detection self-test: one warp waits, through the decode kernel's
+// bounded wait (the same slow loop), on a barrier that nothing arrives at.
+// Nothing else is issued (no bulk copy, no MMA, no tensor memory), so
+// nothing is in flight when the wait gives up; the kernel records
+// KVQ_ERR_DEVICE_TIMEOUT and the time the `limit` polls took.
+__global__ void __launch_bounds__(32) wait_timeout_probe_kernel(int* status, uint32_t limit, uint64_t* elapsed_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  const int lane = threadIdx.x;
+  if (lane == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncwarp();
+  uint64_t t0, t1;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+  const bool ok = mbar_wait_slow<0>(&bar, 0u, &abort_flag, limit);
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t1));
+  if (lane == 0) {
+    if (!ok) record_status(status, KVQ_ERR_DEVICE_TIMEOUT);
+    if (elapsed_ns != nullptr) *elapsed_ns = t1 - t0;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_wait_probe(int* status, uint32_t limit, uint64_t* elapsed_ns, cudaStream_t stream) {
+  wait_timeout_probe_kernel<<<1, 32, 0, stream>>>(status, limit, elapsed_ns);
+  return cudaGetLastError();
+}
+uint32_t wait_poll_limit() { return kWaitLimit; }
 
 int decode_ctas_per_sm() {
   static int cached[64] = {};

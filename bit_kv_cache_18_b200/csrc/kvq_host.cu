@@ -408,7 +408,10 @@ int kvq_decode_attention_noalloc(const kvq_cache_desc* desc, const void* q, kvq_
                                  kvq_dtype out_dtype, void* stream) {
   int rc = check_desc(desc);
   if (rc != KVQ_OK) return rc;
-  if (batch < 0 || num_q_heads <= 0 || num_q_heads % desc->num_kv_heads != 0) return KVQ_ERR_INVALID;
+  // the argument rules of kvq_decode_attention, checked before the scratch
+  // is sized (decode_impl repeats them)
+  if (batch < 0 || num_q_heads <= 0) return KVQ_ERR_INVALID;
+  if (num_q_heads % desc->num_kv_heads != 0) return KVQ_ERR_UNSUPPORTED;
   if (batch == 0) return KVQ_OK;
   DecodePlan plan;
   rc = plan_decode(batch, desc->num_kv_heads, num_q_heads, max_seq_len, 0, &plan);
@@ -423,6 +426,15 @@ int kvq_decode_attention_noalloc(const kvq_cache_desc* desc, const void* q, kvq_
   return kvq_decode_attention_ex(desc, q, q_dtype, batch, num_q_heads, block_table, max_blocks_per_seq,
                                  seq_lens, max_seq_len, softmax_scale, out, out_dtype, scratch,
                                  kStaticScratchBytes, 0, stream);
+}
+
+int kvq_selftest_wait_timeout(uint32_t polls, uint64_t* elapsed_ns, void* stream) {
+  if (polls == 0 || polls > wait_poll_limit()) return KVQ_ERR_INVALID;
+  int* status = device_status_ptr();
+  if (!status) return KVQ_ERR_CUDA;
+  return launch_wait_probe(status, polls, elapsed_ns, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? KVQ_OK
+             : KVQ_ERR_CUDA;
 }
 
 int kvq_last_device_status(void* stream) {

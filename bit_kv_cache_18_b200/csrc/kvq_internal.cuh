@@ -192,8 +192,20 @@ __device__ __forceinline__ void quantize_vector_warp(const uint8_t* src, uint8_t
 // may become resident while the kernel before it in the stream is still
 // finishing.  It executes pdl_wait() before it reads or writes any memory
 // that an earlier kernel may touch (inputs, pool, workspace, outputs), and
-// pdl_trigger() once it holds no resource a still-unlaunched CTA of its own
-// grid could need (tensor memory), which lets the next kernel's CTAs set up.
+// pdl_trigger(), which lets the next kernel's CTAs become resident and set
+// up, at a point chosen by the tensor-memory rule below.
+//
+// Tensor-memory rule.  The decode and bulk-quantize kernels allocate tensor
+// memory (256 of an SM's 512 columns) before their pdl_wait(), and an
+// allocation blocks until the columns are free.  A CTA that waits in
+// pdl_wait() for grid A must therefore never hold columns that a CTA of A
+// still has to allocate.  Each kernel triggers only after its own CTA
+// holds all the tensor memory it will ever take (the bulk quantize: right
+// after its allocation; decode: after its deallocation), so by the time a
+// dependent CTA allocates, every CTA of the grid before it has either
+// allocated already or finished.  Shared memory backs this up: no SM can
+// hold three CTAs of these kernels at once (each asks for more than a third
+// of the SM's 228 KB), so at most two 256-column allocations meet on an SM.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
@@ -257,6 +269,11 @@ struct DecodeArgs {
   int32_t k_bits, v_bits;  // preset
 };
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+
+// Failure-detection self-test (kvq_selftest_wait_timeout) and the polls a
+// kernel's bounded wait makes before it gives up.
+cudaError_t launch_wait_probe(int* status, uint32_t limit, uint64_t* elapsed_ns, cudaStream_t stream);
+uint32_t wait_poll_limit();
 
 // Split-K plan of a decode call on the current device.
 struct DecodePlan {

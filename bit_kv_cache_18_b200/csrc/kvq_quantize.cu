@@ -189,6 +189,10 @@ struct __align__(1024) BulkSmem {
 };
 constexpr int kBulkSmemBytes = static_cast<int>(sizeof(BulkSmem));
 static_assert(kBulkSmemBytes <= 113 * 1024, "two CTAs per SM");
+// The tensor-memory rule of kvq_internal.cuh: three CTAs that allocate 256
+// columns each (this kernel's and the decode kernel's, whose shared memory
+// is larger) never fit on one SM's 228 KB.
+static_assert(3 * (kBulkSmemBytes + 1024) > 228 * 1024, "at most two tensor-memory CTAs per SM");
 
 // Instruction descriptor, kind::f16: D f32, A and B f16 or bf16, A in
 // tensor memory, B K-major, N = 128, M = 128.
@@ -385,7 +389,6 @@ __global__ void __launch_bounds__(kBulkThreads, 2)
                     int32_t n_tokens, int64_t stride_bytes, const int32_t* __restrict__ slots, int* status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   BulkSmem& sm = *reinterpret_cast<BulkSmem*>(smem_raw);
-  pdl_trigger();  // (the grid is persistent: every CTA is resident at once)
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
@@ -417,6 +420,13 @@ __global__ void __launch_bounds__(kBulkThreads, 2)
     }
   }
   async_proxy_fence();  // (H is read by the tensor cores)
+  // Release the dependent grid only once this CTA holds its tensor memory
+  // (the barrier orders warp 0's allocation before every thread's trigger):
+  // a dependent CTA that lands on this SM may allocate before its own
+  // dependency wait, and must then never take columns this CTA still needs.
+  // (The grid is persistent: every CTA is resident at once.)
+  __syncthreads();
+  pdl_trigger();
   pdl_wait();
 
   const int64_t n_vec = static_cast<int64_t>(n_tokens) * hkv;

@@ -57,9 +57,11 @@
  *     exception, abort or device trap ever leaves the library: argument
  *     errors are caught on the host; out-of-range block ids and slots met on
  *     the device are skipped and recorded in the device status word.
- *   - Supported geometry: head_dim 128, group 128, block_size 16, k_bits 4,
- *     v_bits 2, num_q_heads a multiple of num_kv_heads with G = Hq/Hkv in
- *     {1, 2, 4, 8}.  Anything else returns KVQ_ERR_UNSUPPORTED.
+ *   - Supported geometry: head_dim 128, group 128, block_size 16, and one of
+ *     four presets (k_bits, v_bits) = (4, 2) (the pages' default,
+ *     kvarn_k4v2_g128), (4, 4), (2, 2) or (8, 4); num_q_heads a multiple of
+ *     num_kv_heads with G = Hq/Hkv in {1, 2, 4, 8}.  Anything else returns
+ *     KVQ_ERR_UNSUPPORTED.
  */
 #ifndef KVQ_H
 #define KVQ_H
@@ -107,10 +109,21 @@ int kvq_parse_dtype(const char* s, int32_t* k_bits, int32_t* v_bits, int32_t* gr
 
 /* Bytes of the pool described by desc (num_blocks * num_kv_heads * SEG, SEG
  * = 1664 for k4v2_g128, 2176 for k4v4, 1152 for k2v2, 3200 for k8v4), or 0
- * if desc is NULL or unsupported.  Host only. */
+ * if desc is NULL or unsupported.  Host only.  The pool is the paged cache
+ * the KVarN backend writes into ("блоки кэша": the cache blocks of "Трюк
+ * Huawei с KV-кэшем", section "Заявка, которая ломает привычный
+ * компромисс", whose 3-5x capacity over FP16 is this byte count's ratio to
+ * 512 bytes per token-head); per-token cache bytes are the quantity the
+ * HBM-math section of "Kompresja pamięci podręcznej KV to decyzja
+ * infrastrukturalna..." (encorp.ai) reasons with. */
 size_t kvq_cache_bytes(const kvq_cache_desc* desc);
 
-/* Assign physical blocks to sequences, host only (no device work).
+/* Assign physical blocks to sequences, host only (no device work): the job
+ * of vLLM's paged block manager, which the KVarN backend plugs into ("Трюк
+ * Huawei с KV-кэшем": lede, a ready vLLM backend; section "Заявка, которая
+ * ломает привычный компромисс": the cache blocks; "KVarN vs TurboQuant"
+ * (dothoosh.com), next-step list: fixed-size pages today, variable page
+ * sizes announced).  Here it builds the tables the tests and benchmarks use.
  * Sequence b needs ceil(seq_lens[b]/block_size) blocks, which are taken in
  * order from a permutation of 0..num_blocks-1: the identity when
  * shuffle_seed == 0, otherwise a seeded shuffle (SplitMix64-driven
@@ -124,7 +137,10 @@ int kvq_block_table(int32_t num_blocks, int32_t block_size, const int32_t* seq_l
                     int32_t* blocks_used_out);
 
 /* slots_out[i] = block_table[seq_ids[i]][positions[i]/block_size] *
- * block_size + positions[i] % block_size, host only.  An entry whose block
+ * block_size + positions[i] % block_size, host only: vLLM's slot rule for
+ * where a token's entry goes in the paged cache (the vLLM backend and its
+ * cache blocks of "Трюк Huawei с KV-кэшем", section "Заявка, которая ломает
+ * привычный компромисс"); kvq_quantize_append takes these slots.  An entry whose block
  * is -1 gives -1 (the write path then skips that token).  All pointers are
  * host memory; returns KVQ_ERR_INVALID for a negative position or a position
  * beyond the table row. */
@@ -147,7 +163,12 @@ int kvq_quantize_append(const kvq_cache_desc* desc, const void* k, const void* v
 /* Workspace bytes kvq_decode_attention needs for this problem on the current
  * device (split-K partials plus one int32 ticket per (sequence, kv head)),
  * or 0 for an unsupported geometry.  Host only (reads cached device
- * attributes). */
+ * attributes).  The read path (scale folding at read time, "KVarN vs
+ * TurboQuant" (dothoosh.com), pipeline list, fourth stage) is split across
+ * the context because a long-context decode is bound by dragging the cache
+ * through HBM (HBM-math section of "Kompresja pamięci podręcznej KV to
+ * decyzja infrastrukturalna..." (encorp.ai)); these are the partial results
+ * of the splits. */
 size_t kvq_decode_workspace_bytes(const kvq_cache_desc* desc, int32_t batch, int32_t num_q_heads,
                                   int32_t max_seq_len);
 
@@ -203,7 +224,10 @@ int kvq_decode_attention_ex(const kvq_cache_desc* desc, const void* q, kvq_dtype
  * One kernel launch: the CTA whose split holds position L-1 writes the new
  * row before it reads that block.  The same arguments, workspace and status
  * rules as kvq_decode_attention; the new token's block must not be read by
- * another sequence of the same call.  Follows the KVarN write path (Hadamard
+ * another sequence of the same call.  A seq_lens[b] outside [0,
+ * max_seq_len] or beyond the table row appends nothing for that sequence
+ * (the pool is left as it was), truncates its read as kvq_decode_attention
+ * does and records KVQ_ERR_OUT_OF_RANGE.  Follows the KVarN write path (Hadamard
  * rotation, variance normalisation, asymmetric RTN) and read path (scale
  * folding at read time) of "KVarN vs TurboQuant" (dothoosh.com). */
 int kvq_append_decode_attention(const kvq_cache_desc* desc, const void* k_new, const void* v_new,
@@ -241,10 +265,26 @@ int kvq_decode_attention_noalloc(const kvq_cache_desc* desc, const void* q, kvq_
 /* Synchronise the stream, then read and clear the current device's status
  * word: KVQ_OK, or the first error that a kernel recorded since the last
  * read (KVQ_ERR_OUT_OF_RANGE, KVQ_ERR_DEVICE_TIMEOUT).  Returns
- * KVQ_ERR_CUDA if the synchronisation itself fails. */
+ * KVQ_ERR_CUDA if the synchronisation itself fails.  (The pages have no
+ * counterpart: this is how the kernels, which never trap, report bad block
+ * ids, slots and lengths and bounded waits that ran out.) */
 int kvq_last_device_status(void* stream);
 
-/* Static description of a status code; never NULL. */
+/* Failure-detection self-test (the pages have no counterpart).  Every
+ * device-side wait of the kernels is bounded: after a fixed number of polls
+ * (4194304, the largest value `polls` takes) it gives up and the kernel
+ * records KVQ_ERR_DEVICE_TIMEOUT in the device status word, without a trap,
+ * and returns with nothing of its own left in flight.  This call launches
+ * one warp that makes such a wait, with the same code, on a barrier that
+ * nothing ever arrives at, giving up after `polls` polls (1 .. 4194304), so
+ * that a test can watch the path run: kvq_last_device_status then returns
+ * KVQ_ERR_DEVICE_TIMEOUT and the context stays usable.  elapsed_ns (device
+ * memory, may be NULL) receives the time the polls took.  Asynchronous on
+ * the stream; KVQ_ERR_INVALID for polls out of range. */
+int kvq_selftest_wait_timeout(uint32_t polls, uint64_t* elapsed_ns, void* stream);
+
+/* Static description of a status code; never NULL.  (The pages have no
+ * counterpart: error reporting of this library.) */
 const char* kvq_error_string(int status);
 
 #ifdef __cplusplus

@@ -17,7 +17,7 @@ def test_every_declared_symbol_is_exported(kvq):
 
 def test_parse_dtype(kvq):
     assert kvq.kvq_parse_dtype("kvarn_k4v2_g128") == (0, (4, 2, 128))
-    # the other presets built (SURVEY: the same kernels at other bit widths)
+    # the other presets built: the same kernels at other bit widths
     for kb, vb in ((4, 4), (2, 2), (8, 4)):
         assert kvq.kvq_parse_dtype(f"kvarn_k{kb}v{vb}_g128") == (0, (kb, vb, 128))
     # well formed but not built: other widths, other groups
@@ -133,10 +133,15 @@ def test_fused_and_noalloc_argument_checks_need_no_device(kvq):
     assert fused(k_new, v_new, kvq.KVQ_BF16, 256, 1) == kvq.KVQ_ERR_WORKSPACE
     # an empty batch launches nothing
     assert fused(None, None, kvq.KVQ_BF16, 256, 0) == kvq.KVQ_OK
-    # no-allocation entry point: an empty batch is a no-op, a bad head count is rejected
+    # no-allocation entry point: an empty batch is a no-op; a head count that
+    # the kv heads do not divide gets the same code as from kvq_decode_attention
     assert L.kvq_decode_attention_noalloc(ctypes.byref(d), one, kvq.KVQ_BF16, 0, 16, one, 1, one, 16, 0.0, one,
                                           kvq.KVQ_F32, None) == kvq.KVQ_OK
     assert L.kvq_decode_attention_noalloc(ctypes.byref(d), one, kvq.KVQ_BF16, 1, 15, one, 1, one, 16, 0.0, one,
+                                          kvq.KVQ_F32, None) == kvq.KVQ_ERR_UNSUPPORTED
+    assert L.kvq_decode_attention(ctypes.byref(d), one, kvq.KVQ_BF16, 1, 15, one, 1, one, 16, 0.0, one,
+                                  kvq.KVQ_F32, one, 1 << 20, None) == kvq.KVQ_ERR_UNSUPPORTED
+    assert L.kvq_decode_attention_noalloc(ctypes.byref(d), one, kvq.KVQ_BF16, -1, 16, one, 1, one, 16, 0.0, one,
                                           kvq.KVQ_F32, None) == kvq.KVQ_ERR_INVALID
 
 
@@ -186,3 +191,10 @@ def test_workspace_bytes(kvq):
     n1 = kvq.kvq_decode_workspace_bytes(1024, 8, 1, 64, 16384, blocks_per_split=1024)
     assert n1 == 256 + 64 * 1 * 132 * 4
     assert kvq.kvq_decode_workspace_bytes(1024, 8, 1, 60, 16384) == 0
+
+
+def test_selftest_rejects_poll_counts_out_of_range(kvq):
+    """Checked on the host, before anything is launched."""
+    L = kvq.lib()
+    assert L.kvq_selftest_wait_timeout(0, None, None) == kvq.KVQ_ERR_INVALID
+    assert L.kvq_selftest_wait_timeout((1 << 22) + 1, None, None) == kvq.KVQ_ERR_INVALID

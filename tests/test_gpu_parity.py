@@ -204,9 +204,9 @@ def test_decode_ragged_gqa8(kvq, cuda, bps):
 
 @pytest.mark.parametrize("bps", [1, 2])
 def test_decode_many_splits(kvq, cuda, bps):
-    """More splits than one thread-block cluster holds (clusters of 16 merge
-    through distributed shared memory, then across clusters through the
-    workspace), with empty splits and whole empty clusters."""
+    """Many splits per sequence (400 tokens in splits of one or two blocks:
+    more records than the merge takes in one batch of 16), empty splits of
+    a shorter sequence, and an empty sequence."""
     wl = synth.Workload("m", 3, 16, 2, 128, [400, 33, 0], 16, synth.BF16, 3, 10.0, 30.0, seed=23, extra_blocks=2)
     g, pool, _, _ = _oracle_pool(wl)
     q = wl.query()
@@ -301,6 +301,45 @@ def test_append_decode_matches_append_then_decode(kvq, cuda, case):
     for b in range(wl.batch):
         if wl.seq_lens[b] == 0:  # an empty sequence appends nothing and reads nothing
             assert not out2[b].any()
+
+
+def test_append_decode_with_bad_length_writes_nothing(kvq, cuda):
+    """A sequence length beyond max_seq_len (or the table row) is recorded as
+    out of range, its read is truncated, and the fused step appends nothing:
+    the pool bytes stay as they were (the write position would otherwise be
+    a clamped one, not seq_lens[b] - 1)."""
+    torch = _torch()
+    wl = synth.Workload("bl", 2, 16, 2, 128, [48, 40], 16, synth.BF16, 3, 10.0, 30.0, seed=26, extra_blocks=4)
+    g, pool, _, _ = _oracle_pool(wl)
+    msl = int(wl.seq_lens.max())
+    # sequence 0 claims 16 more tokens than max_seq_len (and than its row)
+    bad_lens = wl.seq_lens.copy()
+    bad_lens[0] = msl + 16
+    kn = wl.kv_rows(synth.TID_NEWK, 0, wl.batch)
+    vn = wl.kv_rows(synth.TID_NEWV, 0, wl.batch)
+    dpool = torch.from_numpy(pool.copy()).cuda()
+    out = torch.empty((wl.batch, wl.hq, 128), dtype=torch.float32, device="cuda")
+    ws = kvq.new_workspace(wl.num_blocks, wl.hkv, wl.batch, wl.hq, msl)
+    kvq.kvq_append_decode_attention(dpool, wl.num_blocks, wl.hkv, _dev_u16(kn, wl.dtype).reshape(wl.batch, -1),
+                                    _dev_u16(vn, wl.dtype).reshape(wl.batch, -1), _dev_u16(wl.query(), wl.dtype),
+                                    torch.from_numpy(wl.block_table).cuda(), torch.from_numpy(bad_lens).cuda(), msl,
+                                    out, ws)
+    assert kvq.kvq_last_device_status() == kvq.KVQ_ERR_OUT_OF_RANGE
+    after = dpool.cpu().numpy()
+    seg = lambda a: a.reshape(wl.num_blocks, wl.hkv, 1664)
+    # sequence 0's blocks are untouched; sequence 1 appended its new token at position 39
+    rows0 = wl.block_table[0][wl.block_table[0] >= 0]
+    assert np.array_equal(seg(after)[rows0], seg(pool)[rows0])
+    p1, o1 = divmod(int(wl.block_table[1][39 // 16]) * 16 + 39 % 16, 16)
+    changed = np.nonzero(np.any(seg(after) != seg(pool), axis=2))
+    assert set(changed[0].tolist()) <= {p1}
+    rep = helpers.QuantReport()
+    helpers.check_pool_tokens(rep, after, wl.num_blocks, wl.hkv, kn, vn, wl.dtype,
+                              np.array([-1, p1 * 16 + o1], np.int32), [1])
+    assert rep.ok(), rep
+    # the truncated read of sequence 0 (its 48 tokens) and the read of sequence 1 match the oracle
+    want = oracle.decode_attention(g, after, wl.query(), wl.dtype, wl.block_table, wl.seq_lens)
+    assert np.max(np.abs(out.cpu().numpy().astype(np.float64) - want)) <= helpers.ATTN_TOL
 
 
 def test_decode_workspace_is_reusable(kvq, cuda):

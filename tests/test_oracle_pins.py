@@ -104,6 +104,27 @@ def test_worked_example_d4(orc):
         assert np.array_equal(rh, np.array(g["rhat"], float))
 
 
+def test_meta_exact_and_quotients_hand_values(orc):
+    """The two checker helpers the parity rules rest on (the unrounded S, Z
+    and the unrounded quotients) against values worked by hand."""
+    g = golden("meta_quotients_d4.json")
+    a = g["case_a"]
+    assert np.array_equal(orc.rotate(np.array(a["x"], float)), np.array(a["r"], float))
+    s_ex, z_ex = orc.meta_exact(np.array(a["x"], float), a["bits"], normalize=False)
+    assert s_ex == a["s_exact"] and z_ex == a["z_exact"]
+    s_ex, z_ex = orc.meta_exact(np.array(a["x"], float), a["bits"], normalize=True)
+    assert math.isclose(s_ex, a["s_exact"], rel_tol=1e-14) and math.isclose(z_ex, a["z_exact"], rel_tol=1e-14)
+    # 2 bits: the same range over 3 steps
+    s2, z2 = orc.meta_exact(np.array(a["x"], float), 2, normalize=False)
+    assert s2 == 4.0 / 3.0 and z2 == 1.0
+    b = g["case_b"]
+    assert orc.f16_to_f64(b["S_bits"]) == 0.5 and orc.f16_to_f64(b["Z_bits"]) == -1.0
+    q = orc.quotients(np.array(b["r"], float), b["S_bits"], b["Z_bits"])
+    assert np.array_equal(q, np.array(b["quotients"], float))
+    # the codes of those quotients: ties to even (2.5 -> 2), clamped to 0..3
+    assert list(orc.codes_given_meta(np.array(b["r"], float), 2, b["S_bits"], b["Z_bits"])) == [0, 2, 2, 3]
+
+
 @pytest.mark.parametrize("bits", [4, 2, 8])
 @pytest.mark.parametrize("normalize", [False, True])
 def test_grid_exact_groups_are_recovered(orc, bits, normalize):
