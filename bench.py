@@ -374,37 +374,129 @@ def prefill_quantize_gbs(kvq, torch, dev, seed=0, seqs=16, tokens=16384, reps=10
     return {"us": ms * 1e3, "gbs": nbytes / (ms * 1e-3) / 1e9, "bytes": nbytes, "status": status}
 
 
-def preset_decode_gbs(kvq, torch, dev, preset, batch=32, context=8192, reps=10):
-    """Decode of batch x context tokens (64/8 heads) on a pool of the preset
-    larger than L2: random code bytes with fp16 factors 0.01 (the work does
-    not depend on the values); µs per launch and GB/s on packed bytes."""
-    wl = synth.mixed_decode(0, batch=batch, context=context)
-    seg = seg_bytes(preset)
-    pool = torch.empty(wl.num_blocks * wl.hkv * seg, dtype=torch.uint8, device=dev).random_(0, 256)
-    pool.view(wl.num_blocks * wl.hkv, seg)[:, seg - 128:].view(torch.float16).fill_(0.01)
-    q = torch.randn(wl.batch, wl.hq, 128, device=dev, dtype=torch.bfloat16)
+def seeded_pool(kvq, torch, dev, wl, preset=(4, 2)):
+    """A pool for workload wl filled from its seeded stream: the first
+    min(16384, total) tokens are quantized through the library and their
+    segments repeated over the rest of the pool (the same value distribution,
+    hence the same running-max behaviour, without generating gigabytes of
+    K/V on the host)."""
+    T0 = min(16384, wl.total_tokens)
+    nb0 = (T0 + 15) // 16
+    k = torch.from_numpy(wl.kv_rows(synth.TID_K, 0, T0).view(np.int16)).to(dev).view(torch.bfloat16)
+    v = torch.from_numpy(wl.kv_rows(synth.TID_V, 0, T0).view(np.int16)).to(dev).view(torch.bfloat16)
+    base = kvq.new_pool(nb0, wl.hkv, device=dev, preset=preset)
+    kvq.kvq_quantize_append(base, nb0, wl.hkv, k.reshape(T0, -1), v.reshape(T0, -1),
+                            torch.arange(T0, dtype=torch.int32, device=dev), preset=preset)
+    del k, v
+    pool = kvq.new_pool(wl.num_blocks, wl.hkv, device=dev, preset=preset)
+    seg = pool.view(wl.num_blocks, -1)
+    b0 = base.view(nb0, -1)
+    for s0 in range(0, wl.num_blocks, nb0):
+        n = min(nb0, wl.num_blocks - s0)
+        seg[s0:s0 + n].copy_(b0[:n])
+    del base
+    return pool
+
+
+def time_decode_workload(kvq, torch, dev, wl, preset=(4, 2), reps=10, fused=False):
+    """Decode launches (or, fused=True, the one-step append + decode launch
+    with each sequence's new token) on a seeded pool of workload wl; CUDA
+    events on the launching stream around `reps` launches after 3 warm-ups.
+    Every workload's pool is larger than L2 except where noted by the caller.
+    Returns µs per launch and GB/s on packed-cache bytes."""
+    pool = seeded_pool(kvq, torch, dev, wl, preset)
+    q = torch.from_numpy(wl.query().view(np.int16)).to(dev).view(torch.bfloat16)
     bt = torch.from_numpy(wl.block_table).to(dev)
     lens = torch.from_numpy(wl.seq_lens).to(dev)
-    out = torch.empty(wl.batch, wl.hq, 128, device=dev, dtype=torch.bfloat16)
-    ws = kvq.new_workspace(wl.num_blocks, wl.hkv, wl.batch, wl.hq, context, device=dev, preset=preset)
+    msl = int(wl.seq_lens.max())
+    out = torch.empty((wl.batch, wl.hq, 128), dtype=torch.bfloat16, device=dev)
+    ws = kvq.new_workspace(wl.num_blocks, wl.hkv, wl.batch, wl.hq, msl, device=dev, preset=preset)
+    if fused:
+        kn = torch.from_numpy(wl.kv_rows(synth.TID_NEWK, 0, wl.batch).view(np.int16)).to(dev).view(torch.bfloat16)
+        vn = torch.from_numpy(wl.kv_rows(synth.TID_NEWV, 0, wl.batch).view(np.int16)).to(dev).view(torch.bfloat16)
+        kn, vn = kn.reshape(wl.batch, -1), vn.reshape(wl.batch, -1)
 
     def launch():
-        kvq.kvq_decode_attention(pool, wl.num_blocks, wl.hkv, q, bt, lens, context, out, ws, preset=preset)
+        if fused:
+            kvq.kvq_append_decode_attention(pool, wl.num_blocks, wl.hkv, kn, vn, q, bt, lens, msl, out, ws,
+                                            preset=preset)
+        else:
+            kvq.kvq_decode_attention(pool, wl.num_blocks, wl.hkv, q, bt, lens, msl, out, ws, preset=preset)
 
     for _ in range(3):
         launch()
     torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
+    e0.record(s)
     for _ in range(reps):
         launch()
-    e1.record()
+    e1.record(s)
     torch.cuda.synchronize()
     us = e0.elapsed_time(e1) * 1e3 / reps
-    nbytes = batch * context * wl.hkv * seg // 16
+    nbytes = int(wl.seq_lens.astype(np.int64).sum()) * wl.hkv * seg_bytes(preset) // 16
     status = kvq.kvq_last_device_status()
     del pool, ws
-    return {"us": us, "gbs": nbytes / (us * 1e-6) / 1e9, "bytes": nbytes, "status": status}
+    peak = measured_peaks()[0]
+    gbs = nbytes / (us * 1e-6) / 1e9
+    return {"us": us, "bytes": nbytes, "gbs": gbs, "frac": gbs / peak, "frac_of_8000": gbs / 8000.0,
+            "query_tokens_per_s": wl.batch / (us * 1e-6),
+            "context_tokens_per_s": float(wl.seq_lens.astype(np.int64).sum()) / (us * 1e-6), "status": status}
+
+
+def preset_decode_gbs(kvq, torch, dev, preset, batch=32, context=8192, reps=10):
+    """Decode of batch x context tokens (64/8 heads) on a seeded pool of the
+    preset (larger than L2); µs per launch and GB/s on packed bytes."""
+    return time_decode_workload(kvq, torch, dev, synth.mixed_decode(0, batch=batch, context=context), preset, reps)
+
+
+def workload_suite(kvq, torch, dev, reps=10):
+    """The other decode workloads, each on its own seeded pool (all larger
+    than L2): batched ragged 32 x U[4096, 16384]; Llama-3.1-70B-shaped 8 x
+    131072; the mixed step (64 x 8192, the new token of every sequence
+    appended and read in one fused launch), plus its decode alone."""
+    res = {}
+    for key, wl, fused in (("batched_32x_u4096_16384", synth.batched(0), False),
+                           ("long_8x131072", synth.long_context(0), False),
+                           ("mixed_step_64x8192", synth.mixed_decode(0), True),
+                           ("mixed_decode_64x8192", synth.mixed_decode(0), False)):
+        r = time_decode_workload(kvq, torch, dev, wl, reps=reps, fused=fused)
+        r["launch"] = ("fused 1-token append + decode" if fused else "decode")
+        res[key] = r
+    return res
+
+
+def dense_error_sample(kvq, torch, dev, seed=0, kv_head=0):
+    """Max abs error of the GPU read path against unquantized attention on the
+    raw bf16 K/V (the oracle's dense attention in double), for the query heads
+    of one kv head of the Qwen3-32B-shaped layer: the error quantisation adds.
+    Reported, not gated (the pages give no number for it)."""
+    import oracle
+    wl = synth.qwen3_32b_layer(seed)
+    T = wl.total_tokens
+    k = wl.kv_rows(synth.TID_K, 0, T)
+    v = wl.kv_rows(synth.TID_V, 0, T)
+    kd = torch.from_numpy(k.view(np.int16)).to(dev).view(torch.bfloat16).reshape(T, -1)
+    vd = torch.from_numpy(v.view(np.int16)).to(dev).view(torch.bfloat16).reshape(T, -1)
+    pool = kvq.new_pool(wl.num_blocks, wl.hkv, device=dev)
+    kvq.kvq_quantize_append(pool, wl.num_blocks, wl.hkv, kd, vd, torch.from_numpy(wl.slots()).to(dev))
+    q = wl.query()
+    out = torch.empty((wl.batch, wl.hq, 128), dtype=torch.float32, device=dev)
+    ws = kvq.new_workspace(wl.num_blocks, wl.hkv, wl.batch, wl.hq, T, device=dev)
+    kvq.kvq_decode_attention(pool, wl.num_blocks, wl.hkv, torch.from_numpy(q.view(np.int16)).to(dev)
+                             .view(torch.bfloat16), torch.from_numpy(wl.block_table).to(dev),
+                             torch.from_numpy(wl.seq_lens).to(dev), T, out, ws)
+    got = out.cpu().numpy().astype(np.float64)
+    G = wl.hq // wl.hkv
+    # tokens in the order of the sequence (the slots follow it)
+    err, ref_max = 0.0, 0.0
+    for j in range(kv_head * G, (kv_head + 1) * G):
+        ref = oracle.attention_dense(k, v, wl.dtype, q[0, j], wl.dtype, wl.hq, j)
+        err = max(err, float(np.max(np.abs(got[0, j] - ref))))
+        ref_max = max(ref_max, float(np.max(np.abs(ref))))
+    del pool, ws, kd, vd
+    return {"max_abs_err": err, "max_abs_output": ref_max, "query_heads": G, "tokens": T,
+            "against": "unquantized attention in double on the raw bf16 K/V (oracle)", "gated": False}
 
 
 # --------------------------------------------------------------------------- CPU oracle
@@ -413,7 +505,12 @@ class OracleSample:
     """The oracle, as it stands, on a bounded sample of one step: the 1-token
     write plus the decode of one kv head (8 query heads over 16384 tokens) of
     one layer.  A step is 64 layers x 8 kv heads of such units.  The cache
-    state it reads is written by the oracle itself, once, untimed."""
+    state it reads is written by the oracle itself, once, untimed.
+
+    unit() runs one such unit on one thread.  unit_mt(n) runs n units at once
+    on n threads (the oracle's own std::thread split over (sequence, kv head)
+    pairs: the sample's one kv head is read by n batch rows), which is how
+    the oracle uses all the host's cores."""
 
     desc = ("oracle 1-token write + decode of 1 kv head (8 query heads x 16384 tokens) of 1 layer, single "
             "thread; one step = 64 layers x 8 kv heads of these units")
@@ -439,6 +536,24 @@ class OracleSample:
         o.decode_attention(self.g, self.pool, self.q, wl.dtype, wl.block_table, wl.seq_lens, nthreads=1)
         return time.perf_counter() - t0
 
+    def unit_mt(self, n: int) -> float:
+        """Seconds per unit when n units run at once on n threads."""
+        o, wl = self.oracle, self.wl
+        q = np.ascontiguousarray(np.repeat(self.q, n, axis=0))
+        bt = np.ascontiguousarray(np.repeat(wl.block_table, n, axis=0))
+        lens = np.ascontiguousarray(np.repeat(wl.seq_lens, n))
+        t0 = time.perf_counter()
+        assert o.quantize_append(self.g, self.pool, self.k[-1:], self.v[-1:], wl.dtype, self.slots[-1:]) == 0
+        o.decode_attention(self.g, self.pool, q, wl.dtype, bt, lens, nthreads=n)
+        return (time.perf_counter() - t0) / n
+
+
+def host_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
 
 # --------------------------------------------------------------------------- profile mode
 
@@ -462,20 +577,7 @@ def profile_decode(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     wl = PROFILE_WORKLOADS[args.profile]()
-    T0 = min(16384, wl.total_tokens)
-    nb0 = (T0 + 15) // 16
-    k = torch.from_numpy(wl.kv_rows(synth.TID_K, 0, T0).view(np.int16)).to(dev).view(torch.bfloat16)
-    v = torch.from_numpy(wl.kv_rows(synth.TID_V, 0, T0).view(np.int16)).to(dev).view(torch.bfloat16)
-    base = kvq.new_pool(nb0, wl.hkv, device=dev)
-    kvq.kvq_quantize_append(base, nb0, wl.hkv, k.reshape(T0, -1), v.reshape(T0, -1),
-                            torch.arange(T0, dtype=torch.int32, device=dev))
-    del k, v
-    pool = kvq.new_pool(wl.num_blocks, wl.hkv, device=dev)
-    seg = pool.view(wl.num_blocks, -1)
-    b0 = base.view(nb0, -1)
-    for s in range(0, wl.num_blocks, nb0):
-        n = min(nb0, wl.num_blocks - s)
-        seg[s:s + n].copy_(b0[:n])
+    pool = seeded_pool(kvq, torch, dev, wl)
     q = torch.from_numpy(wl.query().view(np.int16)).to(dev).view(torch.bfloat16)
     bt = torch.from_numpy(wl.block_table).to(dev)
     lens = torch.from_numpy(wl.seq_lens).to(dev)
@@ -514,20 +616,26 @@ def run_reference(args, world, rank):
         return 0
     units_per_step = QwenStep.layers * QwenStep.hkv
     sample = OracleSample()
+    n = host_threads()
     for _ in range(args.warmup):
-        sample.unit()
-    samples = [sample.unit() for _ in range(args.steps)]
+        sample.unit_mt(n)
+    samples = [sample.unit_mt(n) for _ in range(args.steps)]
     per_unit = sum(samples) / len(samples)
-    desc = sample.desc + f"; each timed step runs one unit, {args.steps} steps"
+    desc = (f"oracle 1-token write + decode of 1 kv head (8 query heads x 16384 tokens) of 1 layer per unit, "
+            f"{n} units at once on {n} threads; one step = 64 layers x 8 kv heads of these units; each timed "
+            f"step runs one such batch of units, {args.steps} steps")
     step_s = per_unit * units_per_step
     value = QwenStep.batch / step_s
+    single = 1.0 / (sample.unit() * units_per_step)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": "qwen3-32b-16k-64layers", "batch": 1, "num_q_heads": 64, "num_kv_heads": 8,
                        "head_dim": 128, "context": 16384, "layers": 64, "block_size": 16},
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": n, "kind": "oracle",
                              "sample": desc},
+            "cpu_baseline_single_thread": {"value": single, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                           "sample": sample.desc + "; one unit"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
     return 0
@@ -540,6 +648,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-suite", action="store_true",
+                    help="skip the other workloads (batched, long, mixed step), the presets and the error sample")
+    ap.add_argument("--clock-log", default=None, help="write the clock samples of the timed region here (CSV)")
     ap.add_argument("--profile", choices=sorted(PROFILE_WORKLOADS) + ["prefill-quantize"], default=None,
                     help="time decode launches alone on one workload, or the bulk quantize-append "
                          "(1 GPU; for ncu captures)")
@@ -580,7 +691,7 @@ def main():
         raise RuntimeError("device status set during warm-up")
 
     # timed region: K steps
-    with ClockSampler(local, device_uuid(torch, dev)) as clocks:
+    with ClockSampler(local, device_uuid(torch, dev), log_path=args.clock_log) as clocks:
         ms = time_replays(torch, g_step, args.steps, barrier)
     ms_max, tokens = aggregate(dist, ms, args.steps * stepper.tokens_per_step(), dev)
     value = tokens / (ms_max * 1e-3)
@@ -605,27 +716,37 @@ def main():
     e2e_ms_max, e2e_tokens = aggregate(dist, e2e_ms, args.steps * stepper.tokens_per_step(), dev)
 
     quant = prefill_quantize_gbs(kvq, torch, dev)
-    # every preset on the same shapes: decode of 32 x 8192 tokens and the
-    # prefill append of 4 x 16384 tokens (the default preset included, for
-    # comparison)
-    presets = {}
-    for pr in kvq.PRESETS:
-        dq = preset_decode_gbs(kvq, torch, dev, pr)
-        pq = prefill_quantize_gbs(kvq, torch, dev, seqs=4, reps=5, preset=pr)
-        presets[f"kvarn_k{pr[0]}v{pr[1]}_g128"] = {
-            "segment_bytes": seg_bytes(pr),
-            "decode_32x8192": {"us": dq["us"], "gbs": dq["gbs"], "frac": dq["gbs"] / measured_peaks()[0]},
-            "quantize_4x16384": {"us": pq["us"], "gbs": pq["gbs"], "frac": pq["gbs"] / measured_peaks()[0]},
-            "device_status": dq["status"] or pq["status"]}
+    presets, suite, dense = {}, None, None
+    if not args.no_suite:
+        # the other configurations, each on a seeded pool larger than L2
+        suite = workload_suite(kvq, torch, dev)
+        # every preset on the same shapes: decode of 32 x 8192 tokens on a
+        # seeded pool and the prefill append of 4 x 16384 tokens (the default
+        # preset included, for comparison)
+        for pr in kvq.PRESETS:
+            dq = preset_decode_gbs(kvq, torch, dev, pr)
+            pq = prefill_quantize_gbs(kvq, torch, dev, seqs=4, reps=5, preset=pr)
+            presets[f"kvarn_k{pr[0]}v{pr[1]}_g128"] = {
+                "segment_bytes": seg_bytes(pr),
+                "decode_32x8192": {"us": dq["us"], "gbs": dq["gbs"], "frac": dq["frac"]},
+                "quantize_4x16384": {"us": pq["us"], "gbs": pq["gbs"], "frac": pq["gbs"] / measured_peaks()[0]},
+                "device_status": dq["status"] or pq["status"]}
+        if rank == 0:
+            dense = dense_error_sample(kvq, torch, dev)
     status = kvq.kvq_last_device_status()
 
-    cpu = None
+    cpu = cpu_mt = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         sample = OracleSample()
         per_unit = sum(sample.unit() for _ in range(3)) / 3
         cpu_value = 1.0 / (per_unit * stepper.layers * stepper.hkv)
         cpu = {"value": cpu_value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                "sample": sample.desc + "; mean of 3 units"}
+        n = host_threads()
+        per_unit_mt = sample.unit_mt(n)
+        cpu_mt = {"value": 1.0 / (per_unit_mt * stepper.layers * stepper.hkv), "unit": "tokens/s", "cores": n,
+                  "kind": "oracle",
+                  "sample": f"{n} such units at once on {n} threads (the oracle's std::thread split), one run"}
 
     if rank == 0:
         line = {
@@ -635,6 +756,7 @@ def main():
             "config": {"workload": "qwen3-32b-16k-64layers", "batch": 1, "num_q_heads": 64, "num_kv_heads": 8,
                        "head_dim": 128, "context": 16384, "layers": 64, "block_size": 16,
                        "cache": "kvarn_k4v2_g128", "step": "per layer: one fused launch (1-token quantize-append + decode attention)",
+                       "q_dtype": "bf16", "kv_in_dtype": "bf16", "out_dtype": "bf16",
                        "l2": "inputs larger than L2: 64 distinct 13.6 MB pools (872 MB) per step",
                        "parallelism": f"replicas x{world}"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
@@ -648,6 +770,8 @@ def main():
             "quantize": {"workload": "prefill append 16 x 16384 tokens, 8 kv heads, bf16", "us": quant["us"],
                          "gbs": quant["gbs"], "bytes": quant["bytes"], "frac": quant["gbs"] / peak},
             "presets": presets,
+            "workloads": suite,
+            "error_vs_unquantized": dense,
             "e2e": {"value": e2e_tokens / (e2e_ms_max * 1e-3), "unit": "tokens/s",
                     "h2d_bytes_per_step": stepper.h_in.numel() * 2, "d2h_bytes_per_step": stepper.h_out.numel() * 2},
             "gpu_launches": stepper.launches_per_step() * args.steps,
@@ -656,6 +780,8 @@ def main():
         }
         if cpu:
             line["cpu_baseline"] = cpu
+        if cpu_mt:
+            line["cpu_baseline_mt"] = cpu_mt
         print(json.dumps(line))
     if dist:
         del g_step, g_dec

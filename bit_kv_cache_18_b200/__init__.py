@@ -242,10 +242,11 @@ def kvq_decode_attention_noalloc(pool, num_blocks, num_kv_heads, q, block_table,
     _check(rc, "kvq_decode_attention_noalloc")
 
 
-def kvq_selftest_wait_timeout(polls: int, elapsed_ns=None, stream=None):
+def kvq_selftest_wait_timeout(limit_us: int, elapsed_ns=None, stream=None):
     """Launch the bounded-wait self-test (a wait that must give up after
-    `polls` polls); elapsed_ns: optional int64 device tensor of one element."""
-    rc = lib().kvq_selftest_wait_timeout(polls, _ptr(elapsed_ns), _stream_ptr(stream))
+    limit_us microseconds); elapsed_ns: optional int64 device tensor of one
+    element."""
+    rc = lib().kvq_selftest_wait_timeout(limit_us, _ptr(elapsed_ns), _stream_ptr(stream))
     _check(rc, "kvq_selftest_wait_timeout")
 
 

@@ -103,7 +103,7 @@ constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColA = 0;    // key codes of chunk c: kColA + 32 (c % 3)
 constexpr uint32_t kColS = 96;   // S of chunk c: kColS + 32 (c % 2)
 constexpr uint32_t kColO = 160;  // O accumulators: kColO + 32 k, k = 0, 1
-constexpr uint32_t kWaitLimit = 1u << 22;
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // a device-side wait gives up after one second
 constexpr int kBarSoftSync = 1;  // named barrier of the 128 softmax threads
 constexpr int kBarSoftVote = 2;  // named barrier for their vote
 
@@ -205,17 +205,28 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return done != 0;
 }
-// Bounded, warp-uniform wait for a barrier phase.  False if it never came
-// within `limit` polls or another warp already gave up (then every later
-// wait returns at once and the kernel runs to its end on void data, which it
-// reports; the loaders stop issuing copies and wait for those in flight
-// before the CTA exits).  The slow loop is a call, one copy per preset
-// (kTag), which keeps the wait sites small.
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Bounded, warp-uniform wait for a barrier phase.  False if it did not come
+// within `limit_ns` nanoseconds (the global timer decides; a try_wait may
+// suspend the thread for a while, so a count of polls would bound nothing)
+// or another warp already gave up (then every later wait returns at once
+// and the kernel runs to its end on void data, which it reports; the loaders
+// stop issuing copies and wait for those in flight before the CTA exits).
+// The slow loop is a call, one copy per preset (kTag), which keeps the wait
+// sites small.
 template <int kTag>
-__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t limit) {
-  for (uint32_t it = 0; it < limit; ++it) {
+__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort, uint64_t limit_ns) {
+  const uint64_t t0 = global_ns();
+  for (uint32_t it = 1;; ++it) {
     if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
-    if ((it & 15u) == 15u && __any_sync(0xffffffffu, *abort != 0)) return false;
+    if ((it & 15u) == 0u) {
+      if (__any_sync(0xffffffffu, *abort != 0)) return false;
+      if (__any_sync(0xffffffffu, global_ns() - t0 > limit_ns)) break;
+    }
   }
   *abort = 1;
   return false;
@@ -223,7 +234,7 @@ __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, vola
 template <int kTag>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
-  return mbar_wait_slow<kTag>(bar, parity, abort, kWaitLimit);
+  return mbar_wait_slow<kTag>(bar, parity, abort, kWaitLimitNs);
 }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -449,9 +460,11 @@ __device__ __forceinline__ void KeyRaw<2>::spread(uint32_t (&w)[16]) const {
 // Bounded wait that ignores the abort flag: the issuer's last wait for its
 // own MMAs, so tensor memory is never released under a running MMA.
 __device__ __forceinline__ bool mbar_wait_final(uint64_t* bar, uint32_t parity) {
-  for (uint32_t it = 0; it < kWaitLimit; ++it)
+  const uint64_t t0 = global_ns();
+  for (uint32_t it = 1;; ++it) {
     if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
-  return false;
+    if ((it & 15u) == 0u && __any_sync(0xffffffffu, global_ns() - t0 > kWaitLimitNs)) return false;
+  }
 }
 // CTAs per SM the shared memory of a preset allows (two for k4v2 and k2v2).
 template <int KB, int VB>
@@ -1156,9 +1169,9 @@ cudaError_t launch_p(const DecodeArgs& a, cudaStream_t stream) {
 // Failure-detection self-test: one warp waits, through the decode kernel's
 // bounded wait (the same slow loop), on a barrier that nothing arrives at.
 // Nothing else is issued (no bulk copy, no MMA, no tensor memory), so
-// nothing is in flight when the wait gives up; the kernel records
-// KVQ_ERR_DEVICE_TIMEOUT and the time the `limit` polls took.
-__global__ void __launch_bounds__(32) wait_timeout_probe_kernel(int* status, uint32_t limit, uint64_t* elapsed_ns) {
+// nothing is in flight when the wait gives up after limit_ns; the kernel
+// records KVQ_ERR_DEVICE_TIMEOUT and the time the wait took.
+__global__ void __launch_bounds__(32) wait_timeout_probe_kernel(int* status, uint64_t limit_ns, uint64_t* elapsed_ns) {
   __shared__ uint64_t bar;
   __shared__ int abort_flag;
   const int lane = threadIdx.x;
@@ -1168,10 +1181,9 @@ __global__ void __launch_bounds__(32) wait_timeout_probe_kernel(int* status, uin
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncwarp();
-  uint64_t t0, t1;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
-  const bool ok = mbar_wait_slow<0>(&bar, 0u, &abort_flag, limit);
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t1));
+  const uint64_t t0 = global_ns();
+  const bool ok = mbar_wait_slow<0>(&bar, 0u, &abort_flag, limit_ns);
+  const uint64_t t1 = global_ns();
   if (lane == 0) {
     if (!ok) record_status(status, KVQ_ERR_DEVICE_TIMEOUT);
     if (elapsed_ns != nullptr) *elapsed_ns = t1 - t0;
@@ -1180,11 +1192,11 @@ __global__ void __launch_bounds__(32) wait_timeout_probe_kernel(int* status, uin
 
 }  // namespace
 
-cudaError_t launch_wait_probe(int* status, uint32_t limit, uint64_t* elapsed_ns, cudaStream_t stream) {
-  wait_timeout_probe_kernel<<<1, 32, 0, stream>>>(status, limit, elapsed_ns);
+cudaError_t launch_wait_probe(int* status, uint64_t limit_ns, uint64_t* elapsed_ns, cudaStream_t stream) {
+  wait_timeout_probe_kernel<<<1, 32, 0, stream>>>(status, limit_ns, elapsed_ns);
   return cudaGetLastError();
 }
-uint32_t wait_poll_limit() { return kWaitLimit; }
+uint64_t wait_limit_ns() { return kWaitLimitNs; }
 
 int decode_ctas_per_sm() {
   static int cached[64] = {};

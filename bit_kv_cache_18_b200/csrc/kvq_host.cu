@@ -428,11 +428,12 @@ int kvq_decode_attention_noalloc(const kvq_cache_desc* desc, const void* q, kvq_
                                  kStaticScratchBytes, 0, stream);
 }
 
-int kvq_selftest_wait_timeout(uint32_t polls, uint64_t* elapsed_ns, void* stream) {
-  if (polls == 0 || polls > wait_poll_limit()) return KVQ_ERR_INVALID;
+int kvq_selftest_wait_timeout(uint32_t limit_us, uint64_t* elapsed_ns, void* stream) {
+  if (limit_us == 0 || static_cast<uint64_t>(limit_us) * 1000u > wait_limit_ns()) return KVQ_ERR_INVALID;
   int* status = device_status_ptr();
   if (!status) return KVQ_ERR_CUDA;
-  return launch_wait_probe(status, polls, elapsed_ns, static_cast<cudaStream_t>(stream)) == cudaSuccess
+  return launch_wait_probe(status, static_cast<uint64_t>(limit_us) * 1000u, elapsed_ns,
+                           static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? KVQ_OK
              : KVQ_ERR_CUDA;
 }

@@ -270,10 +270,10 @@ struct DecodeArgs {
 };
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 
-// Failure-detection self-test (kvq_selftest_wait_timeout) and the polls a
-// kernel's bounded wait makes before it gives up.
-cudaError_t launch_wait_probe(int* status, uint32_t limit, uint64_t* elapsed_ns, cudaStream_t stream);
-uint32_t wait_poll_limit();
+// Failure-detection self-test (kvq_selftest_wait_timeout) and the time after
+// which a kernel's bounded wait gives up.
+cudaError_t launch_wait_probe(int* status, uint64_t limit_ns, uint64_t* elapsed_ns, cudaStream_t stream);
+uint64_t wait_limit_ns();
 
 // Split-K plan of a decode call on the current device.
 struct DecodePlan {

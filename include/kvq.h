@@ -271,17 +271,17 @@ int kvq_decode_attention_noalloc(const kvq_cache_desc* desc, const void* q, kvq_
 int kvq_last_device_status(void* stream);
 
 /* Failure-detection self-test (the pages have no counterpart).  Every
- * device-side wait of the kernels is bounded: after a fixed number of polls
- * (4194304, the largest value `polls` takes) it gives up and the kernel
+ * device-side wait of the kernels is bounded in time: after one second
+ * (1000000 us, the largest value limit_us takes) it gives up and the kernel
  * records KVQ_ERR_DEVICE_TIMEOUT in the device status word, without a trap,
  * and returns with nothing of its own left in flight.  This call launches
  * one warp that makes such a wait, with the same code, on a barrier that
- * nothing ever arrives at, giving up after `polls` polls (1 .. 4194304), so
- * that a test can watch the path run: kvq_last_device_status then returns
- * KVQ_ERR_DEVICE_TIMEOUT and the context stays usable.  elapsed_ns (device
- * memory, may be NULL) receives the time the polls took.  Asynchronous on
- * the stream; KVQ_ERR_INVALID for polls out of range. */
-int kvq_selftest_wait_timeout(uint32_t polls, uint64_t* elapsed_ns, void* stream);
+ * nothing ever arrives at, giving up after limit_us microseconds (1 ..
+ * 1000000), so that a test can watch the path run: kvq_last_device_status
+ * then returns KVQ_ERR_DEVICE_TIMEOUT and the context stays usable.
+ * elapsed_ns (device memory, may be NULL) receives the time the wait took.
+ * Asynchronous on the stream; KVQ_ERR_INVALID for limit_us out of range. */
+int kvq_selftest_wait_timeout(uint32_t limit_us, uint64_t* elapsed_ns, void* stream);
 
 /* Static description of a status code; never NULL.  (The pages have no
  * counterpart: error reporting of this library.) */

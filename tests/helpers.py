@@ -91,3 +91,72 @@ def check_pool_tokens(rep: QuantReport, gpu_pool: np.ndarray, num_blocks: int, h
             kc, Sk, Zk, vc, Sv, Zv = oracle.unpack_token(g, gpu_pool, p, o, h)
             check_vector(rep, to_f64(k_rows[t, h], in_dtype), preset[0], kc, Sk, Zk, f"t{t} h{h} K")
             check_vector(rep, to_f64(v_rows[t, h], in_dtype), preset[1], vc, Sv, Zv, f"t{t} h{h} V")
+
+
+# ---------------------------------------------------------------- full sizes
+
+def threads() -> int:
+    import os
+    return max(1, min(64, os.cpu_count() or 1))
+
+
+def oracle_append_threaded(g, pool: np.ndarray, k, v, in_dtype: int, slots, nthreads: int | None = None):
+    """oracle.quantize_append over token ranges on several threads (the
+    calls write disjoint slots of the same pool; ctypes releases the GIL)."""
+    from concurrent.futures import ThreadPoolExecutor
+    n = int(slots.size)
+    nt = nthreads or threads()
+    step = max(1024, -(-n // (4 * nt)))
+
+    def work(t0):
+        t1 = min(n, t0 + step)
+        rc = oracle.quantize_append(g, pool, np.ascontiguousarray(k[t0:t1]), np.ascontiguousarray(v[t0:t1]),
+                                    in_dtype, np.ascontiguousarray(slots[t0:t1]))
+        assert rc == 0, rc
+
+    with ThreadPoolExecutor(nt) as ex:
+        list(ex.map(work, range(0, n, step)))
+
+
+def _token_bytes(pool: np.ndarray, num_blocks: int, hkv: int, slots, preset):
+    """[n, hkv, bytes of one token-head] gathered from a pool: K row, V row
+    and the four fp16 factors of each (token, head)."""
+    kb, vb = preset
+    kr, vr = 16 * kb, 16 * vb
+    seg = 16 * (kr + vr) + 128
+    offk = 16 * kr
+    p = (slots // 16).astype(np.int64)
+    o = (slots % 16).astype(np.int64)
+    cols = [o[:, None] * kr + np.arange(kr)[None, :], offk + o[:, None] * vr + np.arange(vr)[None, :]]
+    for f in range(4):  # S_K, Z_K, S_V, Z_V
+        base = 16 * (kr + vr) + 32 * f
+        cols.append(base + 2 * o[:, None] + np.arange(2)[None, :])
+    cols = np.concatenate(cols, axis=1)                             # [n, bytes]
+    flat = pool.reshape(num_blocks, hkv, seg)
+    return flat[p[:, None, None], np.arange(hkv)[None, :, None], cols[:, None, :]]
+
+
+def compare_pools(rep: QuantReport, gpu_pool: np.ndarray, oracle_pool: np.ndarray, num_blocks: int, hkv: int,
+                  k_rows, v_rows, in_dtype: int, slots, tokens=None, preset=(4, 2), chunk=65536):
+    """Every (token, head) group of `tokens` (default: all with a slot): the
+    GPU-written bytes against the oracle-written ones; groups whose bytes
+    differ go through check_vector (near-tie and midpoint rules)."""
+    slots = np.asarray(slots)
+    tokens = np.arange(slots.size) if tokens is None else np.asarray(tokens)
+    tokens = tokens[slots[tokens] >= 0]
+    per = 2 * 128 + 0  # elements per token-head (K and V)
+    for c0 in range(0, tokens.size, chunk):
+        tk = tokens[c0:c0 + chunk]
+        a = _token_bytes(gpu_pool, num_blocks, hkv, slots[tk], preset)
+        b = _token_bytes(oracle_pool, num_blocks, hkv, slots[tk], preset)
+        diff = np.any(a != b, axis=2)
+        rep.vectors += 2 * diff.size
+        rep.elements += per * diff.size
+        for ti, h in zip(*np.nonzero(diff)):
+            t = int(tk[ti])
+            sub = QuantReport()
+            check_pool_tokens(sub, gpu_pool, num_blocks, hkv, k_rows, v_rows, in_dtype, slots, [t], heads=[int(h)],
+                              preset=preset)
+            rep.code_mismatches += sub.code_mismatches
+            rep.meta_mismatch_groups += sub.meta_mismatch_groups
+            rep.failures += sub.failures

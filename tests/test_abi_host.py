@@ -193,8 +193,8 @@ def test_workspace_bytes(kvq):
     assert kvq.kvq_decode_workspace_bytes(1024, 8, 1, 60, 16384) == 0
 
 
-def test_selftest_rejects_poll_counts_out_of_range(kvq):
-    """Checked on the host, before anything is launched."""
+def test_selftest_rejects_limits_out_of_range(kvq):
+    """Checked on the host, before anything is launched: 1 us .. 1 s."""
     L = kvq.lib()
     assert L.kvq_selftest_wait_timeout(0, None, None) == kvq.KVQ_ERR_INVALID
-    assert L.kvq_selftest_wait_timeout((1 << 22) + 1, None, None) == kvq.KVQ_ERR_INVALID
+    assert L.kvq_selftest_wait_timeout(1000001, None, None) == kvq.KVQ_ERR_INVALID

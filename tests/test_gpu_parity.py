@@ -402,75 +402,6 @@ def test_end_to_end_against_unquantized(kvq, cuda):
     assert math.isfinite(dense_err)
 
 
-# ------------------------------------------------------------------ full sizes
-
-def _full_size_decode(kvq, wl, sample_heads, sample_batches):
-    """Pool written by the GPU for every head, then the sampled kv heads'
-    segments replaced by oracle-written bytes; GPU decode in the default
-    (benchmarked) launch configuration; sampled outputs against the oracle."""
-    torch = _torch()
-    T = wl.total_tokens
-    k = wl.kv_rows(synth.TID_K, 0, T)
-    v = wl.kv_rows(synth.TID_V, 0, T)
-    slots = wl.slots()
-    pool = torch.zeros(wl.num_blocks * wl.hkv * 1664, dtype=torch.uint8, device="cuda")
-    kvq.kvq_quantize_append(pool, wl.num_blocks, wl.hkv, _dev_u16(k, wl.dtype).reshape(T, -1),
-                            _dev_u16(v, wl.dtype).reshape(T, -1), torch.from_numpy(slots).cuda())
-    assert kvq.kvq_last_device_status() == 0
-    # sampled write-path parity on the GPU-written pool
-    rng = np.random.default_rng(wl.seed)
-    host = pool.cpu().numpy()
-    rep = helpers.QuantReport()
-    helpers.check_pool_tokens(rep, host, wl.num_blocks, wl.hkv, k, v, wl.dtype, slots,
-                              rng.choice(T, 48, replace=False))
-    assert rep.ok(), rep
-    G = wl.hq // wl.hkv
-    q = wl.query()
-    seg = pool.view(wl.num_blocks, wl.hkv, 1664)
-    g1 = oracle.geom(num_blocks=wl.num_blocks, num_kv_heads=1)
-    opools = {}
-    for h in sample_heads:
-        op = oracle.new_pool(g1)
-        sel = np.zeros(T, bool)
-        for b in sample_batches:
-            off = int(wl.token_offsets[b])
-            sel[off:off + int(wl.seq_lens[b])] = True
-        idx = np.nonzero(sel)[0]
-        assert oracle.quantize_append(g1, op, np.ascontiguousarray(k[idx, h:h + 1]),
-                                      np.ascontiguousarray(v[idx, h:h + 1]), wl.dtype, slots[idx]) == 0
-        opools[h] = op
-        opv = torch.from_numpy(op.reshape(wl.num_blocks, 1664)).cuda()
-        used = torch.from_numpy(np.unique(slots[idx] // 16)).cuda().long()
-        seg[used, h] = opv[used]
-    msl = int(wl.seq_lens.max())
-    out = torch.empty((wl.batch, wl.hq, 128), dtype=torch.float32, device="cuda")
-    ws = kvq.new_workspace(wl.num_blocks, wl.hkv, wl.batch, wl.hq, msl)
-    kvq.kvq_decode_attention(pool, wl.num_blocks, wl.hkv, _dev_u16(q, wl.dtype), torch.from_numpy(wl.block_table)
-                             .cuda(), torch.from_numpy(wl.seq_lens).cuda(), msl, out, ws)
-    got = out.cpu().numpy().astype(np.float64)
-    assert kvq.kvq_last_device_status() == 0
-    worst = 0.0
-    for h in sample_heads:
-        for b in sample_batches:
-            qh = np.ascontiguousarray(q[b:b + 1, h * G:(h + 1) * G])
-            want = oracle.decode_attention(g1, opools[h], qh, wl.dtype, wl.block_table[b:b + 1],
-                                           wl.seq_lens[b:b + 1], nthreads=1)
-            worst = max(worst, float(np.max(np.abs(got[b, h * G:(h + 1) * G] - want[0]))))
-    print(f"\n{wl.name}: sampled decode max abs err {worst:.2e}")
-    assert worst <= helpers.ATTN_TOL
-    return worst
-
-
-def test_full_size_qwen3_32b_layer(kvq, cuda):
-    _full_size_decode(kvq, synth.qwen3_32b_layer(0), sample_heads=[0, 5], sample_batches=[0])
-
-
-def test_full_size_batched_ragged(kvq, cuda):
-    wl = synth.batched(0)
-    _full_size_decode(kvq, wl, sample_heads=[3], sample_batches=[int(np.argmax(wl.seq_lens)),
-                                                                int(np.argmin(wl.seq_lens))])
-
-
 def test_decode_ignores_garbage_in_unused_slots(kvq, cuda):
     """Rows past the end of a sequence hold whatever the pool held before
     (here 0xFF bytes: NaN scales and zero points); they must not leak in."""

@@ -399,3 +399,41 @@ def test_capacity_ratio_within_the_claim(orc):
     packed = orc.packed_bytes_per_token_head(128, 4, 2)
     assert packed == 104
     assert g["ratio_min"] <= 2 * 128 * 2 / packed <= g["ratio_max"]
+
+
+def test_pool_comparison_catches_a_planted_code_error(orc, syn):
+    """The full-size checker (tests/helpers.compare_pools) on two oracle-written
+    pools: identical pools pass; a code moved by two steps in the oracle's
+    copy (a planted mistake, not a near-tie) fails; a flipped S fails."""
+    import helpers
+    wl = syn.Workload("cmp", 2, 4, 2, 128, [40, 21], 16, syn.BF16, 3, 10.0, 30.0, seed=5)
+    T = wl.total_tokens
+    k = wl.kv_rows(syn.TID_K, 0, T)
+    v = wl.kv_rows(syn.TID_V, 0, T)
+    slots = wl.slots()
+    g = orc.geom(num_blocks=wl.num_blocks, num_kv_heads=wl.hkv)
+    a = orc.new_pool(g)
+    helpers.oracle_append_threaded(g, a, k, v, wl.dtype, slots, nthreads=3)
+    b = orc.new_pool(g)
+    assert orc.quantize_append(g, b, k, v, wl.dtype, slots) == 0
+    assert np.array_equal(a, b)
+    rep = helpers.QuantReport()
+    helpers.compare_pools(rep, a, b, wl.num_blocks, wl.hkv, k, v, wl.dtype, slots)
+    assert rep.ok() and rep.vectors == 2 * T * wl.hkv and rep.code_mismatches == 0
+    # plant: token 7, head 1, key element 10 moved by two codes
+    p_, o_ = divmod(int(slots[7]), 16)
+    kc, Sk, Zk, vc, Sv, Zv = orc.unpack_token(g, a, p_, o_, 1)
+    kc = kc.copy()
+    kc[10] = (int(kc[10]) + 2) % 16
+    bad = a.copy()
+    orc.pack_token(g, bad, p_, o_, 1, kc, Sk, Zk, vc, Sv, Zv)
+    rep = helpers.QuantReport()
+    helpers.compare_pools(rep, bad, b, wl.num_blocks, wl.hkv, k, v, wl.dtype, slots)
+    assert not rep.ok()
+    # plant: a scale off by 8 ulps
+    bad = a.copy()
+    kc, Sk, Zk, vc, Sv, Zv = orc.unpack_token(g, a, p_, o_, 0)
+    orc.pack_token(g, bad, p_, o_, 0, kc, Sk + 8, Zk, vc, Sv, Zv)
+    rep = helpers.QuantReport()
+    helpers.compare_pools(rep, bad, b, wl.num_blocks, wl.hkv, k, v, wl.dtype, slots)
+    assert not rep.ok()
