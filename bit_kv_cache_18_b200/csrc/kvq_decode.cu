@@ -61,8 +61,9 @@
 // then switch to the second integer accumulator, and the first is folded
 // into fp32 registers with the factor 2^(m_old - m_new) one chunk later,
 // when the PVs that ran into it are complete, so no warp waits for a PV.
-// The accumulator is also restarted every 128 chunks, which keeps every s32
-// sum below 2^31.
+// A split is at most 128 chunks (the block ids a CTA stages), which keeps
+// every s32 sum of an accumulator below 2^31 (128 chunks x 128 tokens x 255
+// x 255 < 2^31) without a restart.
 //
 // Code order.  The byte spreading permutes the 128 positions of a row (for
 // k4v2 keys: position 32j + 8m + 4h + b holds dim 32m + 8j + 2b + h; values:
@@ -86,10 +87,12 @@ constexpr int kMmaWarp = kLoadWarps + kSoftWarps;        // warp 8: tensor memor
 constexpr int kThreads = 32 * (kMmaWarp + 1);             // 288
 constexpr int kChunkBlocks = 8;
 constexpr int kChunkTokens = kChunkBlocks * kBlockSize;  // 128
-constexpr int kMaxSplits = 64;     // the plan never cuts a sequence finer
+constexpr int kMaxSplits = 256;    // the plan never cuts a sequence finer
+constexpr int kTblBlocks = 1024;   // block ids a CTA stages in shared memory: no split is longer
+// an integer accumulator of O takes at most this many chunks of u8 x u8 sums
+static_assert(kTblBlocks / 8 * 128 * 255 * 255 < 2147483647ll, "s32 sums of one split stay below 2^31");
 constexpr int kNS = 2;             // score buffers in tensor memory
 constexpr int kNV = 3;             // key-code buffers in tensor memory; value / P' / factor buffers in smem
-constexpr int kFlushChunks = 128;  // integer accumulator restarted at least this often
 constexpr float kFix = 536870912.0f;  // P'_int = rne(P' 2^29) < 2^32
 constexpr float kFixInv = 1.0f / 536870912.0f;
 constexpr float kTrigger = 2.9f;    // move the max when s + E > m + kTrigger
@@ -103,6 +106,7 @@ constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColA = 0;    // key codes of chunk c: kColA + 32 (c % 3)
 constexpr uint32_t kColS = 96;   // S of chunk c: kColS + 32 (c % 2)
 constexpr uint32_t kColO = 160;  // O accumulators: kColO + 32 k, k = 0, 1
+constexpr uint32_t kColAcc = 224;  // per value position (lane): o~ so far in fp32, column g for head g
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // a device-side wait gives up after one second
 constexpr int kBarSoftSync = 1;  // named barrier of the 128 softmax threads
 constexpr int kBarSoftVote = 2;  // named barrier for their vote
@@ -131,6 +135,8 @@ struct __align__(1024) Smem {
     uint8_t stg[kLoadWarps][kNV][2 * kSeg];  // loader warp w: its two segments of chunk c in slot c % 3
     float obuf[8][kHeadDim];                      // o~ (epilogue, after the scan)
   };
+  int32_t tbl[kTblBlocks];                   // the split's block ids, -1 where absent (outside the split,
+                                             // the sequence or the pool)
   float2 hq[8];                              // per head: sum(q~), max|q~|
   float red[kSoftWarps][8][2];               // cross-warp reductions
   float palpha[kSoftWarps][8];               // per softmax warp: factor of the pending O buffer
@@ -294,6 +300,11 @@ __device__ __forceinline__ void tmem_ld8(uint32_t addr, uint32_t (&r)[8]) {
                : "r"(addr)
                : "memory");
 }
+__device__ __forceinline__ void tmem_st8(uint32_t addr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(addr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -354,6 +365,27 @@ __device__ __forceinline__ void fwht_warp(float (&x)[4], int lane, float scale) 
   const float f = 0.088388347648318440550f * scale;
 #pragma unroll
   for (int k = 0; k < 4; ++k) x[k] *= f;
+}
+
+// The same transform of a 128-vector held with element 4 lane + k in x[k]:
+// strides 1 and 2 in registers, strides 4 .. 64 by shuffles (lane xor
+// stride / 4), then the 1/sqrt(128) factor.
+__device__ __forceinline__ void fwht_warp_blocked(float (&x)[4], int lane) {
+  const float y0 = x[0] + x[1], y1 = x[0] - x[1], y2 = x[2] + x[3], y3 = x[2] - x[3];
+  x[0] = y0 + y2;
+  x[1] = y1 + y3;
+  x[2] = y0 - y2;
+  x[3] = y1 - y3;
+#pragma unroll
+  for (int st = 1; st < 32; st <<= 1) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float o = __shfl_xor_sync(0xffffffffu, x[k], st);
+      x[k] = (lane & st) ? o - x[k] : x[k] + o;
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) x[k] *= 0.088388347648318440550f;
 }
 
 // Position of dim d in a spread key row of KB-bit codes (with 32m + 8j + 4h
@@ -497,14 +529,14 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
     if (lane == 0) {
 #pragma unroll
       for (int i = 0; i < kNV; ++i) {
-        mbar_init(&sm.kv_ready[i], 32 * kLoadWarps);
-        mbar_init(&sm.p_ready[i], 32 * kSoftWarps);
+        mbar_init(&sm.kv_ready[i], kLoadWarps);  // one elected lane per warp arrives
+        mbar_init(&sm.p_ready[i], kSoftWarps);
         mbar_init(&sm.pv_done[i], 1);
       }
 #pragma unroll
       for (int i = 0; i < kNS; ++i) {
         mbar_init(&sm.qk_done[i], 1);
-        mbar_init(&sm.s_free[i], 32 * kSoftWarps);
+        mbar_init(&sm.s_free[i], kSoftWarps);
       }
       mbar_init(&sm.fin, 1);
       sm.abort = 0;
@@ -537,18 +569,21 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
 
   // ---- the split: blocks [blk0, blk1) of sequence b, in chunks of 8 -------
   // Loader warp w owns blocks 2w and 2w+1 of every chunk (tokens 32w ..
-  // 32w + 31 = TMEM lanes of its quarter); its lanes read the block ids of
-  // segment lane & 1 of chunks 0 .. 8 at once, before the sequence length
-  // is known (every entry of the row is in bounds), and cut them to the
-  // split below.
+  // 32w + 31 = TMEM lanes of its quarter).  Before the sequence length is
+  // known (every entry read is inside the table row), lanes 0 and 1 read the
+  // block ids of their segment of chunks 0 .. 2; the split's whole slice of
+  // the row goes to shared memory in the set-up below, cut to the split and
+  // the pool.
   const int blk0 = split * a.blocks_per_split;
   const int32_t* bt_row = a.block_table + static_cast<int64_t>(b) * a.max_blocks_per_seq;
-  int32_t braw[kNV + 6];
+  constexpr int kTblPer = kTblBlocks / (32 * kLoadWarps);
+  int32_t bfirst[kNV];  // loaders, lanes 0 and 1: block ids of chunks 0 .. 2
   if (is_loader) {
+    const int nload = min(a.blocks_per_split, a.max_blocks_per_seq - blk0);
 #pragma unroll
-    for (int i = 0; i < kNV + 6; ++i) {
-      const int blk = blk0 + kChunkBlocks * i + 2 * warp + (lane & 1);
-      braw[i] = blk < a.max_blocks_per_seq ? __ldg(bt_row + blk) : -1;
+    for (int i = 0; i < kNV; ++i) {
+      const int j = kChunkBlocks * i + 2 * warp + lane;
+      bfirst[i] = lane < 2 && j < nload ? __ldg(bt_row + blk0 + j) : -1;
     }
   }
   int L = a.seq_lens[b];
@@ -572,37 +607,21 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
   const int64_t pstride = static_cast<int64_t>(a.num_kv_heads) * kSeg;
   const int mseg = lane >> 4;  // segment of my factor bytes
 
-  // physical block of segment lane & 1 of my warp in chunk c (-1: none)
-  auto bid_of = [&](int c) -> int32_t {
-    const int blk = blk0 + kChunkBlocks * c + 2 * warp + (lane & 1);
-    return blk < blk1 ? __ldg(bt_row + blk) : -1;
-  };
-  auto prefetch_seg = [&](int32_t p) {
-    if (lane < 2 && p >= 0 && p < a.num_blocks) prefetch_l2(pool_h + static_cast<int64_t>(p) * pstride, kSeg);
-  };
   const uint32_t my_stg = smem_u32(sm.stg[warp < kLoadWarps ? warp : 0][0]);
-  // lanes 0 and 1: bulk copy of segment lane & 1 of chunk c (block p) into
-  // staging slot `slot`; every lane gets the pair of segment flags
-  // (bit s: segment s is inside the split and the pool)
-  auto issue = [&](int c, int32_t p, int slot) -> uint32_t {
-    const int blk = blk0 + kChunkBlocks * c + 2 * warp + (lane & 1);
-    const bool live = blk < blk1;
-    const bool ok = live && p >= 0 && p < a.num_blocks;
-    if (lane < 2) {
-      bad_blk |= live && !ok;
-      uint64_t* bar = &sm.full[warp][slot];
-      if (lane == 0) mbar_arrive_expect_tx(bar, a.num_blocks > 0 ? 2u * kSeg : 0u);
-      if (a.num_blocks > 0)  // (an empty pool has no block 0 to stand in)
-        bulk_g2s(my_stg + slot * (2 * kSeg) + lane * kSeg, pool_h + static_cast<int64_t>(ok ? p : 0) * pstride, kSeg,
-                 bar);
-    }
-    return __ballot_sync(0xffffffffu, ok && lane < 2) & 3u;
+  // Bulk copies of the loader warp's two segments of a chunk into staging
+  // slot `slot`: lanes 0 and 1 pass their segment's block id (-1: absent,
+  // nothing copied; the factors mark its tokens absent), every lane calls.
+  // The expected byte count is posted before any copy is issued.
+  auto issue = [&](int32_t p, int slot) {
+    uint64_t* bar = &sm.full[warp][slot];
+    const uint32_t okm = __ballot_sync(0xffffffffu, lane < 2 && p >= 0);
+    if (lane == 0) mbar_arrive_expect_tx(bar, static_cast<uint32_t>(__popc(okm)) * kSeg);
+    __syncwarp();
+    if (lane < 2 && p >= 0)
+      bulk_g2s(my_stg + slot * (2 * kSeg) + lane * kSeg, pool_h + static_cast<int64_t>(p) * pstride, kSeg, bar);
   };
 
   // ---- 0. set-up: barriers and tensor memory; first loads; query digits ----
-  int32_t bfirst[kNV];  // loaders: block ids of chunks 0 .. 2
-  int32_t bq[6];        // loaders: block ids of chunks c+3 .. c+8 at the start of iteration c
-  uint32_t okq[kNV] = {0u, 0u, 0u};  // loaders: segment flags of chunks c .. c+2
   // the chunk holding the block that the fused append writes is copied only
   // after the set-up barrier (-1: none)
   int c_defer = -1;
@@ -612,15 +631,13 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
   }
 
   if (is_loader) {
+    // my block ids of chunks 0 .. 2, cut to the split and the pool
+    const int nblk = blk1 - blk0;
 #pragma unroll
-    for (int i = 0; i < kNV; ++i) bfirst[i] = blk0 + kChunkBlocks * i + 2 * warp + (lane & 1) < blk1 ? braw[i] : -1;
-#pragma unroll
-    for (int i = 0; i < 6; ++i)
-      bq[i] = blk0 + kChunkBlocks * (kNV + i) + 2 * warp + (lane & 1) < blk1 ? braw[kNV + i] : -1;
-    // the split's block-table slice into L2: the ids of later chunks are
-    // read six chunks ahead of use, and a miss would stall the ring
-    for (int ln = tid; ln * 128 < (blk1 - blk0) * 4; ln += 32 * kLoadWarps)
-      prefetch_line_l2(reinterpret_cast<const char*>(bt_row + blk0) + ln * 128);
+    for (int i = 0; i < kNV; ++i) {
+      const int j = kChunkBlocks * i + 2 * warp + lane;
+      if (!(j < nblk && bfirst[i] >= 0 && bfirst[i] < a.num_blocks)) bfirst[i] = -1;
+    }
     // my staging ring's barriers, then the first three chunks' copies go out
     // while the query is rotated
     if (lane == 0) {
@@ -631,9 +648,19 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
     __syncwarp();
 #pragma unroll
     for (int i = 0; i < kNV; ++i)
-      if (i < nchunks && i != c_defer) okq[i] = issue(i, bfirst[i], i);
-#pragma unroll
-    for (int i = 0; i < 3; ++i) prefetch_seg(bq[i]);
+      if (i < nchunks && i != c_defer) issue(bfirst[i], i);
+    // the split's slice of the block table, cut to the split and the pool
+    // (an entry inside the sequence that names no block of the pool is
+    // recorded and its tokens skipped); the set-up barrier publishes it
+#pragma unroll 4
+    for (int i = 0; i < kTblPer; ++i) {
+      const int j = tid + 32 * kLoadWarps * i;
+      const bool inside = j < nblk;
+      const int32_t p = inside ? __ldg(bt_row + blk0 + j) : -1;
+      const bool okp = inside && p >= 0 && p < a.num_blocks;
+      bad_blk |= inside && !okp;
+      sm.tbl[j] = okp ? p : -1;
+    }
   } else if (is_soft) {
     const int sw = warp - kLoadWarps;
     const int stok = tid - 32 * kLoadWarps;
@@ -731,7 +758,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
     const uint32_t my_meta = smem_u32(&sm.meta[0][mkind][32 * warp + 16 * mseg + mrow0]);
 #pragma unroll
     for (int i = 0; i < kNV; ++i)  // the deferred chunk, if it is one of the first three
-      if (i == c_defer) okq[i] = issue(i, bfirst[i], i);
+      if (i == c_defer) issue(bfirst[i], i);
     Ring3 r{0, 0u};  // chunk c: staging slot, key-code, value and factor buffers r.i
     // staging slots whose bulk copy is still in flight after a failed wait:
     // bit i, and its phase parity in bit 4 + i
@@ -752,19 +779,19 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
         for (int i = 0; i < VB / 2; ++i) vr[sg][i] = lds128(sb + sg * kSeg + F::kOffV + 512 * i + 16 * lane);
       }
       const uint2 mr2 = lds64(sb + mseg * kSeg + F::kOffSK + 8 * (lane & 15));
-      const uint32_t ok = okq[0];
+      const bool seg_ok = sm.tbl[kChunkBlocks * c + 2 * warp + mseg] >= 0;  // my factor segment is present
       // the slot is read: refill it with chunk c+3 (the reads above are
-      // ordered before the copy's writes by the proxy fence)
+      // ordered before the copy's writes by the proxy fence); lanes 2 and 3
+      // prefetch their segments of chunk c+6 into L2.  (After a failed wait
+      // no copy is issued any more: see the drain below.)
       async_proxy_fence();
       __syncwarp();
-      okq[0] = okq[1];
-      okq[1] = okq[2];
-      // (after a failed wait no copy is issued any more: see the drain below)
-      okq[2] = c + kNV < nchunks && !bad ? issue(c + kNV, bq[0], r.i) : 0u;
-      prefetch_seg(bq[3]);
-#pragma unroll
-      for (int i = 0; i < 5; ++i) bq[i] = bq[i + 1];
-      bq[5] = bid_of(c + kNV + 6);
+      if (!bad) {
+        const int cc = c + kNV + kNV * (lane >> 1);
+        const int32_t p = lane < 4 && cc < nchunks ? sm.tbl[kChunkBlocks * cc + 2 * warp + (lane & 1)] : -1;
+        if (lane >= 2 && p >= 0) prefetch_l2(pool_h + static_cast<int64_t>(p) * pstride, kSeg);
+        if (c + kNV < nchunks) issue(lane < 2 ? p : -1, r.i);
+      }
 
       if (c >= kNV) {  // buffers r.i are free once PV(c-3) (issued after QK(c-2)) is done
         if (!mbar_wait<kWaitTag>(&sm.pv_done[r.i], r.ph ^ 1u, abort)) bad = true;
@@ -798,7 +825,6 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
       {  // factors of my four rows, as stored; S_V = -1 marks an absent token
          // (a segment outside the split or the pool, a row past the end of
          // the sequence: only in the block holding position L-1)
-        const bool seg_ok = ((ok >> mseg) & 1u) != 0;
         uint32_t m0 = seg_ok ? mr2.x : mnone, m1 = seg_ok ? mr2.y : mnone;
         const int blk = blk0 + kChunkBlocks * c + 2 * warp + mseg;
         if (blk == blk_last) {
@@ -813,7 +839,8 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
       tmem_wait_st();
       tc_fence_before();
       async_proxy_fence();
-      mbar_arrive(&sm.kv_ready[r.i]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.kv_ready[r.i]);
       r.next();
     }
     // Exit ordering after a wait gave up: this warp issued no copy since, and
@@ -873,12 +900,15 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
     const int stok = tid - 32 * kLoadWarps;
     const uint32_t my_lanes = tbase + (static_cast<uint32_t>(sw * 32) << 16);
     const uint32_t my_pm = smem_u32(sm.pm[0]) + (stok >> 3) * 256 + (stok & 7) * 16;
-    float qs[G], mr[G], lr[G], zr[G], oacc[G];  // oacc: in units of the output scale below
+    // (o~ so far, in units of the output scale below, lives in tensor memory
+    // at kColAcc: it is touched only when the running max moves and at the
+    // end, and registers are the scarce resource of this loop)
+    float qs[G], mr[G], lr[G], zr[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       qs[g] = sm.hq[g].x;
       mr[g] = kNoMax;
-      lr[g] = zr[g] = oacc[g] = 0.0f;
+      lr[g] = zr[g] = 0.0f;
     }
     int fresh_c = 0;  // the chunk whose PV started the integer accumulator
     int ob = 0;       // the O buffer the PVs of chunks fresh_c .. run into
@@ -888,12 +918,18 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
     // the PVs issued before it; nothing waits for a PV at the move.
     bool pend = false;  // (its per-head factor is in sm.palpha[sw], one copy per warp)
 
-    // fold O buffer k (my lane = value position stok) into oacc, with the
-    // pending factor of each head (scaled) or 1
+    {  // o~ so far: 0
+      const uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+      tmem_st8(my_lanes + kColAcc, z);
+      tmem_wait_st();
+    }
+    // fold O buffer k (my lane = value position stok) into o~ so far, with
+    // the pending factor of each head (scaled) or 1
     auto fold_o = [&](int k, bool scaled) {
-      uint32_t r[16], r2[16];
+      uint32_t r[16], r2[16], oa[8];
       tmem_ld16(my_lanes + kColO + 32 * k, r);
       tmem_ld16(my_lanes + kColO + 32 * k + 16, r2);
+      tmem_ld8(my_lanes + kColAcc, oa);
       tmem_wait_ld();
 #pragma unroll
       for (int g = 0; g < G; ++g) {
@@ -902,8 +938,11 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
                              fmaf(static_cast<float>(static_cast<int>(q[2])), 65536.0f,
                                   fmaf(static_cast<float>(static_cast<int>(q[1])), 256.0f,
                                        static_cast<float>(static_cast<int>(q[0])))));
-        oacc[g] = scaled ? fmaf(v, sm.palpha[sw][g], oacc[g]) : oacc[g] + v;
+        const float o = __uint_as_float(oa[g]);
+        oa[g] = __float_as_uint(scaled ? fmaf(v, sm.palpha[sw][g], o) : o + v);
       }
+      tmem_st8(my_lanes + kColAcc, oa);
+      tmem_wait_st();
     };
 
     Ring3 r{0, 0u};  // chunk c: buffers r.i
@@ -922,9 +961,14 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
       if (!mbar_wait<kWaitTag>(&sm.kv_ready[r.i], r.ph, abort)) bad = true;
       const uint32_t hsv = sm.meta[r.i][2][stok];
       const bool valid = (hsv & 0x8000u) == 0;  // a token (not marked absent by the loaders)
-      // S_K c1, Z_K, S_V 2^29, Z_V (0 for an absent token)
-      const float4 mt = make_float4(h2f(sm.meta[r.i][0][stok]) * c1, h2f(sm.meta[r.i][1][stok]), h2f(hsv) * kFix,
-                                    valid ? h2f(sm.meta[r.i][3][stok]) : 0.0f);
+      // S_K c1, Z_K, S_V 2^29, Z_V (0 for an absent token); a flat value row
+      // (S_V = 0: every code 0) takes 2^29 instead, so that its P' still
+      // stands for p (its codes add nothing to O, its p Z_V goes to zeta)
+      const float sv = h2f(hsv);
+      const float4 mt = make_float4(h2f(sm.meta[r.i][0][stok]) * c1, h2f(sm.meta[r.i][1][stok]),
+                                    (sv == 0.0f ? 1.0f : sv) * kFix, valid ? h2f(sm.meta[r.i][3][stok]) : 0.0f);
+      float pinv;  // 1 / (S_V 2^29)
+      asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(pinv) : "f"(mt.z));
       // E with S_V < 2^E, from the fp16 exponent of S_V (-14 for subnormals and 0)
       const float e = static_cast<float>(static_cast<int>((hsv >> 10) & 31u) - 14);
       tmem_wait_ld();
@@ -938,7 +982,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
         dmax = fmaxf(dmax, dg[g]);
       }
       const bool flag = valid && (dmax + e > kTrigger);
-      const bool any = soft_vote_any(flag) || c - fresh_c >= kFlushChunks;
+      const bool any = soft_vote_any(flag);
       if (any) {
         // rare: move the running max of each head to the chunk's max of
         // s + E plus the headroom; the scores are formed again from S (still
@@ -970,8 +1014,15 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
           dg[g] = sg[g] - mn;
           mr[g] = mn;
         }
+        {  // o~ so far in units of the new max
+          uint32_t oa[8];
+          tmem_ld8(my_lanes + kColAcc, oa);
+          tmem_wait_ld();
 #pragma unroll
-        for (int g = 0; g < G; ++g) oacc[g] *= alpha[g];
+          for (int g = 0; g < G; ++g) oa[g] = __float_as_uint(__uint_as_float(oa[g]) * alpha[g]);
+          tmem_st8(my_lanes + kColAcc, oa);
+          tmem_wait_st();
+        }
         if (c > fresh_c) {  // PVs of chunks fresh_c .. c-1 ran into buffer ob: pending
           if (lane == 0) {
 #pragma unroll
@@ -985,15 +1036,20 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
         // the reductions above read sm.red: none writes it again before the next vote
       }
       tc_fence_before();
-      mbar_arrive(&sm.s_free[P]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.s_free[P]);
       // P' of chunk c -> pm[r.i] (free: PV(c-3) was issued before QK(c), which is done)
       uint32_t pw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const float p = valid ? ex2(dg[g]) : 0.0f;
-        lr[g] += p;
-        zr[g] = fmaf(p, mt.w, zr[g]);
         pw[g] = __float2uint_rn(p * mt.z);  // rne(P' 2^29) < 2^32
+        // l and zeta take the p that the rounded P' stands for, so that a
+        // token enters the output as a whole or not at all (no bias from
+        // tokens whose P' rounds to zero)
+        const float pt = __uint2float_rn(pw[g]) * pinv;
+        lr[g] += pt;
+        zr[g] = fmaf(pt, mt.w, zr[g]);
       }
       const uint32_t pa = my_pm + r.i * (kChunkTokens * 32);
       sts128(pa, pw[0], pw[1], pw[2], pw[3]);
@@ -1001,7 +1057,8 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
       if (stok == 0) sm.fresh[r.i] = (fresh_c == c ? 1 : 0) | (ob << 1);
       async_proxy_fence();
       tc_fence_before();
-      mbar_arrive(&sm.p_ready[r.i]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.p_ready[r.i]);
       r.next();
     }
     if (nchunks > 0) {  // the last PV, then the accumulator
@@ -1030,48 +1087,57 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
     const int d = value_dim_of_pos<VB>(stok);
     // output scale of my value position: the fixed point and the factor of the spread
     const float oscale = kFixInv * __uint_as_float((127u - value_scale_log2<VB>(stok)) << 23);
+    // With several splits, every thread writes its dim of the split's record
+    // (o~[128], m, l per head) straight to the workspace; with one, the
+    // normalised o~ goes to shared memory for the output rotation.
+    float* rec = a.partials + ((static_cast<int64_t>(b) * a.num_q_heads + h * G) * a.nsplit + split) * kPartialFloats;
+    uint32_t oacc[8];
+    tmem_ld8(my_lanes + kColAcc, oacc);
+    tmem_wait_ld();
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       const float z = (sm.red[0][g][1] + sm.red[1][g][1]) + (sm.red[2][g][1] + sm.red[3][g][1]);
-      sm.obuf[g][d] = fmaf(oacc[g], oscale, z);
-      if (stok == g) {
-        sm.hl[g] = (sm.red[0][g][0] + sm.red[1][g][0]) + (sm.red[2][g][0] + sm.red[3][g][0]);
-        sm.hm[g] = mr[g];
+      const float lsum = (sm.red[0][g][0] + sm.red[1][g][0]) + (sm.red[2][g][0] + sm.red[3][g][0]);
+      const float o = fmaf(__uint_as_float(oacc[g]), oscale, z);
+      if (a.nsplit > 1) {
+        float* rg = rec + static_cast<int64_t>(g) * a.nsplit * kPartialFloats;
+        rg[d] = o;
+        if (stok == g) *reinterpret_cast<float2*>(rg + kHeadDim) = make_float2(mr[g], lsum);
+      } else {
+        sm.obuf[g][d] = lsum > 0.0f ? o / lsum : 0.0f;
       }
     }
   }
   if (bad) record_status(a.status, KVQ_ERR_DEVICE_TIMEOUT);
-  if (bad_blk && lane == 0) record_status(a.status, KVQ_ERR_OUT_OF_RANGE);
+  // (any loader thread may have met a bad entry of the block table)
+  if (__any_sync(0xffffffffu, bad_blk) && lane == 0) record_status(a.status, KVQ_ERR_OUT_OF_RANGE);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (warp == kMmaWarp)  // every MMA and tensor-memory load is complete
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "n"(kTmemCols));
   pdl_trigger();  // this CTA holds no tensor memory any more
-  __syncthreads();
 
-  // ---- 2. partial record, ticket, merge -------------------------------------
-  for (int t = tid; t < G * kHeadDim; t += kThreads) {
-    const int g = t / kHeadDim, d = t % kHeadDim;
-    const float lsum = sm.hl[g];
-    if (a.nsplit == 1) {
-      sm.obuf[g][d] = lsum > 0.0f ? sm.obuf[g][d] / lsum : 0.0f;
-    } else {
-      float* rec =
-          a.partials + ((static_cast<int64_t>(b) * a.num_q_heads + h * G + g) * a.nsplit + split) * kPartialFloats;
-      rec[d] = sm.obuf[g][d];
-      if (d == 0) {
-        rec[kHeadDim] = sm.hm[g];
-        rec[kHeadDim + 1] = lsum;
-      }
+  // ---- 2. output rotation (one split), or ticket and merge ----------------------
+  if (a.nsplit == 1) {
+    // rotate back once (warp w owns heads w, w + 9, ...) and store; the CTA
+    // barrier above published obuf
+    for (int g = warp; g < G; g += kThreads / 32) {
+      float x[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) x[k] = sm.obuf[g][lane + 32 * k];
+      fwht_warp(x, lane, 1.0f);
+      const int64_t o0 = (static_cast<int64_t>(b) * a.num_q_heads + h * G + g) * kHeadDim;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) store_from_f32(a.out, a.out_dtype, o0 + lane + 32 * k, x[k]);
     }
+    return;
   }
-  if (a.nsplit > 1) {
-    // ticket: one acquire-release add by thread 0 between two CTA barriers
+  {
+    // ticket: one acquire-release add by thread 0 after the CTA barrier above
     // publishes every thread's record stores (they happen before the add)
     // and, in the last CTA, makes every split's record visible to every
-    // thread's loads below
-    __syncthreads();
+    // thread's loads below (the barrier after the add)
     if (tid == 0) {
       int t;
       asm volatile("atom.add.acq_rel.gpu.global.s32 %0, [%1], 1;"
@@ -1127,22 +1193,16 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
         }
         M = Mb;
       }
+      // normalise and rotate back once, in the layout the merge left (lane l
+      // holds dims 4l .. 4l+3), and store
       const float inv = lsum > 0.0f ? 1.0f / lsum : 0.0f;
-      reinterpret_cast<float4*>(sm.obuf[g])[lane] = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+      float x[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
+      fwht_warp_blocked(x, lane);
+      const int64_t o0 = (static_cast<int64_t>(b) * a.num_q_heads + h * G + g) * kHeadDim + 4 * lane;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) store_from_f32(a.out, a.out_dtype, o0 + k, x[k]);
     }
     if (tid == 0) a.tickets[b * a.num_kv_heads + h] = 0;  // ready for the next call
-  }
-  __syncthreads();
-
-  // rotate back once (warp w owns heads w, w + 9, ...) and store
-  for (int g = warp; g < G; g += kThreads / 32) {
-    float x[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) x[k] = sm.obuf[g][lane + 32 * k];
-    fwht_warp(x, lane, 1.0f);
-    const int64_t o0 = (static_cast<int64_t>(b) * a.num_q_heads + h * G + g) * kHeadDim;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) store_from_f32(a.out, a.out_dtype, o0 + lane + 32 * k, x[k]);
   }
 }
 
@@ -1214,6 +1274,7 @@ int decode_ctas_per_sm() {
 }
 
 int decode_max_splits() { return kMaxSplits; }
+int decode_max_split_blocks() { return kTblBlocks; }
 int decode_chunk_blocks() { return kChunkBlocks; }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {

@@ -100,13 +100,9 @@ int device_sm_count() {
 // start-up worth about two chunks (the first loads, the query rotation, the
 // partial record), and every extra split adds a tenth of a chunk of merge
 // work.  Default splits are whole chunks.  A requested blocks_per_split is
-// raised if it would need more splits than the cap.  No split is longer
-// than kMaxSplitBlocks blocks unless the split cap forces it: the kernel's
-// fixed-point probabilities drop tokens more than about 2^30 below the
-// split's running max, a bias that grows with the tokens of one split (an
-// emulation of the arithmetic on a 131072-token sequence: 1.9e-3 in one
-// split, 2.5e-4 in splits of 2048 blocks, 1.1e-4 in splits of 512).
-constexpr int64_t kMaxSplitBlocks = 2048;
+// raised if it would need more splits than the cap, and lowered to
+// decode_max_split_blocks(), the block ids a CTA stages in shared memory;
+// a sequence longer than cap x that many blocks is not supported.
 
 int plan_decode(int32_t batch, int32_t num_kv_heads, int32_t num_q_heads, int32_t max_seq_len,
                 int32_t bps_request, DecodePlan* plan) {
@@ -115,7 +111,8 @@ int plan_decode(int32_t batch, int32_t num_kv_heads, int32_t num_q_heads, int32_
   const int64_t nb = (static_cast<int64_t>(max_seq_len) + kBlockSize - 1) / kBlockSize;
   const int64_t cap = decode_max_splits();
   const int64_t cb = decode_chunk_blocks();
-  const int64_t bmax = nb > kMaxSplitBlocks * cap ? (nb + cap - 1) / cap : kMaxSplitBlocks;
+  const int64_t bmax = decode_max_split_blocks();
+  if (nb > bmax * cap) return KVQ_ERR_UNSUPPORTED;
   int64_t bps = bps_request;
   if (nb == 0) {
     bps = 1;
@@ -140,7 +137,7 @@ int plan_decode(int32_t batch, int32_t num_kv_heads, int32_t num_q_heads, int32_
     }
   } else {
     if ((nb + bps - 1) / bps > cap) bps = (nb + cap - 1) / cap;
-    if (bps > bmax) bps = bmax;
+    if (bps > bmax) bps = bmax;  // (cap x bmax blocks cover the sequence)
   }
   const int64_t nsplit = nb > 0 ? (nb + bps - 1) / bps : 1;
   plan->blocks_per_split = static_cast<int32_t>(bps);

@@ -289,6 +289,7 @@ int plan_decode(int32_t batch, int32_t num_kv_heads, int32_t num_q_heads, int32_
 int device_sm_count();
 int decode_ctas_per_sm();  // resident decode CTAs per SM on the current device
 int decode_max_splits();   // upper bound the split plan respects
+int decode_max_split_blocks();  // longest split (blocks) a decode CTA takes
 int decode_chunk_blocks();  // blocks the decode kernel takes per step (splits are multiples of it)
 
 // Raise a kernel's dynamic shared-memory limit once per device (a host call

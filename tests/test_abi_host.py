@@ -168,21 +168,25 @@ def test_workspace_bytes_do_not_depend_on_the_preset(kvq, preset):
 
 
 def test_split_length_is_capped(kvq):
-    """A requested split longer than 2048 blocks (32768 tokens) is cut
-    further, unless 64 splits could not cover the sequence then; the
-    workspace holds one partial record per query head and split."""
+    """A decode CTA stages its split's block ids in shared memory, 1024 of
+    them: a requested split longer than 1024 blocks (16384 tokens) is cut
+    further; at most 256 splits, so a sequence beyond 256 x 1024 blocks is
+    not supported (the workspace query returns 0); the workspace holds one
+    partial record per query head and split."""
     rec = 64 * 132 * 4
-    assert kvq.kvq_decode_workspace_bytes(8192, 8, 1, 64, 131072, blocks_per_split=8192) == 256 + 4 * rec
-    assert kvq.kvq_decode_workspace_bytes(8192, 8, 1, 64, 131072, blocks_per_split=2048) == 256 + 4 * rec
+    assert kvq.kvq_decode_workspace_bytes(8192, 8, 1, 64, 131072, blocks_per_split=8192) == 256 + 8 * rec
     assert kvq.kvq_decode_workspace_bytes(8192, 8, 1, 64, 131072, blocks_per_split=1024) == 256 + 8 * rec
-    # 16549 tokens = 1035 blocks still fit in one split
-    assert kvq.kvq_decode_workspace_bytes(1035, 8, 1, 64, 16549, blocks_per_split=1035) == 256 + 1 * rec
-    # beyond 64 x 2048 blocks the split cap wins: 64 splits of ceil(blocks / 64)
-    big = 64 * 2048 * 16 + 80
-    assert kvq.kvq_decode_workspace_bytes(1, 8, 1, 64, big, blocks_per_split=100000) == 256 + 64 * rec
+    assert kvq.kvq_decode_workspace_bytes(8192, 8, 1, 64, 131072, blocks_per_split=512) == 256 + 16 * rec
+    # 16384 tokens = 1024 blocks still fit in one split; one block more does not
+    assert kvq.kvq_decode_workspace_bytes(1024, 8, 1, 64, 16384, blocks_per_split=1024) == 256 + 1 * rec
+    assert kvq.kvq_decode_workspace_bytes(1025, 8, 1, 64, 16400, blocks_per_split=1025) == 256 + 2 * rec
+    # too few splits requested: raised to what 256 splits of 1024 blocks allow
+    longest = 256 * 1024 * 16
+    assert kvq.kvq_decode_workspace_bytes(1, 8, 1, 64, longest, blocks_per_split=100000) == 256 + 256 * rec
+    assert kvq.kvq_decode_workspace_bytes(1, 8, 1, 64, longest + 16, blocks_per_split=0) == 0
     # the default plan obeys the same bound
     n_default = (kvq.kvq_decode_workspace_bytes(8192, 8, 1, 64, 131072) - 256) // rec
-    assert n_default >= 4
+    assert n_default >= 8
 
 
 def test_workspace_bytes(kvq):

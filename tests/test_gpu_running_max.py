@@ -7,7 +7,7 @@ sums run in an integer accumulator on the tensor cores, and a move switches
 to a second accumulator whose predecessor is folded one chunk later.  These
 tests build inputs whose scores rise steadily along the sequence, so that
 (nearly) every chunk of 128 tokens moves the max, and a split longer than
-the accumulator's restart interval.  Expected values come from the oracle's
+a split of the longest kind.  Expected values come from the oracle's
 plain softmax attention on the same packed bytes ("KVarN vs TurboQuant",
 dothoosh.com: scale folding at read time).
 """
@@ -73,10 +73,11 @@ def test_decode_rising_scores_slowly(kvq, cuda):
     _check_decode(wl, g, pool, q, wl.dtype, got)
 
 
-def test_decode_single_split_longer_than_accumulator_restart(kvq, cuda):
-    """One split of 130 chunks: the integer accumulator is restarted (folded
-    into fp32) after 128 chunks even without a max move."""
-    L = 129 * 128 + 37
+def test_decode_single_split_of_the_longest_kind(kvq, cuda):
+    """One split of 128 chunks (1024 blocks, the longest a CTA takes, less a
+    ragged tail): the integer accumulators run the whole split without a
+    restart and stay exact."""
+    L = 128 * 128 - 37
     wl = synth.Workload("long1", 1, 8, 1, 128, [L], 16, synth.F16, 2, 4.0, 8.0, seed=93)
     g = oracle.geom(num_blocks=wl.num_blocks, num_kv_heads=wl.hkv)
     pool = oracle.new_pool(g)

@@ -209,9 +209,8 @@ def test_full_size_long_context_sampled_pairs(kvq, cuda):
     """Llama-3.1-70B-shaped: batch 8 x 131072 tokens, 64/8 heads.  One kv head
     per sequence (head b of sequence b: eight distinct heads) holds oracle
     bytes; its 8 query heads (64 (b, j) pairs in all) are checked against the
-    oracle's plain attention, in the default split plan and with four splits
-    per sequence (256 chunks in one CTA, past the integer accumulator's
-    restart after 128)."""
+    oracle's plain attention, in the default split plan and with splits of
+    the longest kind (1024 blocks = 128 chunks per CTA, eight per sequence)."""
     torch = _torch()
     wl = synth.long_context(0)
     G = wl.hq // wl.hkv
@@ -229,7 +228,7 @@ def test_full_size_long_context_sampled_pairs(kvq, cuda):
 
     with ThreadPoolExecutor(min(len(sampled), helpers.threads())) as ex:
         wants = dict(zip(sampled, ex.map(want_of, sampled)))
-    for bps in (0, wl.max_blocks_per_seq // 4):
+    for bps in (0, 1024):
         got = _decode(kvq, wl, pool, q, bps=bps)
         assert np.all(np.isfinite(got))
         worst = max(float(np.max(np.abs(got[b, h * G:(h + 1) * G] - w))) for (b, h), w in wants.items())
