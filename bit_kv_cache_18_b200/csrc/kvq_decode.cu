@@ -330,6 +330,33 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, ui
   asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
+typedef unsigned long long u64x;
+__device__ __forceinline__ u64x pk2(float a, float b) {
+  u64x r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void upk2(u64x v, float& a, float& b) { asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v)); }
+__device__ __forceinline__ u64x add2(u64x a, u64x b) {
+  u64x d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ u64x mul2(u64x a, u64x b) {
+  u64x d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ u64x fma2(u64x a, u64x b, u64x c) {
+  u64x d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
 __device__ __forceinline__ float ex2(float x) {  // 2^x (MUFU.EX2); ex2(-inf) = 0
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -542,6 +569,45 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
       sm.abort = 0;
       asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
+  } else if (warp < kLoadWarps) {
+    // my staging ring's barriers (used by this warp only)
+    if (lane == 0) {
+#pragma unroll
+      for (int i = 0; i < kNV; ++i) mbar_init(&sm.full[warp][i], 1);
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncwarp();
+    // Before the dependency wait: L2 prefetches only.  Nothing read here is
+    // used for anything else (every real read comes after the wait, which
+    // orders it after the previous kernel's writes; a stale line prefetched
+    // now is updated in L2, the point of coherence, by any later write): the
+    // split's block-table slice, the sequence length and, by the block ids
+    // as they read now, the first three chunks' segments.
+    const int pblk0 = blockIdx.x * a.blocks_per_split;
+    const int pn = min(a.blocks_per_split, a.max_blocks_per_seq - pblk0);
+    const int32_t* prow = a.block_table + static_cast<int64_t>(blockIdx.z) * a.max_blocks_per_seq + pblk0;
+    for (int ln = tid; ln * 32 < pn; ln += 32 * kLoadWarps) prefetch_line_l2(prow + ln * 32);
+    if (tid == 0) prefetch_line_l2(a.seq_lens + blockIdx.z);
+    if (lane < 2 * kNV) {
+      const int blk = kChunkBlocks * (lane >> 1) + 2 * warp + (lane & 1);
+      if (blk < pn) {
+        int32_t p;
+        asm volatile("ld.global.cg.s32 %0, [%1];" : "=r"(p) : "l"(prow + blk));
+        if (p >= 0 && p < a.num_blocks)
+          prefetch_l2(a.pool + (static_cast<int64_t>(p) * a.num_kv_heads + blockIdx.y) * Fmt<KB, VB>::kSegBytes,
+                      Fmt<KB, VB>::kSegBytes);
+      }
+    }
+  } else {
+    // the query rows of this CTA's G heads (L2 prefetch, as above)
+    const int sw = warp - kLoadWarps;
+    const int esz = a.q_dtype == KVQ_F32 ? 4 : 2;  // a row is esz 128-byte lines
+    const int g = sw + 4 * (lane >> 2);
+    if (g < G && (lane & 3) < esz) {
+      const char* qrow = static_cast<const char*>(a.q) +
+                         ((static_cast<int64_t>(blockIdx.z) * a.num_q_heads + blockIdx.y * G + g) * kHeadDim) * esz;
+      prefetch_line_l2(qrow + 128 * (lane & 3));
+    }
   }
   pdl_wait();
 
@@ -638,14 +704,8 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
       const int j = kChunkBlocks * i + 2 * warp + lane;
       if (!(j < nblk && bfirst[i] >= 0 && bfirst[i] < a.num_blocks)) bfirst[i] = -1;
     }
-    // my staging ring's barriers, then the first three chunks' copies go out
-    // while the query is rotated
-    if (lane == 0) {
-#pragma unroll
-      for (int i = 0; i < kNV; ++i) mbar_init(&sm.full[warp][i], 1);
-      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    __syncwarp();
+    // the first three chunks' copies go out while the query is rotated (each
+    // warp set up its staging ring's barriers before the dependency wait)
 #pragma unroll
     for (int i = 0; i < kNV; ++i)
       if (i < nchunks && i != c_defer) issue(bfirst[i], i);
@@ -974,12 +1034,24 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
       tmem_wait_ld();
       float dg[G];
       float dmax = -CUDART_INF_F;
+      if (G == 1) {
+        const int e12 = static_cast<int>(sr[8]) * 254 + static_cast<int>(sr2[0]);
+        const float xg = fmaf(__int2float_rn(e12), 1.0f / 64516.0f, small_i2f(sr[0]));
+        dg[0] = fmaf(mt.x, xg, fmaf(mt.y, qs[0], -mr[0]));
+        dmax = dg[0];
+      } else {
+        const u64x mx2 = pk2(mt.x, mt.x), my2 = pk2(mt.y, mt.y);
+        const u64x k2 = pk2(1.0f / 64516.0f, 1.0f / 64516.0f), m2 = pk2(-12582912.0f, -12582912.0f);
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const int e12 = static_cast<int>(sr[8 + g]) * 254 + static_cast<int>(sr2[g]);
-        const float xg = fmaf(__int2float_rn(e12), 1.0f / 64516.0f, small_i2f(sr[g]));
-        dg[g] = fmaf(mt.x, xg, fmaf(mt.y, qs[g], -mr[g]));
-        dmax = fmaxf(dmax, dg[g]);
+        for (int g = 0; g < (G > 1 ? G : 2); g += 2) {
+          const float xe0 = __int2float_rn(static_cast<int>(sr[8 + g]) * 254 + static_cast<int>(sr2[g]));
+          const float xe1 = __int2float_rn(static_cast<int>(sr[9 + g]) * 254 + static_cast<int>(sr2[g + 1]));
+          const u64x s0 = add2(pk2(__uint_as_float(sr[g] + 0x4B400000u), __uint_as_float(sr[g + 1] + 0x4B400000u)), m2);
+          const u64x xg = fma2(pk2(xe0, xe1), k2, s0);
+          const u64x d = fma2(mx2, xg, fma2(my2, pk2(qs[g], qs[g + 1]), pk2(-mr[g], -mr[g + 1])));
+          upk2(d, dg[g], dg[g + 1]);
+          dmax = max3f(dmax, dg[g], dg[g + 1]);
+        }
       }
       const bool flag = valid && (dmax + e > kTrigger);
       const bool any = soft_vote_any(flag);
@@ -1040,16 +1112,27 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
       if (lane == 0) mbar_arrive(&sm.s_free[P]);
       // P' of chunk c -> pm[r.i] (free: PV(c-3) was issued before QK(c), which is done)
       uint32_t pw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+      if (G == 1) {
+        const float p = valid ? ex2(dg[0]) : 0.0f;
+        pw[0] = __float2uint_rn(p * mt.z);
+        const float pt = __uint2float_rn(pw[0]) * pinv;
+        lr[0] += pt;
+        zr[0] = fmaf(pt, mt.w, zr[0]);
+      } else {
+        const u64x z2 = pk2(mt.z, mt.z), i2 = pk2(pinv, pinv), w2 = pk2(mt.w, mt.w);
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float p = valid ? ex2(dg[g]) : 0.0f;
-        pw[g] = __float2uint_rn(p * mt.z);  // rne(P' 2^29) < 2^32
-        // l and zeta take the p that the rounded P' stands for, so that a
-        // token enters the output as a whole or not at all (no bias from
-        // tokens whose P' rounds to zero)
-        const float pt = __uint2float_rn(pw[g]) * pinv;
-        lr[g] += pt;
-        zr[g] = fmaf(pt, mt.w, zr[g]);
+        for (int g = 0; g < (G > 1 ? G : 2); g += 2) {
+          float x0, x1, t0, t1, l0, l1, q0, q1;
+          upk2(mul2(pk2(valid ? ex2(dg[g]) : 0.0f, valid ? ex2(dg[g + 1]) : 0.0f), z2), x0, x1);
+          pw[g] = __float2uint_rn(x0);  // rne(P' 2^29) < 2^32
+          pw[g + 1] = __float2uint_rn(x1);
+          // l and zeta take the p that the rounded P' stands for
+          const u64x pt = mul2(pk2(__uint2float_rn(pw[g]), __uint2float_rn(pw[g + 1])), i2);
+          upk2(add2(pk2(lr[g], lr[g + 1]), pt), l0, l1);
+          upk2(fma2(pt, w2, pk2(zr[g], zr[g + 1])), q0, q1);
+          lr[g] = l0; lr[g + 1] = l1; zr[g] = q0; zr[g + 1] = q1;
+          (void)t0; (void)t1;
+        }
       }
       const uint32_t pa = my_pm + r.i * (kChunkTokens * 32);
       sts128(pa, pw[0], pw[1], pw[2], pw[3]);

@@ -160,69 +160,67 @@ __device__ __forceinline__ void tmem_ld128(uint32_t addr, float (&v)[128]) {
 // ---- bulk path ------------------------------------------------------------------
 // A CTA of 128 threads walks tiles of 128 head vectors (one tensor, K or V);
 // thread t owns vector t of a tile and tensor-memory lane t.  Warp w stages
-// its 32 rows (vectors 32w .. 32w+31 of the tile) itself, two tiles ahead,
-// with coalesced 16-byte cp.async copies into a 272-byte-pitch ring; each
-// lane reads its row back (conflict free) and stores its 64 pairs of 16-bit
-// elements, unconverted, into its tensor-memory lane: the A operand.  The
-// rotation y = x H (H the 128 x 128 Sylvester Hadamard matrix,
-// unnormalised, exact in 16-bit floats) is then one tcgen05.mma chain
-// (M = 128 vectors, N = 128, K = 128 in 8 steps of 16; B = H in shared
-// memory) into 128 fp32 columns, which every thread reads back in one load
-// for the moments, range and codes of its vector.
+// its 32 rows (vectors 32w .. 32w+31 of the tile), two tiles ahead, with
+// coalesced 16-byte cp.async copies straight into the A operand of the
+// rotation: a 128-byte-swizzled K-major tile in shared memory (three such
+// tiles rotate: one being staged, one read by the tensor cores, one whose
+// staging is in flight).  The rotation y = x H (H the 128 x 128 Sylvester
+// Hadamard matrix, unnormalised, exact in 16-bit floats) runs on the tensor
+// cores into one of two 128-column fp32 accumulators, so that the MMAs of
+// tile i run while every thread computes the moments, range and codes of
+// its vector of tile i-1 from the other accumulator.  H is applied through
+// its Sylvester halves, H = [[H64, H64], [H64, -H64]]: with x = (x0, x1),
+// y0 = x0 H64 + x1 H64 and y1 = x0 H64 - x1 H64, sixteen MMAs of N = 64
+// (B = H64 and -H64, 16 KB of shared memory instead of 32).
 constexpr int kTileVecs = 128;
 constexpr int kBulkThreads = 128;
-constexpr int kWarpRows = 32;                     // rows a warp stages per tile
-constexpr int kPitch = kHeadDim * 2 + 16;         // 272-byte pitch of a 256-byte row
-constexpr int kStageBytes = kWarpRows * kPitch;   // 8.5 KB
-constexpr uint32_t kBulkTmemCols = 256;
-constexpr uint32_t kColD = 0;    // y: 128 fp32 columns
-constexpr uint32_t kColA = 128;  // x: 64 columns of 16-bit pairs
+constexpr int kWarpRows = 32;   // rows a warp stages per tile
+constexpr int kNA = 3;          // A tiles in shared memory
+constexpr uint32_t kBulkTmemCols = 256;  // two accumulators of 128 fp32 columns
+constexpr int kHalfBytes = kTileVecs * 128;  // one K-half (64 elements) of a tile: 128 rows of 128 B
 
-// B = H in the no-swizzle K-major layout of 8-row x 16-byte core matrices:
-// element (n, k) at (k/8)*2048 + n*16 + (k%8)*2 (leading, i.e. K, offset
-// 2048; stride offset 128).
+// Shared memory, every operand tile in the 128-byte-swizzled K-major layout
+// (8-row x 128-byte atoms, 16-byte chunk c of row r stored at chunk c ^ (r %
+// 8) of that row; atoms 1024 B apart along M):
+//   a[i][h]: elements 64h .. 64h+63 of the 128 rows of a tile
+//   hb[0] = H64, hb[1] = -H64 (row n = output column n, 64 elements)
 struct __align__(1024) BulkSmem {
-  uint8_t hm[kHeadDim * kHeadDim * 2];   // 32 KB
-  uint8_t stg[4][2][kStageBytes];        // warp w: its rows of tiles i (slot i % 2) and i+1
-  uint64_t mma_done;                     // the MMA chain of the tile is complete
+  uint8_t a[kNA][2][kHalfBytes];   // 96 KB
+  uint8_t hb[2][64 * 128];         // 16 KB
+  uint64_t mma_done[2];            // the MMAs into accumulator j are complete
   uint32_t tmem_base;
+  int abort;                       // a wait ran out: every other wait gives up at once
 };
 constexpr int kBulkSmemBytes = static_cast<int>(sizeof(BulkSmem));
 static_assert(kBulkSmemBytes <= 113 * 1024, "two CTAs per SM");
 // The tensor-memory rule of kvq_internal.cuh: three CTAs that allocate 256
-// columns each (this kernel's and the decode kernel's, whose shared memory
-// is larger) never fit on one SM's 228 KB.
+// columns each (this kernel's and the decode kernel's) never fit on one SM's
+// 228 KB.
 static_assert(3 * (kBulkSmemBytes + 1024) > 228 * 1024, "at most two tensor-memory CTAs per SM");
 
-// Instruction descriptor, kind::f16: D f32, A and B f16 or bf16, A in
-// tensor memory, B K-major, N = 128, M = 128.
-template <bool kBF16>
-__host__ __device__ constexpr uint32_t idesc_h() {
-  return (1u << 4) | ((kBF16 ? 1u : 0u) << 7) | ((kBF16 ? 1u : 0u) << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+// Byte offset of 16-byte chunk c of row r in a 128-byte-swizzled K-major
+// operand whose atoms start at 1024-byte boundaries.
+__device__ __forceinline__ uint32_t sw128(int r, int c) {
+  return static_cast<uint32_t>((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
 }
-__device__ __forceinline__ void mma_f16_ta(uint32_t d, uint32_t a, uint64_t bdesc, uint32_t idesc, bool acc) {
+// sm_100 shared-memory matrix descriptor of a 128-byte-swizzled K-major
+// operand: start address, stride offset 1024 B between 8-row atoms, version
+// 1, layout type 2 (128-byte swizzle).
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t addr) {
+  return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(1u) << 16) |
+         (static_cast<uint64_t>(1024u >> 4) << 32) | (1ull << 46) | (2ull << 61);
+}
+// Instruction descriptor, kind::f16: D f32, A and B f16 or bf16, both
+// K-major, N = 64, M = 128.
+template <bool kBF16>
+__host__ __device__ constexpr uint32_t idesc_h64() {
+  return (1u << 4) | ((kBF16 ? 1u : 0u) << 7) | ((kBF16 ? 1u : 0u) << 10) | ((64u >> 3) << 17) | ((128u >> 4) << 24);
+}
+__device__ __forceinline__ void mma_f16_ss(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, bool acc) {
   asm volatile(
       "{ .reg .pred p; setp.ne.b32 p, %3, 0;\n"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %4, p; }" ::"r"(d),
-      "r"(a), "l"(bdesc), "r"(static_cast<uint32_t>(acc)), "r"(idesc)
-      : "memory");
-}
-// 64 consecutive columns of this thread's lane from 64 registers.
-__device__ __forceinline__ void tmem_st64(uint32_t addr, const uint32_t (&r)[64]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], {"
-      "%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,"
-      "%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,"
-      "%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64};" ::"r"(addr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
-      "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
-      "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]),
-      "r"(r[32]), "r"(r[33]), "r"(r[34]), "r"(r[35]), "r"(r[36]), "r"(r[37]), "r"(r[38]), "r"(r[39]),
-      "r"(r[40]), "r"(r[41]), "r"(r[42]), "r"(r[43]), "r"(r[44]), "r"(r[45]), "r"(r[46]), "r"(r[47]),
-      "r"(r[48]), "r"(r[49]), "r"(r[50]), "r"(r[51]), "r"(r[52]), "r"(r[53]), "r"(r[54]), "r"(r[55]),
-      "r"(r[56]), "r"(r[57]), "r"(r[58]), "r"(r[59]), "r"(r[60]), "r"(r[61]), "r"(r[62]), "r"(r[63])
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %4, p; }" ::"r"(d),
+      "l"(adesc), "l"(bdesc), "r"(static_cast<uint32_t>(acc)), "r"(idesc)
       : "memory");
 }
 
@@ -232,26 +230,28 @@ __device__ __forceinline__ int64_t token_of(int64_t n, int64_t n_vec, int hkv) {
                                : n / hkv;
 }
 
-// Stage rows row0 .. row0+31 (vector n = token n / Hkv, head n % Hkv) into a
-// warp's slot: in copy j lane l moves 16-byte chunk l % 16 of row 2j + l/16
-// (two whole rows per instruction); the row addresses are computed once per
-// lane (its own row) and handed round by shuffles.  Rows past the tensor are
-// zero filled.
-__device__ __forceinline__ void stage_rows(uint32_t dst, const uint8_t* src, int64_t n_vec, int hkv,
-                                           int64_t stride_bytes, int64_t row0, int lane) {
+// Stage rows row0 .. row0+31 (vector n = token n / Hkv, head n % Hkv) into
+// rows 32w .. 32w+31 of an A tile (a0: its first K-half): in copy j lane l
+// moves 16-byte chunk l % 16 of row 2j + l/16 (two whole rows per
+// instruction, conflict free in the swizzled layout); the row addresses are
+// computed once per lane (its own row) and handed round by shuffles.  Rows
+// past the tensor are zero filled.
+__device__ __forceinline__ void stage_rows(uint32_t a0, const uint8_t* src, int64_t n_vec, int hkv,
+                                           int64_t stride_bytes, int64_t row0, int w, int lane) {
   const int64_t n = row0 + lane;
   const bool mine = n < n_vec;
   const int64_t tok = mine ? token_of(n, n_vec, hkv) : 0;
   const int hh = mine ? static_cast<int>(n - tok * hkv) : 0;
   const uint8_t* my_row = src + tok * stride_bytes + static_cast<int64_t>(hh) * (kHeadDim * 2);
+  const int col = lane & 15;
+  const uint32_t half = a0 + static_cast<uint32_t>(col >> 3) * kHalfBytes;
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
     const int row = 2 * j + (lane >> 4);
-    const int col = lane & 15;
     const uint8_t* row_ptr = reinterpret_cast<const uint8_t*>(
         __shfl_sync(0xffffffffu, static_cast<unsigned long long>(reinterpret_cast<uintptr_t>(my_row)), row));
     const bool valid = row0 + row < n_vec;
-    cp_async16(dst + row * kPitch + col * 16, valid ? row_ptr + col * 16 : src, valid);
+    cp_async16(half + sw128(32 * w + row, col & 7), valid ? row_ptr + col * 16 : src, valid);
   }
 }
 
@@ -382,6 +382,23 @@ __device__ __forceinline__ void quantize_lane(uint32_t taddr, float x0, uint8_t*
   reinterpret_cast<__half*>(seg + (kIsV ? F::kOffZV : F::kOffZK))[row_in_block] = Zh;
 }
 
+// Wait for a barrier phase, at most about a second, giving up at once once
+// another thread of the CTA has given up (false: it never came).
+__device__ __forceinline__ bool mbar_wait_ab(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (*abort) return false;
+      if (global_ns() - t0 > 1000000000ull) {
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
 template <bool kBF16, int KB, int VB>
 __global__ void __launch_bounds__(kBulkThreads, 2)
     quantize_kernel(uint8_t* __restrict__ pool, int32_t num_blocks, int32_t hkv,
@@ -389,11 +406,12 @@ __global__ void __launch_bounds__(kBulkThreads, 2)
                     int32_t n_tokens, int64_t stride_bytes, const int32_t* __restrict__ slots, int* status) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   BulkSmem& sm = *reinterpret_cast<BulkSmem*>(smem_raw);
+  volatile int* abort = &sm.abort;
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
 
-  // tensor memory, the barrier and H need no global memory: before the wait
+  // tensor memory, the barriers and H need no global memory: before the wait
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sm.tmem_base)),
                  "n"(kBulkTmemCols)
@@ -401,22 +419,25 @@ __global__ void __launch_bounds__(kBulkThreads, 2)
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   if (tid == 0) {
-    mbar_init(&sm.mma_done, 1);
+    mbar_init(&sm.mma_done[0], 1);
+    mbar_init(&sm.mma_done[1], 1);
+    sm.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  {  // H row n = tid: entry (n, k) = (-1)^popcount(n & k), as 16-bit +-1
+  {  // B: H64 (table 0) and -H64 (table 1); row n: entries (-1)^popcount(n & k), k < 64, as 16-bit +-1
     const uint32_t one = kBF16 ? 0x3F80u : 0x3C00u;
+    const int tb = tid >> 6, n = tid & 63;
 #pragma unroll
-    for (int c = 0; c < 16; ++c) {
+    for (int cc = 0; cc < 8; ++cc) {
       uint32_t w[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int k0 = 8 * c + 2 * e;
-        const uint32_t h0 = one | ((__popc(tid & k0) & 1u) << 15);
-        const uint32_t h1 = one | ((__popc(tid & (k0 + 1)) & 1u) << 15);
+        const int k0 = 8 * cc + 2 * e;
+        const uint32_t h0 = one | (((__popc(n & k0) + tb) & 1u) << 15);
+        const uint32_t h1 = one | (((__popc(n & (k0 + 1)) + tb) & 1u) << 15);
         w[e] = h0 | (h1 << 16);
       }
-      *reinterpret_cast<uint4*>(sm.hm + c * 2048 + tid * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+      *reinterpret_cast<uint4*>(sm.hb[tb] + sw128(n, cc)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
   }
   async_proxy_fence();  // (H is read by the tensor cores)
@@ -431,100 +452,122 @@ __global__ void __launch_bounds__(kBulkThreads, 2)
 
   const int64_t n_vec = static_cast<int64_t>(n_tokens) * hkv;
   const int64_t tiles_per_tensor = (n_vec + kTileVecs - 1) / kTileVecs;
-  const int64_t total_tiles = 2 * tiles_per_tensor;  // K tiles, then V tiles
+  // (the swizzle is a function of the shared address: the operand tiles must
+  // start on 1024-byte boundaries; never seen otherwise, checked all the same)
+  const bool aligned = (smem_u32(smem_raw) & 1023u) == 0;
+  if (!aligned && tid == 0) record_status(status, KVQ_ERR_UNSUPPORTED);
+  const int64_t total_tiles = aligned ? 2 * tiles_per_tensor : 0;  // K tiles, then V tiles
   const int64_t grid = gridDim.x;
-  const uint32_t hb = smem_u32(sm.hm);
-  const uint32_t my_stg = smem_u32(sm.stg[warp][0]);
-  // my warp's rows of tile t into slot `slot` (a group is committed even when
-  // there is nothing to copy, which keeps the counting uniform)
-  auto stage = [&](int64_t t, int slot) {
+  // my warp's rows of tile t into A buffer `buf` (a group is committed even
+  // when there is nothing to copy, which keeps the counting uniform)
+  auto stage = [&](int64_t t, int buf) {
     if (t < total_tiles) {
       const bool isv = t >= tiles_per_tensor;
-      stage_rows(my_stg + slot * kStageBytes, isv ? v : k, n_vec, hkv, stride_bytes,
-                 (isv ? t - tiles_per_tensor : t) * kTileVecs + kWarpRows * warp, lane);
+      stage_rows(smem_u32(sm.a[buf][0]), isv ? v : k, n_vec, hkv, stride_bytes,
+                 (isv ? t - tiles_per_tensor : t) * kTileVecs + kWarpRows * warp, warp, lane);
     }
     cp_async_commit();
   };
-  int64_t tile = blockIdx.x;
-  stage(tile, 0);
-  stage(tile + grid, 1);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tlane = sm.tmem_base + (static_cast<uint32_t>(32 * warp) << 16);  // my lane
-  bool bad = false;
-  uint32_t ph = 0;
-  int slot = 0;
-  for (; tile < total_tiles; tile += grid) {
-    // my vector and its slot (the load overlaps the copies and the MMAs)
+  const int64_t tile0 = blockIdx.x;
+  stage(tile0, 0);
+  stage(tile0 + grid, 1);
+  const uint32_t tbase = sm.tmem_base;
+  const uint32_t tlane = tbase + (static_cast<uint32_t>(32 * warp) << 16);  // my lane
+  uint32_t issued = 0;  // thread 0: MMA batches committed (batch k to mma_done[k & 1])
+
+  // my vector of the tile whose epilogue runs next: its slot, block row,
+  // head and tensor
+  int32_t e_slot = -1;
+  int e_head = 0;
+  bool e_isv = false;
+  // epilogue of tile kk (A buffer kk % 3, accumulator kk & 1)
+  auto epilogue = [&](int64_t kk, float x0) {
+    if (!mbar_wait_ab(&sm.mma_done[kk & 1], static_cast<uint32_t>((kk >> 1) & 1), abort)) return;
+    tc_fence_after();
+    uint8_t* seg = nullptr;
+    if (e_slot >= 0) {
+      const int32_t p = e_slot / kBlockSize;
+      if (p >= num_blocks)
+        record_status(status, KVQ_ERR_OUT_OF_RANGE);
+      else
+        seg = pool + (static_cast<int64_t>(p) * hkv + e_head) * Fmt<KB, VB>::kSegBytes;
+    }
+    const uint32_t dcol = tlane + 128u * static_cast<uint32_t>(kk & 1);
+    if (e_isv)  // (uniform over the tile)
+      quantize_lane<VB, true, Fmt<KB, VB>>(dcol, x0, seg, e_slot >= 0 ? e_slot % kBlockSize : 0);
+    else
+      quantize_lane<KB, false, Fmt<KB, VB>>(dcol, x0, seg, e_slot >= 0 ? e_slot % kBlockSize : 0);
+  };
+  auto first_elem = [&](int buf) -> float {  // element 0 of my row in A buffer buf
+    const uint16_t u = *reinterpret_cast<const uint16_t*>(sm.a[buf][0] + sw128(tid, 0));
+    return kBF16 ? __uint_as_float(static_cast<uint32_t>(u) << 16) : __half2float(__ushort_as_half(u));
+  };
+
+  int64_t kk = 0;  // tiles of this CTA walked so far
+  for (int64_t tile = tile0; tile < total_tiles; tile += grid, ++kk) {
+    // my vector of this tile: its slot load overlaps the copies and the MMAs
     const bool is_v = tile >= tiles_per_tensor;
     const int64_t n = (is_v ? tile - tiles_per_tensor : tile) * kTileVecs + tid;
     const int64_t tok = n < n_vec ? token_of(n, n_vec, hkv) : 0;
     const int32_t pslot = n < n_vec ? __ldg(slots + tok) : -1;
+    // element 0 of my row of the previous tile, read before its A buffer is
+    // staged again below (the barrier completes the read)
+    const float x0_prev = kk >= 1 ? first_elem(static_cast<int>((kk - 1) % kNA)) : 0.0f;
 
     cp_async_wait<1>();  // my copies of this tile are done
-    __syncwarp();
-    uint32_t x[64];      // my row: 64 pairs of 16-bit elements
-    {
-      const uint8_t* row = reinterpret_cast<const uint8_t*>(sm.stg[warp][slot]) + lane * kPitch;
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const uint4 q = *reinterpret_cast<const uint4*>(row + 16 * c);
-        x[4 * c] = q.x;
-        x[4 * c + 1] = q.y;
-        x[4 * c + 2] = q.z;
-        x[4 * c + 3] = q.w;
-      }
-    }
-    __syncwarp();           // the slot is read
-    stage(tile + 2 * grid, slot);
-    tmem_st64(tlane + kColA, x);  // (the previous chain, which read A, is complete)
-    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+    async_proxy_fence();  // (the tensor cores read them)
     tc_fence_before();
-    __syncthreads();  // A of every lane is written; y of the previous tile is read
+    __syncthreads();  // every row of this tile is in; the accumulator of tile kk-2 is read
     tc_fence_after();
-    if (tid == 0) {
+    if (tid == 0 && !*abort) {
+      // y0 = x0 H64 + x1 H64, y1 = x0 H64 - x1 H64 (N = 64 each, K in steps of 16)
+      const int ab = static_cast<int>(kk % kNA);
+      const uint32_t d = tbase + 128u * static_cast<uint32_t>(kk & 1);
+      const uint32_t a0 = smem_u32(sm.a[ab][0]), a1 = smem_u32(sm.a[ab][1]);
+      const uint32_t h0 = smem_u32(sm.hb[0]), h1 = smem_u32(sm.hb[1]);
+      constexpr uint32_t id = idesc_h64<kBF16>();
 #pragma unroll
-      for (int s = 0; s < kHeadDim / 16; ++s)
-        mma_f16_ta(sm.tmem_base + kColD, sm.tmem_base + kColA + 8 * s, sdesc(hb + 4096 * s, 2048, 128),
-                   idesc_h<kBF16>(), s > 0);
-      mma_commit(&sm.mma_done);
+      for (int st = 0; st < 4; ++st) mma_f16_ss(d, sdesc_sw128(a0 + 32 * st), sdesc_sw128(h0 + 32 * st), id, st > 0);
+#pragma unroll
+      for (int st = 0; st < 4; ++st) mma_f16_ss(d, sdesc_sw128(a1 + 32 * st), sdesc_sw128(h0 + 32 * st), id, true);
+#pragma unroll
+      for (int st = 0; st < 4; ++st)
+        mma_f16_ss(d + 64, sdesc_sw128(a0 + 32 * st), sdesc_sw128(h0 + 32 * st), id, st > 0);
+#pragma unroll
+      for (int st = 0; st < 4; ++st) mma_f16_ss(d + 64, sdesc_sw128(a1 + 32 * st), sdesc_sw128(h1 + 32 * st), id, true);
+      mma_commit(&sm.mma_done[kk & 1]);
+      ++issued;
     }
-    if (__syncthreads_or(!mbar_wait(&sm.mma_done, ph))) {  // (one decision for the CTA)
-      bad = true;
-      break;
+    if (kk >= 1) {
+      // tile kk-1: wait for its MMAs (then its A buffer is free for tile
+      // kk+2), stage tile kk+2 there, then its epilogue from its accumulator
+      epilogue(kk - 1, x0_prev);
+      stage(tile + 2 * grid, static_cast<int>((kk + 2) % kNA));
+    } else {
+      stage(tile + 2 * grid, 2);
     }
-    ph ^= 1u;
-    tc_fence_after();
-
-    // every thread reads its lane (warp-collective loads); vectors without a
-    // slot in the pool are not stored
-    uint8_t* seg = nullptr;
-    if (pslot >= 0) {
-      const int32_t p = pslot / kBlockSize;
-      if (p >= num_blocks)
-        record_status(status, KVQ_ERR_OUT_OF_RANGE);
-      else
-        seg = pool + (static_cast<int64_t>(p) * hkv + static_cast<int>(n - tok * hkv)) * Fmt<KB, VB>::kSegBytes;
-    }
-    const float x0 = kBF16 ? bf16lo_to_f32(x[0]) : __half2float(__ushort_as_half(static_cast<uint16_t>(x[0])));
-    if (is_v)  // (uniform over the tile)
-      quantize_lane<VB, true, Fmt<KB, VB>>(tlane + kColD, x0, seg, pslot >= 0 ? pslot % kBlockSize : 0);
-    else
-      quantize_lane<KB, false, Fmt<KB, VB>>(tlane + kColD, x0, seg, pslot >= 0 ? pslot % kBlockSize : 0);
     tc_fence_before();
-    slot ^= 1;
+    e_slot = pslot;
+    e_head = static_cast<int>(n - tok * hkv);
+    e_isv = is_v;
   }
+  if (kk >= 1) epilogue(kk - 1, first_elem(static_cast<int>((kk - 1) % kNA)));
   cp_async_wait<0>();
-  if (bad) {
-    record_status(status, KVQ_ERR_DEVICE_TIMEOUT);
-    mbar_wait(&sm.mma_done, ph);  // (tensor memory is released only once the chain is complete)
+  if (*abort) {
+    if (tid == 0) {
+      record_status(status, KVQ_ERR_DEVICE_TIMEOUT);
+      // tensor memory is released only once every MMA batch issued is complete
+      // (bounded waits that ignore the abort flag)
+      int zero = 0;
+      for (uint32_t j = issued >= 2 ? issued - 2 : 0; j < issued; ++j)
+        mbar_wait_ab(&sm.mma_done[j & 1], (j >> 1) & 1u, &zero);
+    }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (warp == 0)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(sm.tmem_base), "n"(kBulkTmemCols));
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "n"(kBulkTmemCols));
 }
 
 
