@@ -81,10 +81,21 @@
 namespace kvq {
 namespace {
 
-constexpr int kLoadWarps = 4;                          // warps 0-3
-constexpr int kSoftWarps = 4;                          // warps 4-7
-constexpr int kMmaWarp = kLoadWarps + kSoftWarps;        // warp 8: tensor memory owner, MMA issue
-constexpr int kThreads = 32 * (kMmaWarp + 1);             // 288
+// Warp roles.  The default kernel has 4 loader warps (two segments of a
+// chunk each), 4 softmax warps (one token each thread, all G heads) and the
+// MMA warp: 288 threads, two CTAs per SM.  The wide kernel, for grids that
+// fill the SMs once at one CTA per SM (small batches, where one CTA's chunk
+// latency bounds the whole call), doubles the loader and softmax warps: a
+// loader warp takes one segment, and two softmax threads share a token, four
+// heads each (G = 8).
+template <bool kWide>
+struct Roles {
+  static constexpr int kLoad = kWide ? 8 : 4;      // warps 0 .. kLoad-1
+  static constexpr int kSoft = kWide ? 8 : 4;      // warps kLoad .. kMma-1
+  static constexpr int kMma = kLoad + kSoft;       // tensor memory owner, MMA issue
+  static constexpr int kThreads = 32 * (kMma + 1);  // 288 or 544
+  static constexpr int kSegs = 8 / kLoad;          // segments a loader warp takes per chunk
+};
 constexpr int kChunkBlocks = 8;
 constexpr int kChunkTokens = kChunkBlocks * kBlockSize;  // 128
 constexpr int kMaxSplits = 256;    // the plan never cuts a sequence finer
@@ -108,7 +119,7 @@ constexpr uint32_t kColS = 96;   // S of chunk c: kColS + 32 (c % 2)
 constexpr uint32_t kColO = 160;  // O accumulators: kColO + 32 k, k = 0, 1
 constexpr uint32_t kColAcc = 224;  // per value position (lane): o~ so far in fp32, column g for head g
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // a device-side wait gives up after one second
-constexpr int kBarSoftSync = 1;  // named barrier of the 128 softmax threads
+constexpr int kBarSoftSync = 1;  // named barrier of the softmax threads
 constexpr int kBarSoftVote = 2;  // named barrier for their vote
 
 // Instruction descriptors (kind::i8, D = s32, M = 128, N = 32):
@@ -125,37 +136,37 @@ constexpr uint32_t kIdescPV =
 //   qb (B of QK, K-major):  byte (n, pos)   at (pos/16)*512 + (n/8)*128    + (n%8)*16   + pos%16
 // S column n = 8j + g holds digit j of head g (rows 24..31 of qb are zero);
 // P' and O column n = 4g + j hold byte j of head g.
-template <int kSeg>  // segment bytes of the preset
+template <int kSeg, bool kWide>  // segment bytes of the preset; the role layout
 struct __align__(1024) Smem {
+  using R = Roles<kWide>;
   uint8_t vt[kNV][kChunkTokens * kHeadDim];  // 3 x 16 KB
   uint8_t pm[kNV][kChunkTokens * 32];        // 3 x 4 KB
   uint8_t qb[32 * kHeadDim];                 // 4 KB
   uint16_t meta[kNV][4][kChunkTokens];       // per token, fp16 bits: S_K, Z_K, S_V (-1: segment absent), Z_V
   union {
-    uint8_t stg[kLoadWarps][kNV][2 * kSeg];  // loader warp w: its two segments of chunk c in slot c % 3
+    uint8_t stg[R::kLoad][kNV][R::kSegs * kSeg];  // loader warp w: its segments of chunk c in slot c % 3
     float obuf[8][kHeadDim];                      // o~ (epilogue, after the scan)
   };
   int32_t tbl[kTblBlocks];                   // the split's block ids, -1 where absent (outside the split,
                                              // the sequence or the pool)
   float2 hq[8];                              // per head: sum(q~), max|q~|
-  float red[kSoftWarps][8][2];               // cross-warp reductions
-  float palpha[kSoftWarps][8];               // per softmax warp: factor of the pending O buffer
-  float hm[8], hl[8];
+  float red[R::kSoft][8][2];                 // cross-warp reductions
+  float palpha[R::kSoft][8];                 // per softmax warp: factor of the pending O buffer
   float c1;                                  // max|q~| / 127: the unit of the query digits
   uint64_t kv_ready[kNV];  // loaders -> MMA warp, softmax: codes and factors of chunk c written
   uint64_t qk_done[kNS];   // QK(c) complete -> softmax: S of chunk c ready (and PV(c-3) complete)
   uint64_t s_free[kNS];    // softmax -> MMA warp: S of chunk c read
   uint64_t p_ready[kNV];   // softmax -> MMA warp: P' of chunk c written
   uint64_t pv_done[kNV];   // PV(c) complete -> loaders, softmax (and QK(c+1) complete)
-  uint64_t full[kLoadWarps][kNV];  // TMA -> loader warp w: segments of chunk c in slot c % 3
+  uint64_t full[R::kLoad][kNV];  // TMA -> loader warp w: segments of chunk c in slot c % 3
   uint64_t fin;            // every MMA issued is complete
   uint32_t tmem_base;
   int fresh[kNV];          // PV of chunk c: bit 0 starts the accumulator afresh, bit 1 its O buffer
   int is_last;
   int abort;              // a wait ran out: every other wait gives up at once
 };
-template <int kSeg>
-constexpr int kSmemBytesOf = static_cast<int>((sizeof(Smem<kSeg>) + 1023) / 1024 * 1024);
+template <int kSeg, bool kWide = false>
+constexpr int kSmemBytesOf = static_cast<int>((sizeof(Smem<kSeg, kWide>) + 1023) / 1024 * 1024);
 static_assert(kSmemBytesOf<Fmt<4, 2>::kSegBytes> <= 113 * 1024, "two CTAs per SM (k4v2)");
 static_assert(kSmemBytesOf<Fmt<2, 2>::kSegBytes> <= 113 * 1024, "two CTAs per SM (k2v2)");
 static_assert(kSmemBytesOf<Fmt<8, 4>::kSegBytes> <= 227 * 1024, "one CTA per SM (k8v4)");
@@ -245,13 +256,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void async_proxy_fence() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-__device__ __forceinline__ void soft_sync() { asm volatile("bar.sync %0, %1;" ::"n"(kBarSoftSync), "n"(128) : "memory"); }
+template <int kN>  // the softmax threads
+__device__ __forceinline__ void soft_sync() { asm volatile("bar.sync %0, %1;" ::"n"(kBarSoftSync), "n"(kN) : "memory"); }
+template <int kN>
 __device__ __forceinline__ bool soft_vote_any(bool x) {
   uint32_t r;
   asm volatile(
       "{ .reg .pred p, q; setp.ne.u32 p, %1, 0; bar.red.or.pred q, %2, %3, p; selp.u32 %0, 1, 0, q; }"
       : "=r"(r)
-      : "r"(static_cast<uint32_t>(x)), "n"(kBarSoftVote), "n"(128)
+      : "r"(static_cast<uint32_t>(x)), "n"(kBarSoftVote), "n"(kN)
       : "memory");
   return r != 0;
 }
@@ -529,13 +542,28 @@ __device__ __forceinline__ bool mbar_wait_final(uint64_t* bar, uint32_t parity) 
 template <int KB, int VB>
 constexpr int kMinCtasOf = kSmemBytesOf<Fmt<KB, VB>::kSegBytes> <= 113 * 1024 ? 2 : 1;
 
-template <int G, int KB, int VB>
-__global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(DecodeArgs a) {
+// Segment (block) s of a chunk of 8 that loader warp w takes as its sg-th:
+// TMEM lanes 16 s .. 16 s + 15 lie in the warp's lane quarter w % 4.
+template <bool kWide>
+__device__ __forceinline__ int seg_of(int w, int sg) {
+  return kWide ? 2 * (w & 3) + (w >> 2) : 2 * w + sg;
+}
+
+template <int G, int KB, int VB, bool kWide>
+__global__ void __launch_bounds__(Roles<kWide>::kThreads, kWide ? 1 : kMinCtasOf<KB, VB>)
+    decode_kernel(DecodeArgs a) {
   using F = Fmt<KB, VB>;
+  using R = Roles<kWide>;
+  constexpr int kLoadWarps = R::kLoad, kSoftWarps = R::kSoft, kMmaWarp = R::kMma, kThreads = R::kThreads;
+  constexpr int kSegs = R::kSegs;                  // segments per loader warp and chunk
+  constexpr int kSoftThreads = 32 * kSoftWarps;
+  constexpr int kHeads = kWide ? G / 2 : G;        // heads a softmax thread takes (the wide layout: two threads a token)
+  constexpr int kQHeads = 8 / kSoftWarps;          // query heads a softmax warp rotates at set-up (at most)
+  static_assert(!kWide || G == 8, "the wide layout splits 8 heads over two threads");
   constexpr int kSeg = F::kSegBytes;
-  constexpr int kWaitTag = 16 * KB + VB;
+  constexpr int kWaitTag = 16 * KB + VB + (kWide ? 256 : 0);
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  Smem<kSeg>& sm = *reinterpret_cast<Smem<kSeg>*>(smem_raw);
+  Smem<kSeg, kWide>& sm = *reinterpret_cast<Smem<kSeg, kWide>*>(smem_raw);
   volatile int* abort = &sm.abort;
   const int split = blockIdx.x;
   const int h = blockIdx.y;
@@ -588,8 +616,8 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
     const int32_t* prow = a.block_table + static_cast<int64_t>(blockIdx.z) * a.max_blocks_per_seq + pblk0;
     for (int ln = tid; ln * 32 < pn; ln += 32 * kLoadWarps) prefetch_line_l2(prow + ln * 32);
     if (tid == 0) prefetch_line_l2(a.seq_lens + blockIdx.z);
-    if (lane < 2 * kNV) {
-      const int blk = kChunkBlocks * (lane >> 1) + 2 * warp + (lane & 1);
+    if (lane < kSegs * kNV) {
+      const int blk = kChunkBlocks * (lane / kSegs) + seg_of<kWide>(warp, lane % kSegs);
       if (blk < pn) {
         int32_t p;
         asm volatile("ld.global.cg.s32 %0, [%1];" : "=r"(p) : "l"(prow + blk));
@@ -602,7 +630,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
     // the query rows of this CTA's G heads (L2 prefetch, as above)
     const int sw = warp - kLoadWarps;
     const int esz = a.q_dtype == KVQ_F32 ? 4 : 2;  // a row is esz 128-byte lines
-    const int g = sw + 4 * (lane >> 2);
+    const int g = sw + kSoftWarps * (lane >> 2);
     if (g < G && (lane & 3) < esz) {
       const char* qrow = static_cast<const char*>(a.q) +
                          ((static_cast<int64_t>(blockIdx.z) * a.num_q_heads + blockIdx.y * G + g) * kHeadDim) * esz;
@@ -612,15 +640,15 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
   pdl_wait();
 
   // The loads that need no sequence length go out first: softmax warp sw's
-  // query heads sw and sw + 4 and, in a fused step, the MMA warp's lanes' 8
-  // bytes of the new token's K and V rows.
-  float x[2][4];
+  // query heads sw, sw + kSoftWarps, ... and, in a fused step, the MMA
+  // warp's lanes' 8 bytes of the new token's K and V rows.
+  float x[kQHeads][4];
   uint2 new_k = make_uint2(0u, 0u), new_v = make_uint2(0u, 0u);
   if (is_soft) {
     const int sw = warp - kLoadWarps;
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int g = sw + 4 * i;
+    for (int i = 0; i < kQHeads; ++i) {
+      const int g = sw + kSoftWarps * i;
       if (g < G) {
         const int64_t q0 = (static_cast<int64_t>(b) * a.num_q_heads + h * G + g) * kHeadDim;
 #pragma unroll
@@ -634,22 +662,22 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
   }
 
   // ---- the split: blocks [blk0, blk1) of sequence b, in chunks of 8 -------
-  // Loader warp w owns blocks 2w and 2w+1 of every chunk (tokens 32w ..
-  // 32w + 31 = TMEM lanes of its quarter).  Before the sequence length is
-  // known (every entry read is inside the table row), lanes 0 and 1 read the
-  // block ids of their segment of chunks 0 .. 2; the split's whole slice of
-  // the row goes to shared memory in the set-up below, cut to the split and
-  // the pool.
+  // Loader warp w owns segment(s) seg_of(w, sg) of every chunk (tokens 16 s
+  // .. 16 s + 15 = TMEM lanes of its quarter).  Before the sequence length is
+  // known (every entry read is inside the table row), lanes sg < kSegs read
+  // the block ids of their segment of chunks 0 .. 2; the split's whole slice
+  // of the row goes to shared memory in the set-up below, cut to the split
+  // and the pool.
   const int blk0 = split * a.blocks_per_split;
   const int32_t* bt_row = a.block_table + static_cast<int64_t>(b) * a.max_blocks_per_seq;
   constexpr int kTblPer = kTblBlocks / (32 * kLoadWarps);
-  int32_t bfirst[kNV];  // loaders, lanes 0 and 1: block ids of chunks 0 .. 2
+  int32_t bfirst[kNV];  // loaders, lanes sg < kSegs: block ids of chunks 0 .. 2
   if (is_loader) {
     const int nload = min(a.blocks_per_split, a.max_blocks_per_seq - blk0);
 #pragma unroll
     for (int i = 0; i < kNV; ++i) {
-      const int j = kChunkBlocks * i + 2 * warp + lane;
-      bfirst[i] = lane < 2 && j < nload ? __ldg(bt_row + blk0 + j) : -1;
+      const int j = kChunkBlocks * i + seg_of<kWide>(warp, lane % kSegs);
+      bfirst[i] = lane < kSegs && j < nload ? __ldg(bt_row + blk0 + j) : -1;
     }
   }
   int L = a.seq_lens[b];
@@ -671,20 +699,20 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
 
   const uint8_t* pool_h = a.pool + static_cast<int64_t>(h) * kSeg;
   const int64_t pstride = static_cast<int64_t>(a.num_kv_heads) * kSeg;
-  const int mseg = lane >> 4;  // segment of my factor bytes
+  const int mseg = lane >> 4;  // my factor bytes: those of the loader warp's mseg-th segment (< kSegs)
 
   const uint32_t my_stg = smem_u32(sm.stg[warp < kLoadWarps ? warp : 0][0]);
-  // Bulk copies of the loader warp's two segments of a chunk into staging
-  // slot `slot`: lanes 0 and 1 pass their segment's block id (-1: absent,
+  // Bulk copies of the loader warp's segments of a chunk into staging slot
+  // `slot`: lanes sg < kSegs pass their segment's block id (-1: absent,
   // nothing copied; the factors mark its tokens absent), every lane calls.
   // The expected byte count is posted before any copy is issued.
   auto issue = [&](int32_t p, int slot) {
     uint64_t* bar = &sm.full[warp][slot];
-    const uint32_t okm = __ballot_sync(0xffffffffu, lane < 2 && p >= 0);
+    const uint32_t okm = __ballot_sync(0xffffffffu, lane < kSegs && p >= 0);
     if (lane == 0) mbar_arrive_expect_tx(bar, static_cast<uint32_t>(__popc(okm)) * kSeg);
     __syncwarp();
-    if (lane < 2 && p >= 0)
-      bulk_g2s(my_stg + slot * (2 * kSeg) + lane * kSeg, pool_h + static_cast<int64_t>(p) * pstride, kSeg, bar);
+    if (lane < kSegs && p >= 0)
+      bulk_g2s(my_stg + slot * (kSegs * kSeg) + lane * kSeg, pool_h + static_cast<int64_t>(p) * pstride, kSeg, bar);
   };
 
   // ---- 0. set-up: barriers and tensor memory; first loads; query digits ----
@@ -701,7 +729,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
     const int nblk = blk1 - blk0;
 #pragma unroll
     for (int i = 0; i < kNV; ++i) {
-      const int j = kChunkBlocks * i + 2 * warp + lane;
+      const int j = kChunkBlocks * i + seg_of<kWide>(warp, lane % kSegs);
       if (!(j < nblk && bfirst[i] >= 0 && bfirst[i] < a.num_blocks)) bfirst[i] = -1;
     }
     // the first three chunks' copies go out while the query is rotated (each
@@ -723,14 +751,13 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
     }
   } else if (is_soft) {
     const int sw = warp - kLoadWarps;
-    const int stok = tid - 32 * kLoadWarps;
+    const int st = tid - 32 * kLoadWarps;  // 0 .. kSoftThreads-1
     // rotate the G query heads, then write their digits with one c1 for all
     // heads
-    reinterpret_cast<uint4*>(sm.qb)[stok] = make_uint4(0, 0, 0, 0);
-    reinterpret_cast<uint4*>(sm.qb)[stok + 128] = make_uint4(0, 0, 0, 0);
+    for (int i = st; i < 32 * kHeadDim / 16; i += kSoftThreads) reinterpret_cast<uint4*>(sm.qb)[i] = make_uint4(0, 0, 0, 0);
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int g = sw + 4 * i;
+    for (int i = 0; i < kQHeads; ++i) {
+      const int g = sw + kSoftWarps * i;
       if (g < G) {
         fwht_warp(x[i], lane, a.scale_log2);
         float s4 = (x[i][0] + x[i][1]) + (x[i][2] + x[i][3]);
@@ -743,15 +770,15 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
         if (lane == 0) sm.hq[g] = make_float2(s4, mx);
       }
     }
-    soft_sync();
+    soft_sync<kSoftThreads>();
     float mx = 0.0f;
 #pragma unroll
     for (int g = 0; g < G; ++g) mx = fmaxf(mx, sm.hq[g].y);
     const float inv = mx > 0.0f ? 127.0f / mx : 0.0f;
-    if (stok == 0) sm.c1 = mx * (1.0f / 127.0f);
+    if (st == 0) sm.c1 = mx * (1.0f / 127.0f);
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int g = sw + 4 * i;
+    for (int i = 0; i < kQHeads; ++i) {
+      const int g = sw + kSoftWarps * i;
       if (g < G) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -802,20 +829,25 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
 
   // ---- 1. the paged scan ------------------------------------------------------
   if (is_loader) {
-    const uint32_t my_lanes = tbase + (static_cast<uint32_t>(warp * 32) << 16);
-    // my value rows, segment 1: + 2048.  VB = 2: row lane/2 of the segment,
-    // positions 64 (lane%2) + [0, 64); VB = 4: rows lane/4 and (+ 1024)
-    // 8 + lane/4, positions 32 (lane%4) + [0, 32)
-    const uint32_t my_vt =
-        VB == 2 ? smem_u32(sm.vt[0]) + ((32 * warp + (lane >> 1)) >> 3) * 1024 + (lane & 1) * 512 +
-                      (lane >> 1 & 7) * 16
-                : smem_u32(sm.vt[0]) + 4 * warp * 1024 + (lane >> 2) * 16 + 2 * (lane & 3) * 128;
-    const int mrow0 = 4 * (lane & 3);    // my factor rows mrow0 .. mrow0+3 of segment mseg
+    // TMEM lanes of my segment sg: 16 seg_of(warp, sg) + [0, 16)
+    auto seg_lanes = [&](int sg) { return tbase + (static_cast<uint32_t>(16 * seg_of<kWide>(warp, sg)) << 16); };
+    // my value rows of segment sg (token base tb = 16 s).  VB = 2: row lane/2
+    // of the segment, positions 64 (lane%2) + [0, 64); VB = 4: rows lane/4
+    // and (+ 1024) 8 + lane/4, positions 32 (lane%4) + [0, 32)
+    auto seg_vt = [&](int sg) -> uint32_t {
+      const int tb = 16 * seg_of<kWide>(warp, sg);
+      return VB == 2 ? smem_u32(sm.vt[0]) + ((tb + (lane >> 1)) >> 3) * 1024 + (lane & 1) * 512 + (lane >> 1 & 7) * 16
+                     : smem_u32(sm.vt[0]) + (tb >> 3) * 1024 + (lane >> 2) * 16 + 2 * (lane & 3) * 128;
+    };
+    const int mrow0 = 4 * (lane & 3);    // my factor rows mrow0 .. mrow0+3 of my factor segment
     const int mkind = (lane >> 2) & 3;  // S_K, Z_K, S_V, Z_V
+    const bool mlive = mseg < kSegs;    // (a one-segment loader warp: lanes 16-31 have no factors)
+    const int mslot = mlive ? mseg : 0;
+    const int mblk = seg_of<kWide>(warp, mslot);  // my factor segment's block within a chunk
     const uint32_t mnone = mkind == 2 ? 0xBC00BC00u : 0u;  // the factors of an absent segment (S_V = -1)
     // the block holding position L-1, for the lanes holding S_V (-2: none)
     const int blk_last = mkind == 2 ? (L - 1) / kBlockSize : -2;
-    const uint32_t my_meta = smem_u32(&sm.meta[0][mkind][32 * warp + 16 * mseg + mrow0]);
+    const uint32_t my_meta = smem_u32(&sm.meta[0][mkind][16 * mblk + mrow0]);
 #pragma unroll
     for (int i = 0; i < kNV; ++i)  // the deferred chunk, if it is one of the first three
       if (i == c_defer) issue(bfirst[i], i);
@@ -829,28 +861,30 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
         bad = true;
         pend |= (1u << r.i) | (r.ph << (4 + r.i));
       }
-      const uint32_t sb = my_stg + r.i * (2 * kSeg);
-      KeyRaw<KB> kr[2];
-      uint4 vr[2][VB / 2];  // VB = 2: one 16-byte piece per segment; VB = 4: two
+      const uint32_t sb = my_stg + r.i * (kSegs * kSeg);
+      KeyRaw<KB> kr[kSegs];
+      uint4 vr[kSegs][VB / 2];  // VB = 2: one 16-byte piece per segment; VB = 4: two
 #pragma unroll
-      for (int sg = 0; sg < 2; ++sg) {
+      for (int sg = 0; sg < kSegs; ++sg) {
         kr[sg].load(sb + sg * kSeg + F::kOffK, lane);
 #pragma unroll
         for (int i = 0; i < VB / 2; ++i) vr[sg][i] = lds128(sb + sg * kSeg + F::kOffV + 512 * i + 16 * lane);
       }
-      const uint2 mr2 = lds64(sb + mseg * kSeg + F::kOffSK + 8 * (lane & 15));
-      const bool seg_ok = sm.tbl[kChunkBlocks * c + 2 * warp + mseg] >= 0;  // my factor segment is present
+      const uint2 mr2 = lds64(sb + mslot * kSeg + F::kOffSK + 8 * (lane & 15));
+      const bool seg_ok = sm.tbl[kChunkBlocks * c + mblk] >= 0;  // my factor segment is present
       // the slot is read: refill it with chunk c+3 (the reads above are
-      // ordered before the copy's writes by the proxy fence); lanes 2 and 3
-      // prefetch their segments of chunk c+6 into L2.  (After a failed wait
-      // no copy is issued any more: see the drain below.)
+      // ordered before the copy's writes by the proxy fence); lanes kSegs ..
+      // 2 kSegs - 1 prefetch the segments of chunk c+6 into L2.  (After a
+      // failed wait no copy is issued any more: see the drain below.)
       async_proxy_fence();
       __syncwarp();
       if (!bad) {
-        const int cc = c + kNV + kNV * (lane >> 1);
-        const int32_t p = lane < 4 && cc < nchunks ? sm.tbl[kChunkBlocks * cc + 2 * warp + (lane & 1)] : -1;
-        if (lane >= 2 && p >= 0) prefetch_l2(pool_h + static_cast<int64_t>(p) * pstride, kSeg);
-        if (c + kNV < nchunks) issue(lane < 2 ? p : -1, r.i);
+        const int cc = c + kNV + kNV * (lane / kSegs);
+        const int32_t p = lane < 2 * kSegs && cc < nchunks
+                              ? sm.tbl[kChunkBlocks * cc + seg_of<kWide>(warp, lane % kSegs)]
+                              : -1;
+        if (lane >= kSegs && p >= 0) prefetch_l2(pool_h + static_cast<int64_t>(p) * pstride, kSeg);
+        if (c + kNV < nchunks) issue(lane < kSegs ? p : -1, r.i);
       }
 
       if (c >= kNV) {  // buffers r.i are free once PV(c-3) (issued after QK(c-2)) is done
@@ -858,14 +892,14 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
         tc_fence_after();
       }
 #pragma unroll
-      for (int sg = 0; sg < 2; ++sg) {  // key codes of segment sg -> lanes 32 warp + 16 sg + [0, 16)
+      for (int sg = 0; sg < kSegs; ++sg) {  // key codes of segment sg -> its 16 TMEM lanes
         uint32_t w[16];
         kr[sg].spread(w);
-        tmem_st16x256(my_lanes + (static_cast<uint32_t>(16 * sg) << 16) + kColA + 32 * r.i, w);
+        tmem_st16x256(seg_lanes(sg) + kColA + 32 * r.i, w);
       }
 #pragma unroll
-      for (int sg = 0; sg < 2; ++sg) {  // value codes, one byte each
-        const uint32_t va = my_vt + sg * 2048 + r.i * (kChunkTokens * kHeadDim);
+      for (int sg = 0; sg < kSegs; ++sg) {  // value codes, one byte each
+        const uint32_t va = seg_vt(sg) + r.i * (kChunkTokens * kHeadDim);
         if (VB == 2) {  // crumb k of each byte -> position 16i + 4k + b, times 4^k
           const uint32_t vw[4] = {vr[sg][0].x, vr[sg][0].y, vr[sg][0].z, vr[sg][0].w};
 #pragma unroll
@@ -886,7 +920,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
          // (a segment outside the split or the pool, a row past the end of
          // the sequence: only in the block holding position L-1)
         uint32_t m0 = seg_ok ? mr2.x : mnone, m1 = seg_ok ? mr2.y : mnone;
-        const int blk = blk0 + kChunkBlocks * c + 2 * warp + mseg;
+        const int blk = blk0 + kChunkBlocks * c + mblk;
         if (blk == blk_last) {
           const int nv = L - blk * kBlockSize - mrow0;  // my rows inside the sequence (may be <= 0 or > 4)
           if (nv < 1) m0 = (m0 & 0xFFFF0000u) | 0xBC00u;
@@ -894,7 +928,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
           if (nv < 3) m1 = (m1 & 0xFFFF0000u) | 0xBC00u;
           if (nv < 4) m1 = (m1 & 0x0000FFFFu) | 0xBC000000u;
         }
-        sts64(my_meta + r.i * (4 * kChunkTokens * 2), m0, m1);
+        if (mlive) sts64(my_meta + r.i * (4 * kChunkTokens * 2), m0, m1);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -955,18 +989,37 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
     __syncwarp();
     if (!mbar_wait_final(&sm.fin, 0u)) bad = true;
   } else {
-    // softmax warps: thread stok <-> token stok of S, value position stok of O
+    // softmax warps: thread st <-> token stok = st % 128 of S and value
+    // position stok of O, heads hb .. hb + kHeads - 1 (hb = 0 but in the
+    // wide layout, where the second 128 threads take heads 4 .. 7)
     const int sw = warp - kLoadWarps;
-    const int stok = tid - 32 * kLoadWarps;
-    const uint32_t my_lanes = tbase + (static_cast<uint32_t>(sw * 32) << 16);
+    const int st = tid - 32 * kLoadWarps;
+    const int stok = st & 127;
+    const int hf = kWide ? st >> 7 : 0;
+    const int hb = hf * kHeads;
+    const int wg = sw & ~3;  // the four warps of my heads: wg .. wg + 3
+    const uint32_t my_lanes = tbase + (static_cast<uint32_t>((sw & 3) * 32) << 16);
+    const uint32_t my_acc = my_lanes + kColAcc + 8 * hf;  // o~ so far of my heads (fp32, column per head)
     const uint32_t my_pm = smem_u32(sm.pm[0]) + (stok >> 3) * 256 + (stok & 7) * 16;
-    // (o~ so far, in units of the output scale below, lives in tensor memory
-    // at kColAcc: it is touched only when the running max moves and at the
-    // end, and registers are the scarce resource of this loop)
-    float qs[G], mr[G], lr[G], zr[G];
+    // the three S digits of my heads, by fixed register indices (a register
+    // array indexed by the run-time hb would go to local memory)
+    auto pick_digits = [&](const uint32_t (&a)[16], const uint32_t (&b)[8], uint32_t (&e0)[kHeads],
+                           uint32_t (&e1)[kHeads], uint32_t (&e2)[kHeads]) {
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      qs[g] = sm.hq[g].x;
+      for (int g = 0; g < kHeads; ++g) {
+        const int hi = kWide ? kHeads + g : g;
+        e0[g] = hf ? a[hi] : a[g];
+        e1[g] = hf ? a[8 + hi] : a[8 + g];
+        e2[g] = hf ? b[hi] : b[g];
+      }
+    };
+    // (o~ so far, in units of the output scale below, lives in tensor memory
+    // at my_acc: it is touched only when the running max moves and at the
+    // end, and registers are the scarce resource of this loop)
+    float qs[kHeads], mr[kHeads], lr[kHeads], zr[kHeads];
+#pragma unroll
+    for (int g = 0; g < kHeads; ++g) {
+      qs[g] = sm.hq[hb + g].x;
       mr[g] = kNoMax;
       lr[g] = zr[g] = 0.0f;
     }
@@ -980,28 +1033,29 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
 
     {  // o~ so far: 0
       const uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-      tmem_st8(my_lanes + kColAcc, z);
+      tmem_st8(my_acc, z);
       tmem_wait_st();
     }
-    // fold O buffer k (my lane = value position stok) into o~ so far, with
-    // the pending factor of each head (scaled) or 1
+    // fold O buffer k (my lane = value position stok; my heads' columns
+    // 4 hb .. 4 hb + 4 kHeads - 1) into o~ so far, with the pending factor of
+    // each head (scaled) or 1
     auto fold_o = [&](int k, bool scaled) {
       uint32_t r[16], r2[16], oa[8];
-      tmem_ld16(my_lanes + kColO + 32 * k, r);
-      tmem_ld16(my_lanes + kColO + 32 * k + 16, r2);
-      tmem_ld8(my_lanes + kColAcc, oa);
+      tmem_ld16(my_lanes + kColO + 32 * k + 4 * hb, r);
+      if (kHeads > 4) tmem_ld16(my_lanes + kColO + 32 * k + 16, r2);
+      tmem_ld8(my_acc, oa);
       tmem_wait_ld();
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
+      for (int g = 0; g < kHeads; ++g) {
         const uint32_t* q = g < 4 ? r + 4 * g : r2 + 4 * g - 16;
         const float v = fmaf(static_cast<float>(static_cast<int>(q[3])), 16777216.0f,
                              fmaf(static_cast<float>(static_cast<int>(q[2])), 65536.0f,
                                   fmaf(static_cast<float>(static_cast<int>(q[1])), 256.0f,
                                        static_cast<float>(static_cast<int>(q[0])))));
         const float o = __uint_as_float(oa[g]);
-        oa[g] = __float_as_uint(scaled ? fmaf(v, sm.palpha[sw][g], o) : o + v);
+        oa[g] = __float_as_uint(scaled ? fmaf(v, sm.palpha[sw][hb + g], o) : o + v);
       }
-      tmem_st8(my_lanes + kColAcc, oa);
+      tmem_st8(my_acc, oa);
       tmem_wait_st();
     };
 
@@ -1032,21 +1086,24 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
       // E with S_V < 2^E, from the fp16 exponent of S_V (-14 for subnormals and 0)
       const float e = static_cast<float>(static_cast<int>((hsv >> 10) & 31u) - 14);
       tmem_wait_ld();
-      float dg[G];
+      // S column g holds digit 0 of head g, column 8 + g digit 1, 16 + g digit 2
+      uint32_t d0[kHeads], d1[kHeads], d2[kHeads];
+      pick_digits(sr, sr2, d0, d1, d2);
+      float dg[kHeads];
       float dmax = -CUDART_INF_F;
-      if (G == 1) {
-        const int e12 = static_cast<int>(sr[8]) * 254 + static_cast<int>(sr2[0]);
-        const float xg = fmaf(__int2float_rn(e12), 1.0f / 64516.0f, small_i2f(sr[0]));
+      if (kHeads == 1) {
+        const int e12 = static_cast<int>(d1[0]) * 254 + static_cast<int>(d2[0]);
+        const float xg = fmaf(__int2float_rn(e12), 1.0f / 64516.0f, small_i2f(d0[0]));
         dg[0] = fmaf(mt.x, xg, fmaf(mt.y, qs[0], -mr[0]));
         dmax = dg[0];
       } else {
         const u64x mx2 = pk2(mt.x, mt.x), my2 = pk2(mt.y, mt.y);
         const u64x k2 = pk2(1.0f / 64516.0f, 1.0f / 64516.0f), m2 = pk2(-12582912.0f, -12582912.0f);
 #pragma unroll
-        for (int g = 0; g < (G > 1 ? G : 2); g += 2) {
-          const float xe0 = __int2float_rn(static_cast<int>(sr[8 + g]) * 254 + static_cast<int>(sr2[g]));
-          const float xe1 = __int2float_rn(static_cast<int>(sr[9 + g]) * 254 + static_cast<int>(sr2[g + 1]));
-          const u64x s0 = add2(pk2(__uint_as_float(sr[g] + 0x4B400000u), __uint_as_float(sr[g + 1] + 0x4B400000u)), m2);
+        for (int g = 0; g < (kHeads > 1 ? kHeads : 2); g += 2) {
+          const float xe0 = __int2float_rn(static_cast<int>(d1[g]) * 254 + static_cast<int>(d2[g]));
+          const float xe1 = __int2float_rn(static_cast<int>(d1[g + 1]) * 254 + static_cast<int>(d2[g + 1]));
+          const u64x s0 = add2(pk2(__uint_as_float(d0[g] + 0x4B400000u), __uint_as_float(d0[g + 1] + 0x4B400000u)), m2);
           const u64x xg = fma2(pk2(xe0, xe1), k2, s0);
           const u64x d = fma2(mx2, xg, fma2(my2, pk2(qs[g], qs[g + 1]), pk2(-mr[g], -mr[g + 1])));
           upk2(d, dg[g], dg[g + 1]);
@@ -1054,7 +1111,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
         }
       }
       const bool flag = valid && (dmax + e > kTrigger);
-      const bool any = soft_vote_any(flag);
+      const bool any = soft_vote_any<kSoftThreads>(flag);
       if (any) {
         // rare: move the running max of each head to the chunk's max of
         // s + E plus the headroom; the scores are formed again from S (still
@@ -1063,22 +1120,26 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
         tmem_ld16(my_lanes + kColS + 32 * P, sr);
         tmem_ld8(my_lanes + kColS + 32 * P + 16, sr2);
         tmem_wait_ld();
-        float sg[G];
+        pick_digits(sr, sr2, d0, d1, d2);
+        float sg[kHeads];
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const int e12 = static_cast<int>(sr[8 + g]) * 254 + static_cast<int>(sr2[g]);
-          const float xg = fmaf(__int2float_rn(e12), 1.0f / 64516.0f, small_i2f(sr[g]));
+        for (int g = 0; g < kHeads; ++g) {
+          const int gh = hb + g;
+          const int e12 = static_cast<int>(d1[g]) * 254 + static_cast<int>(d2[g]);
+          const float xg = fmaf(__int2float_rn(e12), 1.0f / 64516.0f, small_i2f(d0[g]));
           sg[g] = fmaf(mt.x, xg, mt.y * qs[g]);
           float u = valid ? sg[g] + e : -CUDART_INF_F;
 #pragma unroll
           for (int o = 16; o; o >>= 1) u = fmaxf(u, __shfl_xor_sync(0xffffffffu, u, o));
-          if (lane == 0) sm.red[sw][g][0] = u;
+          if (lane == 0) sm.red[sw][gh][0] = u;
         }
-        soft_sync();
-        float alpha[G];
+        soft_sync<kSoftThreads>();
+        float alpha[kHeads];
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float M = fmaxf(fmaxf(sm.red[0][g][0], sm.red[1][g][0]), fmaxf(sm.red[2][g][0], sm.red[3][g][0]));
+        for (int g = 0; g < kHeads; ++g) {
+          const int gh = hb + g;
+          const float M = fmaxf(fmaxf(sm.red[wg][gh][0], sm.red[wg + 1][gh][0]),
+                                fmaxf(sm.red[wg + 2][gh][0], sm.red[wg + 3][gh][0]));
           const float mn = fmaxf(mr[g], M + kHeadroom);
           alpha[g] = ex2(mr[g] - mn);
           lr[g] *= alpha[g];
@@ -1088,17 +1149,17 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
         }
         {  // o~ so far in units of the new max
           uint32_t oa[8];
-          tmem_ld8(my_lanes + kColAcc, oa);
+          tmem_ld8(my_acc, oa);
           tmem_wait_ld();
 #pragma unroll
-          for (int g = 0; g < G; ++g) oa[g] = __float_as_uint(__uint_as_float(oa[g]) * alpha[g]);
-          tmem_st8(my_lanes + kColAcc, oa);
+          for (int g = 0; g < kHeads; ++g) oa[g] = __float_as_uint(__uint_as_float(oa[g]) * alpha[g]);
+          tmem_st8(my_acc, oa);
           tmem_wait_st();
         }
         if (c > fresh_c) {  // PVs of chunks fresh_c .. c-1 ran into buffer ob: pending
           if (lane == 0) {
 #pragma unroll
-            for (int g = 0; g < G; ++g) sm.palpha[sw][g] = alpha[g];
+            for (int g = 0; g < kHeads; ++g) sm.palpha[sw][hb + g] = alpha[g];
           }
           __syncwarp();
           pend = true;
@@ -1112,7 +1173,7 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
       if (lane == 0) mbar_arrive(&sm.s_free[P]);
       // P' of chunk c -> pm[r.i] (free: PV(c-3) was issued before QK(c), which is done)
       uint32_t pw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-      if (G == 1) {
+      if (kHeads == 1) {
         const float p = valid ? ex2(dg[0]) : 0.0f;
         pw[0] = __float2uint_rn(p * mt.z);
         const float pt = __uint2float_rn(pw[0]) * pinv;
@@ -1121,8 +1182,8 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
       } else {
         const u64x z2 = pk2(mt.z, mt.z), i2 = pk2(pinv, pinv), w2 = pk2(mt.w, mt.w);
 #pragma unroll
-        for (int g = 0; g < (G > 1 ? G : 2); g += 2) {
-          float x0, x1, t0, t1, l0, l1, q0, q1;
+        for (int g = 0; g < (kHeads > 1 ? kHeads : 2); g += 2) {
+          float x0, x1, l0, l1, q0, q1;
           upk2(mul2(pk2(valid ? ex2(dg[g]) : 0.0f, valid ? ex2(dg[g + 1]) : 0.0f), z2), x0, x1);
           pw[g] = __float2uint_rn(x0);  // rne(P' 2^29) < 2^32
           pw[g + 1] = __float2uint_rn(x1);
@@ -1130,14 +1191,18 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
           const u64x pt = mul2(pk2(__uint2float_rn(pw[g]), __uint2float_rn(pw[g + 1])), i2);
           upk2(add2(pk2(lr[g], lr[g + 1]), pt), l0, l1);
           upk2(fma2(pt, w2, pk2(zr[g], zr[g + 1])), q0, q1);
-          lr[g] = l0; lr[g + 1] = l1; zr[g] = q0; zr[g + 1] = q1;
-          (void)t0; (void)t1;
+          lr[g] = l0;
+          lr[g + 1] = l1;
+          zr[g] = q0;
+          zr[g + 1] = q1;
         }
       }
-      const uint32_t pa = my_pm + r.i * (kChunkTokens * 32);
+      // (P' column n = 4 g + j: my heads' bytes are 16-byte piece hf, and the
+      // next one when I take all eight)
+      const uint32_t pa = my_pm + r.i * (kChunkTokens * 32) + 128 * hf;
       sts128(pa, pw[0], pw[1], pw[2], pw[3]);
-      sts128(pa + 128, pw[4], pw[5], pw[6], pw[7]);
-      if (stok == 0) sm.fresh[r.i] = (fresh_c == c ? 1 : 0) | (ob << 1);
+      if (kHeads > 4) sts128(pa + 128, pw[4], pw[5], pw[6], pw[7]);
+      if (st == 0) sm.fresh[r.i] = (fresh_c == c ? 1 : 0) | (ob << 1);
       async_proxy_fence();
       tc_fence_before();
       __syncwarp();
@@ -1152,9 +1217,9 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
       if (pend) fold_o(ob ^ 1, true);
       fold_o(ob, false);
     }
-    // l and zeta over the 128 tokens' threads; o~ in dim order
+    // l and zeta over the 128 tokens' threads of my heads; o~ in dim order
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
+    for (int g = 0; g < kHeads; ++g) {
       float l = lr[g], z = zr[g];
 #pragma unroll
       for (int o = 16; o; o >>= 1) {
@@ -1162,11 +1227,11 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
         z += __shfl_xor_sync(0xffffffffu, z, o);
       }
       if (lane == 0) {
-        sm.red[sw][g][0] = l;
-        sm.red[sw][g][1] = z;
+        sm.red[sw][hb + g][0] = l;
+        sm.red[sw][hb + g][1] = z;
       }
     }
-    soft_sync();
+    soft_sync<kSoftThreads>();
     const int d = value_dim_of_pos<VB>(stok);
     // output scale of my value position: the fixed point and the factor of the spread
     const float oscale = kFixInv * __uint_as_float((127u - value_scale_log2<VB>(stok)) << 23);
@@ -1175,19 +1240,20 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
     // normalised o~ goes to shared memory for the output rotation.
     float* rec = a.partials + ((static_cast<int64_t>(b) * a.num_q_heads + h * G) * a.nsplit + split) * kPartialFloats;
     uint32_t oacc[8];
-    tmem_ld8(my_lanes + kColAcc, oacc);
+    tmem_ld8(my_acc, oacc);
     tmem_wait_ld();
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float z = (sm.red[0][g][1] + sm.red[1][g][1]) + (sm.red[2][g][1] + sm.red[3][g][1]);
-      const float lsum = (sm.red[0][g][0] + sm.red[1][g][0]) + (sm.red[2][g][0] + sm.red[3][g][0]);
+    for (int g = 0; g < kHeads; ++g) {
+      const int gh = hb + g;
+      const float z = (sm.red[wg][gh][1] + sm.red[wg + 1][gh][1]) + (sm.red[wg + 2][gh][1] + sm.red[wg + 3][gh][1]);
+      const float lsum = (sm.red[wg][gh][0] + sm.red[wg + 1][gh][0]) + (sm.red[wg + 2][gh][0] + sm.red[wg + 3][gh][0]);
       const float o = fmaf(__uint_as_float(oacc[g]), oscale, z);
       if (a.nsplit > 1) {
-        float* rg = rec + static_cast<int64_t>(g) * a.nsplit * kPartialFloats;
+        float* rg = rec + static_cast<int64_t>(gh) * a.nsplit * kPartialFloats;
         rg[d] = o;
-        if (stok == g) *reinterpret_cast<float2*>(rg + kHeadDim) = make_float2(mr[g], lsum);
+        if (stok == gh) *reinterpret_cast<float2*>(rg + kHeadDim) = make_float2(mr[g], lsum);
       } else {
-        sm.obuf[g][d] = lsum > 0.0f ? o / lsum : 0.0f;
+        sm.obuf[gh][d] = lsum > 0.0f ? o / lsum : 0.0f;
       }
     }
   }
@@ -1289,22 +1355,27 @@ __global__ void __launch_bounds__(kThreads, kMinCtasOf<KB, VB>) decode_kernel(De
   }
 }
 
-template <int G, int KB, int VB>
+template <int G, int KB, int VB, bool kWide>
 cudaError_t launch_g(const DecodeArgs& a, cudaStream_t stream) {
-  constexpr int kBytes = kSmemBytesOf<Fmt<KB, VB>::kSegBytes>;
-  const cudaError_t e = ensure_smem_limit<decode_kernel<G, KB, VB>>(kBytes);
+  constexpr int kBytes = kSmemBytesOf<Fmt<KB, VB>::kSegBytes, kWide>;
+  const cudaError_t e = ensure_smem_limit<decode_kernel<G, KB, VB, kWide>>(kBytes);
   if (e != cudaSuccess) return e;
   const dim3 grid(a.nsplit, a.num_kv_heads, a.batch);
-  return launch_pdl(decode_kernel<G, KB, VB>, grid, dim3(kThreads), kBytes, stream, a);
+  return launch_pdl(decode_kernel<G, KB, VB, kWide>, grid, dim3(Roles<kWide>::kThreads), kBytes, stream, a);
 }
 
 template <int KB, int VB>
 cudaError_t launch_p(const DecodeArgs& a, cudaStream_t stream) {
   switch (a.num_q_heads / a.num_kv_heads) {
-    case 1: return launch_g<1, KB, VB>(a, stream);
-    case 2: return launch_g<2, KB, VB>(a, stream);
-    case 4: return launch_g<4, KB, VB>(a, stream);
-    case 8: return launch_g<8, KB, VB>(a, stream);
+    case 1: return launch_g<1, KB, VB, false>(a, stream);
+    case 2: return launch_g<2, KB, VB, false>(a, stream);
+    case 4: return launch_g<4, KB, VB, false>(a, stream);
+    case 8:
+      // a grid that the SMs hold at once, one CTA each: the wide role layout
+      // (its chunks pass each role in about half the time)
+      if (static_cast<int64_t>(a.nsplit) * a.num_kv_heads * a.batch <= device_sm_count())
+        return launch_g<8, KB, VB, true>(a, stream);
+      return launch_g<8, KB, VB, false>(a, stream);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -1348,8 +1419,9 @@ int decode_ctas_per_sm() {
   if (cached[dev] > 0) return cached[dev];
   int n = 0;
   constexpr int kBytes = kSmemBytesOf<Fmt<4, 2>::kSegBytes>;
-  if (ensure_smem_limit<decode_kernel<8, 4, 2>>(kBytes) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<8, 4, 2>, kThreads, kBytes) != cudaSuccess ||
+  if (ensure_smem_limit<decode_kernel<8, 4, 2, false>>(kBytes) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<8, 4, 2, false>, Roles<false>::kThreads, kBytes) !=
+          cudaSuccess ||
       n < 1)
     n = 1;
   cached[dev] = n < 2 ? n : 2;  // two CTAs' tensor memory (2 x 256 columns) fills an SM
