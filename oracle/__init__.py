@@ -70,6 +70,9 @@ def lib():
                 "kvqo_decode_one": (ctypes.c_int, [gp, vp, vp, i32, i32, i32, vp, i32, dbl, i32, vp]),
                 "kvqo_decode_attention": (ctypes.c_int, [gp, vp, vp, i32, i32, i32, vp, i32, vp, dbl, i32, i32, vp]),
                 "kvqo_attention_dense": (ctypes.c_int, [i32, i32, vp, vp, i32, i64, i32, vp, i32, i32, i32, dbl, vp]),
+                "kvqo_window_append": (ctypes.c_int, [i32, i32, i32, i32, i32, vp, vp, vp, i64, vp, vp, i32]),
+                "kvqo_decode_attention_window": (ctypes.c_int, [gp, vp, vp, i32, i32, vp, i32, i32, i32, vp, i32, vp,
+                                                                dbl, i32, vp]),
                 "kvqo_packed_bytes_per_token_head": (dbl, [i32, i32, i32]),
                 "kvqo_dense_bytes_per_token": (dbl, [i32, i32, i32, i32]),
             }
@@ -216,6 +219,40 @@ def decode_attention(g, pool, q, q_dtype, block_table, seq_lens, scale=0.0, form
     out = np.zeros((batch, hq, d), dtype=np.float64)
     _check(lib().kvqo_decode_attention(ctypes.byref(g), _p(pool), _p(q), q_dtype, batch, hq, _p(bt), bt.shape[1],
                                        _p(lens), scale, form, nthreads, _p(out)), "decode_attention")
+    return out
+
+
+def new_window(num_seqs, num_kv_heads, sink, recent, d=128, fill=0) -> np.ndarray:
+    """A window buffer of bf16 bits [num_seqs, Hkv, sink + recent, 2, d]."""
+    return np.full((num_seqs, num_kv_heads, sink + recent, 2, d), fill, dtype=np.uint16)
+
+
+def window_append(win, sink, recent, k, v, seq_ids, positions, token_stride=None) -> None:
+    """k, v: bf16 bits [n, Hkv, d] (rows as in the write path); sequence
+    seq_ids[n] (negative: skipped), position positions[n]."""
+    num_seqs, hkv, rows, _, d = win.shape
+    assert rows == sink + recent
+    n = len(seq_ids)
+    k = np.ascontiguousarray(k, dtype=np.uint16)
+    v = np.ascontiguousarray(v, dtype=np.uint16)
+    ts = hkv * d if token_stride is None else token_stride
+    ids = np.ascontiguousarray(seq_ids, dtype=np.int32)
+    pos = np.ascontiguousarray(positions, dtype=np.int32)
+    _check(lib().kvqo_window_append(d, hkv, sink, recent, num_seqs, _p(win), _p(k), _p(v), ts, _p(ids), _p(pos), n),
+           "window_append")
+
+
+def decode_attention_window(g, pool, win, sink, recent, q, q_dtype, block_table, seq_lens, scale=0.0,
+                            nthreads=1) -> np.ndarray:
+    q = np.ascontiguousarray(q)
+    batch, hq, d = q.shape
+    bt = np.ascontiguousarray(block_table, dtype=np.int32)
+    lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    out = np.zeros((batch, hq, d), dtype=np.float64)
+    w = np.ascontiguousarray(win, dtype=np.uint16)
+    _check(lib().kvqo_decode_attention_window(ctypes.byref(g), _p(pool), _p(w), sink, recent, _p(q), q_dtype, batch,
+                                              hq, _p(bt), bt.shape[1], _p(lens), scale, nthreads, _p(out)),
+           "decode_attention_window")
     return out
 
 

@@ -480,7 +480,15 @@ struct DecodeJob {
   double tau;
   int32_t form;
   double* out;
+  const uint16_t* win;  // bf16 window of sink and recent tokens (form 0 only), or null
+  int32_t sink, recent;
 };
+
+// Element (b, h, row, kv, i) of a window buffer.
+size_t win_index(int32_t H, int32_t rows, int32_t d, int32_t b, int32_t h, int32_t row, int32_t kv,
+                 int32_t i) {
+  return ((((static_cast<size_t>(b) * H + h) * rows + row) * 2 + kv) * d) + i;
+}
 
 // All query heads of one (sequence b, kv head h): the tokens are dequantized
 // once and every query head of the group attends to them.
@@ -493,6 +501,23 @@ int run_pair(const DecodeJob& J, int32_t b, int32_t h) {
   const int rc = gather_tokens(J.g, J.pool, h, J.bt + static_cast<size_t>(b) * J.mbps, L,
                                J.form, gt);
   if (rc) return rc;
+  if (J.win) {  // window positions take the raw rows
+    const int32_t rows = J.sink + J.recent;
+    for (int32_t t = 0; t < L; ++t) {
+      int32_t row = -1;
+      if (t < J.sink)
+        row = t;
+      else if (J.recent > 0 && t >= L - J.recent)
+        row = J.sink + t % J.recent;
+      if (row < 0) continue;
+      for (int32_t i = 0; i < d; ++i) {
+        gt.khat[static_cast<size_t>(t) * d + i] =
+            kvqo_bf16_to_f64(J.win[win_index(J.g->num_kv_heads, rows, d, b, h, row, 0, i)]);
+        gt.vhat[static_cast<size_t>(t) * d + i] =
+            kvqo_bf16_to_f64(J.win[win_index(J.g->num_kv_heads, rows, d, b, h, row, 1, i)]);
+      }
+    }
+  }
   std::vector<double> q(d);
   for (int32_t jj = 0; jj < G; ++jj) {
     const int32_t j = h * G + jj;
@@ -502,31 +527,11 @@ int run_pair(const DecodeJob& J, int32_t b, int32_t h) {
   }
   return 0;
 }
-}  // namespace
 
-int kvqo_decode_attention(const kvqo_geom* g, const uint8_t* pool, const void* q, int32_t q_dtype,
-                          int32_t batch, int32_t num_q_heads, const int32_t* block_table,
-                          int32_t max_blocks_per_seq, const int32_t* seq_lens,
-                          double softmax_scale, int32_t form, int32_t nthreads, double* out) {
-  if (!geom_ok(g) || !pool || !q || !out || !seq_lens || !block_table || batch < 0 ||
-      num_q_heads <= 0 || num_q_heads % g->num_kv_heads != 0 || max_blocks_per_seq < 0 ||
-      (form != 0 && form != 1))
-    return -1;
-  DecodeJob J{g,
-              pool,
-              q,
-              q_dtype,
-              batch,
-              num_q_heads,
-              max_blocks_per_seq,
-              block_table,
-              seq_lens,
-              softmax_scale > 0.0 ? softmax_scale
-                                  : 1.0 / std::sqrt(static_cast<double>(g->head_dim)),
-              form,
-              out};
-  const int32_t H = g->num_kv_heads;
-  const int64_t pairs = static_cast<int64_t>(batch) * H;
+// Every (sequence, kv head) pair of a decode job, on up to nthreads threads.
+int run_all(const DecodeJob& J, int32_t nthreads) {
+  const int32_t H = J.g->num_kv_heads;
+  const int64_t pairs = static_cast<int64_t>(J.batch) * H;
   if (nthreads <= 1 || pairs <= 1) {
     for (int64_t w = 0; w < pairs; ++w) {
       const int rc = run_pair(J, static_cast<int32_t>(w / H), static_cast<int32_t>(w % H));
@@ -552,6 +557,87 @@ int kvqo_decode_attention(const kvqo_geom* g, const uint8_t* pool, const void* q
   for (int rc : rcs)
     if (rc) return rc;
   return 0;
+}
+}  // namespace
+
+int kvqo_decode_attention(const kvqo_geom* g, const uint8_t* pool, const void* q, int32_t q_dtype,
+                          int32_t batch, int32_t num_q_heads, const int32_t* block_table,
+                          int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                          double softmax_scale, int32_t form, int32_t nthreads, double* out) {
+  if (!geom_ok(g) || !pool || !q || !out || !seq_lens || !block_table || batch < 0 ||
+      num_q_heads <= 0 || num_q_heads % g->num_kv_heads != 0 || max_blocks_per_seq < 0 ||
+      (form != 0 && form != 1))
+    return -1;
+  DecodeJob J{g,
+              pool,
+              q,
+              q_dtype,
+              batch,
+              num_q_heads,
+              max_blocks_per_seq,
+              block_table,
+              seq_lens,
+              softmax_scale > 0.0 ? softmax_scale
+                                  : 1.0 / std::sqrt(static_cast<double>(g->head_dim)),
+              form,
+              out,
+              nullptr,
+              0,
+              0};
+  return run_all(J, nthreads);
+}
+
+int kvqo_window_append(int32_t d, int32_t num_kv_heads, int32_t sink, int32_t recent, int32_t num_seqs,
+                       uint16_t* win, const uint16_t* k, const uint16_t* v, int64_t token_stride,
+                       const int32_t* seq_ids, const int32_t* positions, int32_t n_tokens) {
+  if (!is_pow2(d) || num_kv_heads <= 0 || sink < 0 || recent < 0 || num_seqs < 0 || n_tokens < 0 ||
+      (n_tokens > 0 && (!win || !k || !v || !seq_ids || !positions)))
+    return -1;
+  const int32_t rows = sink + recent;
+  for (int32_t n = 0; n < n_tokens; ++n) {
+    const int32_t b = seq_ids[n], t = positions[n];
+    if (b < 0) continue;
+    if (b >= num_seqs || t < 0) return -1;
+    for (int32_t h = 0; h < num_kv_heads; ++h) {
+      const int64_t src = static_cast<int64_t>(n) * token_stride + static_cast<int64_t>(h) * d;
+      for (int32_t kv = 0; kv < 2; ++kv) {
+        const uint16_t* x = kv == 0 ? k : v;
+        if (t < sink)
+          for (int32_t i = 0; i < d; ++i) win[win_index(num_kv_heads, rows, d, b, h, t, kv, i)] = x[src + i];
+        if (recent > 0)
+          for (int32_t i = 0; i < d; ++i)
+            win[win_index(num_kv_heads, rows, d, b, h, sink + t % recent, kv, i)] = x[src + i];
+      }
+    }
+  }
+  return 0;
+}
+
+int kvqo_decode_attention_window(const kvqo_geom* g, const uint8_t* pool, const uint16_t* win,
+                                 int32_t sink, int32_t recent, const void* q, int32_t q_dtype,
+                                 int32_t batch, int32_t num_q_heads, const int32_t* block_table,
+                                 int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                                 double softmax_scale, int32_t nthreads, double* out) {
+  if (!geom_ok(g) || !pool || !q || !out || !seq_lens || !block_table || batch < 0 ||
+      num_q_heads <= 0 || num_q_heads % g->num_kv_heads != 0 || max_blocks_per_seq < 0 || sink < 0 ||
+      recent < 0 || (sink + recent > 0 && !win))
+    return -1;
+  DecodeJob J{g,
+              pool,
+              q,
+              q_dtype,
+              batch,
+              num_q_heads,
+              max_blocks_per_seq,
+              block_table,
+              seq_lens,
+              softmax_scale > 0.0 ? softmax_scale : 1.0 / std::sqrt(static_cast<double>(g->head_dim)),
+              0,
+              out,
+              sink + recent > 0 ? win : nullptr,
+              sink,
+              recent};
+  return run_all(J, nthreads);
 }
 
 int kvqo_attention_dense(int32_t d, int32_t num_kv_heads, const void* k, const void* v,

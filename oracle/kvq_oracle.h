@@ -140,6 +140,34 @@ int kvqo_attention_dense(int32_t d, int32_t num_kv_heads, const void* k, const v
                          const void* q_row, int32_t q_dtype, int32_t num_q_heads, int32_t j,
                          double softmax_scale, double* out);
 
+/* ---- bf16 window of sink and recent tokens ------------------------------
+ * ("Kompresja pamięci podręcznej KV..." (encorp.ai), OSCAR section: the first
+ * "sink" tokens and the most recent tokens stay in BF16 while the history is
+ * compressed.)  Reading: for a sequence of length L, position t is kept raw
+ * when t < sink or t >= L - recent; every other position reads its quantized
+ * token from the pool, which holds every position.  The raw rows live in a
+ * window buffer of bf16 [num_seqs][num_kv_heads][sink + recent][2 (K, V)][d]:
+ * row t holds sink position t (t < sink), row sink + t % recent holds a
+ * recent position t.
+ *
+ * Window append: token n (its K and V rows laid out as in the write path,
+ * element (n, h, i) at n*token_stride + h*d + i, bf16 bits) of sequence
+ * seq_ids[n] at position positions[n] is copied to its sink row when
+ * positions[n] < sink and to its ring row when recent > 0; tokens with a
+ * negative sequence id are skipped.  Returns 0, or -1 for bad arguments. */
+int kvqo_window_append(int32_t d, int32_t num_kv_heads, int32_t sink, int32_t recent, int32_t num_seqs,
+                       uint16_t* win, const uint16_t* k, const uint16_t* v, int64_t token_stride,
+                       const int32_t* seq_ids, const int32_t* positions, int32_t n_tokens);
+
+/* Decode attention over the quantized pool with the window's raw rows
+ * standing in at the window positions (sequence b uses window sequence b).
+ * Plain original-domain definition, as kvqo_decode_attention form 0. */
+int kvqo_decode_attention_window(const kvqo_geom* g, const uint8_t* pool, const uint16_t* win,
+                                 int32_t sink, int32_t recent, const void* q, int32_t q_dtype,
+                                 int32_t batch, int32_t num_q_heads, const int32_t* block_table,
+                                 int32_t max_blocks_per_seq, const int32_t* seq_lens,
+                                 double softmax_scale, int32_t nthreads, double* out);
+
 /* ---- byte accounting ---------------------------------------------------- */
 /* Packed bytes per token per kv head: d*(kb+vb)/8 codes + 4 fp16 metadata. */
 double kvqo_packed_bytes_per_token_head(int32_t d, int32_t k_bits, int32_t v_bits);

@@ -331,6 +331,65 @@ def test_attention_brute_force_tiny(orc, syn):
             assert np.allclose(out[b, j], want, rtol=0, atol=1e-12)
 
 
+def test_window_rows_hand_example(orc):
+    """A bf16 window of 2 sink and 3 recent rows ("Kompresja pamięci
+    podręcznej KV..." (encorp.ai), OSCAR section), worked by hand: tokens 0..6
+    of sequence 1 appended in order leave sink rows = tokens 0, 1 and ring rows
+    (t % 3) = tokens 6, 4, 5; sequence 0 is untouched and a token with sequence
+    id -1 is skipped."""
+    d, hkv, sink, recent = 4, 1, 2, 3
+    win = orc.new_window(2, hkv, sink, recent, d=d, fill=0xFFFF)
+    k = np.array([[[10 * t + i for i in range(d)]] for t in range(8)], dtype=np.uint16)
+    v = k + 1000
+    orc.window_append(win, sink, recent, k, v, [1] * 7 + [-1], list(range(7)) + [3])
+    rows = {0: 0, 1: 1, 2: 6, 3: 4, 4: 5}  # window row -> token, by hand
+    for r, t in rows.items():
+        assert list(win[1, 0, r, 0]) == [10 * t + i for i in range(d)]
+        assert list(win[1, 0, r, 1]) == [1000 + 10 * t + i for i in range(d)]
+    assert (win[0] == 0xFFFF).all()
+    with pytest.raises(RuntimeError):
+        orc.window_append(win, sink, recent, k[:1], v[:1], [2], [0])  # no sequence 2
+
+
+def test_window_decode_brute_force(orc, syn):
+    """Attention with sink and recent tokens raw and the rest dequantized,
+    written out with scipy's Hadamard and a hand softmax in numpy; the raw rows
+    come from the workload, not from the window buffer."""
+    wl = syn.Workload("t", 2, 4, 2, 128, [37, 3], 16, syn.BF16, 3, 10.0, 30.0, seed=3)
+    g, pool, k, v = _build_pool(orc, syn, wl)
+    q = wl.query()
+    R = scipy.linalg.hadamard(128) / math.sqrt(128)
+    for sink, recent in ((2, 5), (0, 9), (4, 0), (0, 0)):
+        win = orc.new_window(wl.batch, wl.hkv, sink, recent)
+        for b in range(wl.batch):
+            L = int(wl.seq_lens[b])
+            rows = wl.token_offsets[b] + np.arange(L)
+            orc.window_append(win, sink, recent, k[rows], v[rows], [b] * L, list(range(L)))
+        out = orc.decode_attention_window(g, pool, win, sink, recent, q, wl.dtype, wl.block_table, wl.seq_lens)
+        for b in range(wl.batch):
+            L = int(wl.seq_lens[b])
+            for j in range(wl.hq):
+                h = j // (wl.hq // wl.hkv)
+                K = np.zeros((L, 128))
+                V = np.zeros((L, 128))
+                for t in range(L):
+                    row = wl.token_offsets[b] + t
+                    raw = t < sink or t >= L - recent if recent else t < sink
+                    for M, src, bits in ((K, k, 4), (V, v, 2)):
+                        x = _to_f64(src[row, h], wl.dtype, syn)
+                        if raw:
+                            M[t] = x
+                        else:
+                            c, S, Z, _ = orc.quantize_vector(x, bits)
+                            M[t] = R @ (orc.f16_to_f64(S) * c + orc.f16_to_f64(Z))
+                s = K @ _to_f64(q[b, j], wl.dtype, syn) / math.sqrt(128)
+                p = np.exp(s - s.max())
+                want = (p / p.sum()) @ V
+                assert np.allclose(out[b, j], want, rtol=0, atol=1e-12), (sink, recent, b, j)
+        if sink == 0 and recent == 0:
+            assert np.array_equal(out, orc.decode_attention(g, pool, q, wl.dtype, wl.block_table, wl.seq_lens))
+
+
 def test_folded_form_equals_plain_form(orc, syn):
     wl = syn.Workload("t", 3, 16, 2, 128, [50, 17, 1], 16, syn.BF16, 3, 10.0, 30.0, seed=4, extra_blocks=2)
     g, pool, _, _ = _build_pool(orc, syn, wl)
