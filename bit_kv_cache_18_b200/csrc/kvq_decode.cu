@@ -9,7 +9,8 @@
 //   * loader warps 0-3 (thread t <-> token t of a chunk <-> TMEM lane t):
 //     bring their two segments of each chunk into a private kNV-slot
 //     shared-memory ring with bulk copies (TMA, one instruction per segment)
-//     kNV chunks ahead, after an L2 prefetch six chunks ahead; read them
+//     kNV chunks ahead (the first ones after an L2 prefetch issued before
+//     the dependency wait on the previous kernel); read them
 //     with conflict-free 16-byte loads; spread the key codes (4 bits in the
 //     default k4v2 preset, 2 or 8 in others) to one byte each into tensor
 //     memory (A of QK, 16x256b stores whose fragment layout matches the
@@ -873,19 +874,15 @@ __global__ void __launch_bounds__(Roles<kWide>::kThreads, kWide ? 1 : kMinCtasOf
       const uint2 mr2 = lds64(sb + mslot * kSeg + F::kOffSK + 8 * (lane & 15));
       const bool seg_ok = sm.tbl[kChunkBlocks * c + mblk] >= 0;  // my factor segment is present
       // the slot is read: refill it with chunk c+3 (the reads above are
-      // ordered before the copy's writes by the proxy fence); lanes kSegs ..
-      // 2 kSegs - 1 prefetch the segments of chunk c+6 into L2.  (After a
-      // failed wait no copy is issued any more: see the drain below.)
+      // ordered before the copy's writes by the proxy fence).  (After a
+      // failed wait no copy is issued any more: see the drain below.)  An
+      // L2 prefetch further ahead bought nothing here: three chunks in
+      // flight cover the latency, and the extra instructions sit on this
+      // warp's path, which sets the chunk rate.
       async_proxy_fence();
       __syncwarp();
-      if (!bad) {
-        const int cc = c + kNV + kNV * (lane / kSegs);
-        const int32_t p = lane < 2 * kSegs && cc < nchunks
-                              ? sm.tbl[kChunkBlocks * cc + seg_of<kWide>(warp, lane % kSegs)]
-                              : -1;
-        if (lane >= kSegs && p >= 0) prefetch_l2(pool_h + static_cast<int64_t>(p) * pstride, kSeg);
-        if (c + kNV < nchunks) issue(lane < kSegs ? p : -1, r.i);
-      }
+      if (!bad && c + kNV < nchunks)
+        issue(lane < kSegs ? sm.tbl[kChunkBlocks * (c + kNV) + seg_of<kWide>(warp, lane)] : -1, r.i);
 
       if (c >= kNV) {  // buffers r.i are free once PV(c-3) (issued after QK(c-2)) is done
         if (!mbar_wait<kWaitTag>(&sm.pv_done[r.i], r.ph ^ 1u, abort)) bad = true;

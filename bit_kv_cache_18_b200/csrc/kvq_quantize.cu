@@ -3,14 +3,17 @@
 // Bulk appends (prefill): the rotation of a tile of 128 head vectors is one
 // matrix product on the fifth-generation tensor cores, Y = X H with H the
 // 128 x 128 Sylvester Hadamard matrix (entries +-1, exact in bf16 and fp16,
-// accumulated in fp32).  Each warp stages its 32 rows two tiles ahead with
-// coalesced 16-byte cp.async copies, each lane moves its row, unconverted,
-// into its tensor-memory lane (the A operand), one thread issues the 8-step
-// tcgen05.mma chain (B = H in shared memory) into 128 fp32 columns, and
-// thread t then owns vector t (tensor-memory lane t): one read of its
-// columns gives the moments, range, (S, Z) and codes, packed with fp32x2
-// arithmetic and written as 16-byte stores into the paged segment plus two
-// fp16 stores.  Two CTAs per SM overlap each other's MMA waits.
+// accumulated in fp32), written as two N = 64 halves over the Sylvester
+// blocks, Y0 = X0 H64 + X1 H64 and Y1 = X0 H64 - X1 H64 (16 MMAs of K = 16).
+// Each warp copies its 32 rows of a tile two tiles ahead with 16-byte
+// cp.async straight into a 3-slot ring of A operands in the 128-byte
+// swizzled K-major layout (conflict free, nothing moves twice); one thread
+// issues tile k's MMAs into accumulator k % 2 of tensor memory, so tile k's
+// rotation runs while the CTA reads tile k-1's accumulator.  Thread t owns
+// vector t (tensor-memory lane t): one read of its 128 columns gives the
+// moments, range, (S, Z) and codes, packed with fp32x2 arithmetic and written
+// as 16-byte stores into the paged segment plus two fp16 stores.  Two CTAs
+// per SM overlap each other's barriers and waits.
 //
 // Small appends (decode steps): one warp per vector (quantize_vector_warp in
 // kvq_internal.cuh), butterflies in registers and shuffles.
