@@ -48,6 +48,11 @@ class CacheDesc(ctypes.Structure):
                 ("pool", ctypes.c_void_p)]
 
 
+class WindowDesc(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("num_seqs", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
+                ("sink", ctypes.c_int32), ("recent", ctypes.c_int32)]
+
+
 def lib():
     """Load libkvq.so (raises if it is absent: there is no other path)."""
     global _lib
@@ -77,6 +82,12 @@ def lib():
                                                                i32, vp, i32, vp, i32, f32, vp, ctypes.c_int, vp, sz,
                                                                vp]),
                 "kvq_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_uint32, vp, vp]),
+                "kvq_window_bytes": (sz, [ctypes.POINTER(WindowDesc)]),
+                "kvq_window_append": (ctypes.c_int, [ctypes.POINTER(WindowDesc), vp, vp, i64, vp, vp, i32, vp]),
+                "kvq_decode_window_workspace_bytes": (sz, [dp, i32, i32, i32]),
+                "kvq_decode_attention_window": (ctypes.c_int, [dp, ctypes.POINTER(WindowDesc), vp, ctypes.c_int, i32,
+                                                               i32, vp, i32, vp, i32, f32, vp, ctypes.c_int, vp, sz,
+                                                               vp]),
                 "kvq_last_device_status": (ctypes.c_int, [vp]),
                 "kvq_error_string": (ctypes.c_char_p, [ctypes.c_int]),
             }
@@ -240,6 +251,57 @@ def kvq_decode_attention_noalloc(pool, num_blocks, num_kv_heads, q, block_table,
                                             _ptr(block_table), block_table.shape[1], _ptr(seq_lens), max_seq_len,
                                             softmax_scale, _ptr(out), _dtype_code(out), _stream_ptr(stream))
     _check(rc, "kvq_decode_attention_noalloc")
+
+
+# ---- bf16 window of sink and recent tokens -------------------------------------
+
+def make_window(num_seqs, num_kv_heads, sink, recent, data=None) -> WindowDesc:
+    return WindowDesc(data.data_ptr() if data is not None else None, num_seqs, num_kv_heads, sink, recent)
+
+
+def kvq_window_bytes(num_seqs, num_kv_heads, sink, recent) -> int:
+    return lib().kvq_window_bytes(ctypes.byref(make_window(num_seqs, num_kv_heads, sink, recent)))
+
+
+def new_window(num_seqs, num_kv_heads, sink, recent, device="cuda"):
+    """A zeroed window buffer: bf16 [num_seqs, Hkv, sink + recent, 2, 128]."""
+    import torch
+    if kvq_window_bytes(num_seqs, num_kv_heads, sink, recent) == 0 and num_seqs * (sink + recent) > 0:
+        raise KvqError(KVQ_ERR_INVALID, "kvq_window_bytes")
+    return torch.zeros((num_seqs, num_kv_heads, sink + recent, 2, HEAD_DIM), dtype=torch.bfloat16, device=device)
+
+
+def kvq_window_append(window, sink, recent, k, v, seq_ids, positions, stream=None, token_stride=None):
+    """k, v: [n, ..., Hkv*128] bf16 rows; seq_ids, positions: int32 [n] device."""
+    num_seqs, hkv = window.shape[0], window.shape[1]
+    w = make_window(num_seqs, hkv, sink, recent, window)
+    ts = k.stride(0) if token_stride is None else token_stride
+    rc = lib().kvq_window_append(ctypes.byref(w), _ptr(k), _ptr(v), ts, _ptr(seq_ids), _ptr(positions),
+                                 seq_ids.numel(), _stream_ptr(stream))
+    _check(rc, "kvq_window_append")
+
+
+def new_window_workspace(num_blocks, num_kv_heads, batch, num_q_heads, max_seq_len, device="cuda", preset=(4, 2)):
+    import torch
+    desc = make_desc(num_blocks, num_kv_heads, preset=preset)
+    n = lib().kvq_decode_window_workspace_bytes(ctypes.byref(desc), batch, num_q_heads, max_seq_len)
+    if n == 0:
+        raise KvqError(KVQ_ERR_UNSUPPORTED, "kvq_decode_window_workspace_bytes")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def kvq_decode_attention_window(pool, num_blocks, num_kv_heads, window, sink, recent, q, block_table, seq_lens,
+                                max_seq_len, out, workspace, softmax_scale=0.0, stream=None, preset=(4, 2)):
+    """kvq_decode_attention with the window's raw rows at the sink and recent
+    positions; workspace from new_window_workspace()."""
+    desc = make_desc(num_blocks, num_kv_heads, pool, preset)
+    w = make_window(window.shape[0], window.shape[1], sink, recent, window)
+    batch, hq, _ = q.shape
+    rc = lib().kvq_decode_attention_window(ctypes.byref(desc), ctypes.byref(w), _ptr(q), _dtype_code(q), batch, hq,
+                                           _ptr(block_table), block_table.shape[1], _ptr(seq_lens), max_seq_len,
+                                           softmax_scale, _ptr(out), _dtype_code(out), _ptr(workspace),
+                                           workspace.numel(), _stream_ptr(stream))
+    _check(rc, "kvq_decode_attention_window")
 
 
 def kvq_selftest_wait_timeout(limit_us: int, elapsed_ns=None, stream=None):

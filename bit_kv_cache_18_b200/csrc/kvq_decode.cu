@@ -550,6 +550,202 @@ __device__ __forceinline__ int seg_of(int w, int sg) {
   return kWide ? 2 * (w & 3) + (w >> 2) : 2 * w + sg;
 }
 
+// Split-K ticket of (b, h): one acquire-release add by thread 0 after the
+// CTA barrier that published every thread's record stores (they happen
+// before the add); in the last CTA, the barrier after the add makes every
+// record visible to every thread's loads.  True in the last CTA.
+__device__ __forceinline__ bool take_ticket(const DecodeArgs& a, int b, int h, int* is_last) {
+  if (threadIdx.x == 0) {
+    int t;
+    asm volatile("atom.add.acq_rel.gpu.global.s32 %0, [%1], 1;"
+                 : "=r"(t)
+                 : "l"(a.tickets + b * a.num_kv_heads + h)
+                 : "memory");
+    *is_last = (t == a.nrec - 1);
+  }
+  __syncthreads();
+  return *is_last != 0;
+}
+
+// The last CTA of (b, h) merges the a.nrec records of each of its G heads
+// and writes the outputs.
+template <int G, int kThreads>
+__device__ __forceinline__ void merge_records(const DecodeArgs& a, int b, int h) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // the last CTA of (b, h) merges the splits: warp g takes head g, lane l
+  // dims 4l .. 4l+3 of every split and, in lane s, (m, l) of split s; all
+  // loads of a batch of 16 splits are in flight at once, the weights go
+  // round by shuffles, and batches merge online (max, rescale, sum)
+  const int ns = a.nrec;
+  const float* base = a.partials + (static_cast<int64_t>(b) * a.num_q_heads + h * G) * ns * kPartialFloats;
+  for (int g = warp; g < G; g += kThreads / 32) {
+    const float* hb = base + static_cast<int64_t>(g) * ns * kPartialFloats;
+    float M = -CUDART_INF_F, lsum = 0.0f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s0 = 0; s0 < ns; s0 += 16) {
+      float4 v[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u)
+        v[u] = s0 + u < ns ? __ldcg(reinterpret_cast<const float4*>(hb + static_cast<int64_t>(s0 + u) * kPartialFloats) + lane)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float2 ml = lane < 16 && s0 + lane < ns
+                            ? __ldcg(reinterpret_cast<const float2*>(hb + static_cast<int64_t>(s0 + lane) * kPartialFloats + kHeadDim))
+                            : make_float2(0.f, 0.f);
+      const bool has = ml.y > 0.0f;  // (an empty split has l = 0)
+      float Mb = has ? ml.x : -CUDART_INF_F;
+#pragma unroll
+      for (int o = 16; o; o >>= 1) Mb = fmaxf(Mb, __shfl_xor_sync(0xffffffffu, Mb, o));
+      Mb = fmaxf(Mb, M);
+      const float f = M == -CUDART_INF_F ? 0.0f : ex2(M - Mb);
+      const float w = has ? ex2(ml.x - Mb) : 0.0f;  // weight of split s0 + lane
+      float lw = w * ml.y;
+#pragma unroll
+      for (int o = 16; o; o >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
+      lsum = fmaf(lsum, f, lw);
+      acc.x *= f;
+      acc.y *= f;
+      acc.z *= f;
+      acc.w *= f;
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const float wu = __shfl_sync(0xffffffffu, w, u);
+        acc.x = fmaf(wu, v[u].x, acc.x);
+        acc.y = fmaf(wu, v[u].y, acc.y);
+        acc.z = fmaf(wu, v[u].z, acc.z);
+        acc.w = fmaf(wu, v[u].w, acc.w);
+      }
+      M = Mb;
+    }
+    // normalise and rotate back once, in the layout the merge left (lane l
+    // holds dims 4l .. 4l+3), and store
+    const float inv = lsum > 0.0f ? 1.0f / lsum : 0.0f;
+    float x[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
+    fwht_warp_blocked(x, lane);
+    const int64_t o0 = (static_cast<int64_t>(b) * a.num_q_heads + h * G + g) * kHeadDim + 4 * lane;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) store_from_f32(a.out, a.out_dtype, o0 + k, x[k]);
+  }
+  if (tid == 0) a.tickets[b * a.num_kv_heads + h] = 0;  // ready for the next call
+}
+
+// ---- bf16 window of sink and recent tokens --------------------------------
+// With a window ("Kompresja pamięci podręcznej KV..." (encorp.ai), OSCAR
+// section: the sink and the most recent tokens are kept in BF16), CTA x =
+// nsplit of each (b, h) attends over the window rows of sequence b in fp32
+// and hands its partial to the split-K merge as record nsplit; the split
+// CTAs skip these positions of the pool.  Scores are formed in the original
+// domain (q.k times the softmax scale and log2 e equals the cache's rotated
+// q~.k~), then m = max s, p = 2^(s - m), l = sum p, o = sum p v, and o is
+// rotated once into the cache's domain (R o; R = R^T = R^-1), which is the
+// domain of every other record.  Window position i is sink row i for i <
+// nsink, else position rec_lo + i - nsink in ring row sink + t % recent.
+constexpr int kWinRowsMax = kMaxWindowSink + kMaxWindowRecent;
+template <int G>
+constexpr int kWindowSmemBytes = (G * kHeadDim + G * kWinRowsMax + 2 * G * kHeadDim + 2 * G + 4) * 4;
+
+template <int G, int kThreads>
+__device__ __forceinline__ void window_part(const DecodeArgs& a, uint8_t* smem) {
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  float* qs = reinterpret_cast<float*>(smem);                     // [G][128]: q times the scale (log2 units)
+  float* sc = qs + G * kHeadDim;                                  // [G][kWinRowsMax]: s, then p
+  float* op = sc + G * kWinRowsMax;                               // [2][G][128]: halves of sum p v
+  float2* ml = reinterpret_cast<float2*>(op + 2 * G * kHeadDim);  // [G]: (m, l)
+  int* is_last = reinterpret_cast<int*>(ml + G);
+  pdl_trigger();  // this CTA holds no tensor memory
+  pdl_wait();
+  // the length, cut as the split CTAs cut it (they record a bad one)
+  int L = a.seq_lens[b];
+  L = max(L, 0);
+  L = min(L, a.max_seq_len);
+  L = min(L, a.max_blocks_per_seq * kBlockSize);
+  const int nsink = min(a.win_sink, L);
+  const int rec_lo = a.win_recent > 0 ? max(L - a.win_recent, nsink) : L;
+  const int nw = nsink + (L - rec_lo);  // <= sink + recent <= kWinRowsMax
+  const uint16_t* wb =
+      a.win + (static_cast<int64_t>(b) * a.num_kv_heads + h) * (a.win_sink + a.win_recent) * (2 * kHeadDim);
+  auto row_of = [&](int i) { return i < nsink ? i : a.win_sink + (rec_lo + i - nsink) % a.win_recent; };
+  for (int i = tid; i < G * kHeadDim; i += kThreads)
+    qs[i] = load_as_f32(a.q, a.q_dtype, (static_cast<int64_t>(b) * a.num_q_heads + h * G) * kHeadDim + i) *
+            a.scale_log2;
+  __syncthreads();
+  // s: a thread per window position, all G heads (q from shared memory, the
+  // same address in every lane)
+  for (int i = tid; i < nw; i += kThreads) {
+    const uint4* kr = reinterpret_cast<const uint4*>(wb + static_cast<int64_t>(row_of(i)) * (2 * kHeadDim));
+    float acc[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) acc[g] = 0.0f;
+#pragma unroll 2
+    for (int c = 0; c < kHeadDim / 8; ++c) {
+      const uint4 w = __ldg(kr + c);
+      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+      float kx[8];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        kx[2 * e] = __uint_as_float(ww[e] << 16);
+        kx[2 * e + 1] = __uint_as_float(ww[e] & 0xFFFF0000u);
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float4 q0 = *reinterpret_cast<const float4*>(qs + g * kHeadDim + 8 * c);
+        const float4 q1 = *reinterpret_cast<const float4*>(qs + g * kHeadDim + 8 * c + 4);
+        acc[g] = fmaf(q0.x, kx[0], fmaf(q0.y, kx[1], fmaf(q0.z, kx[2], fmaf(q0.w, kx[3], acc[g]))));
+        acc[g] = fmaf(q1.x, kx[4], fmaf(q1.y, kx[5], fmaf(q1.z, kx[6], fmaf(q1.w, kx[7], acc[g]))));
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) sc[g * kWinRowsMax + i] = acc[g];
+  }
+  __syncthreads();
+  // per head (warp g): m, p = 2^(s - m) in place, l
+  for (int g = warp; g < G; g += kThreads / 32) {
+    float* sg = sc + g * kWinRowsMax;
+    float m = -CUDART_INF_F;
+    for (int i = lane; i < nw; i += 32) m = fmaxf(m, sg[i]);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float l = 0.0f;
+    for (int i = lane; i < nw; i += 32) {
+      const float pv = ex2(sg[i] - m);
+      sg[i] = pv;
+      l += pv;
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    if (lane == 0) ml[g] = nw > 0 ? make_float2(m, l) : make_float2(0.0f, 0.0f);
+  }
+  __syncthreads();
+  // sum p v: thread (half, dim) for the first 256 threads, alternate positions
+  if (tid < 2 * kHeadDim) {
+    const int half = tid >> 7, d = tid & (kHeadDim - 1);
+    float acc[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) acc[g] = 0.0f;
+    for (int i = half; i < nw; i += 2) {
+      const uint16_t vb = wb[static_cast<int64_t>(row_of(i)) * (2 * kHeadDim) + kHeadDim + d];
+      const float v = __uint_as_float(static_cast<uint32_t>(vb) << 16);
+#pragma unroll
+      for (int g = 0; g < G; ++g) acc[g] = fmaf(sc[g * kWinRowsMax + i], v, acc[g]);
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) op[(half * G + g) * kHeadDim + d] = acc[g];
+  }
+  __syncthreads();
+  // rotate into the cache's domain and write record nsplit (warp g: dims 4 lane + k)
+  for (int g = warp; g < G; g += kThreads / 32) {
+    float x[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) x[k] = op[g * kHeadDim + 4 * lane + k] + op[(G + g) * kHeadDim + 4 * lane + k];
+    fwht_warp_blocked(x, lane);
+    float* rg = a.partials + ((static_cast<int64_t>(b) * a.num_q_heads + h * G + g) * a.nrec + a.nsplit) * kPartialFloats;
+    *reinterpret_cast<float4*>(rg + 4 * lane) = make_float4(x[0], x[1], x[2], x[3]);
+    if (lane == 0) *reinterpret_cast<float2*>(rg + kHeadDim) = ml[g];
+  }
+  __syncthreads();
+  if (take_ticket(a, b, h, is_last)) merge_records<G, kThreads>(a, b, h);
+}
+
 template <int G, int KB, int VB, bool kWide>
 __global__ void __launch_bounds__(Roles<kWide>::kThreads, kWide ? 1 : kMinCtasOf<KB, VB>)
     decode_kernel(DecodeArgs a) {
@@ -574,6 +770,11 @@ __global__ void __launch_bounds__(Roles<kWide>::kThreads, kWide ? 1 : kMinCtasOf
   const int lane = tid & 31;
   const bool is_loader = warp < kLoadWarps;
   const bool is_soft = warp >= kLoadWarps && warp < kMmaWarp;
+  static_assert(kWindowSmemBytes<G> <= kSmemBytesOf<kSeg, kWide>, "the window part fits the CTA's shared memory");
+  if (a.win != nullptr && split == a.nsplit) {  // the window's CTA of (b, h)
+    window_part<G, kThreads>(a, smem_raw);
+    return;
+  }
 
   // tensor memory and barriers touch no global memory: set up before
   // waiting for the previous kernel in the stream
@@ -693,7 +894,17 @@ __global__ void __launch_bounds__(Roles<kWide>::kThreads, kWide ? 1 : kMinCtasOf
     L = min(L, a.max_blocks_per_seq * kBlockSize);
   }
   const int nb = (L + kBlockSize - 1) / kBlockSize;
-  const int blk1 = min(nb, blk0 + a.blocks_per_split);
+  // the positions read from the pool: [qlo, qhi) = [0, L) but, with a
+  // window, its sink and recent positions; the split ends at the last block
+  // that holds any
+  int qlo = 0, qhi = L;
+  if (a.win != nullptr) {
+    qlo = min(a.win_sink, L);
+    qhi = a.win_recent > 0 ? max(L - a.win_recent, qlo) : L;
+  }
+  const int blk1 = min(min(nb, blk0 + a.blocks_per_split), (qhi + kBlockSize - 1) / kBlockSize);
+  // a block holds positions read from the pool
+  auto needed = [&](int blk) { return blk * kBlockSize < qhi && (blk + 1) * kBlockSize > qlo; };
   const int nchunks = blk1 > blk0 ? (blk1 - blk0 + kChunkBlocks - 1) / kChunkBlocks : 0;
   bool bad = false;      // a wait ran out: the results are void, the control flow is kept
   bool bad_blk = false;  // a block-table entry outside the pool (its tokens are skipped)
@@ -731,7 +942,7 @@ __global__ void __launch_bounds__(Roles<kWide>::kThreads, kWide ? 1 : kMinCtasOf
 #pragma unroll
     for (int i = 0; i < kNV; ++i) {
       const int j = kChunkBlocks * i + seg_of<kWide>(warp, lane % kSegs);
-      if (!(j < nblk && bfirst[i] >= 0 && bfirst[i] < a.num_blocks)) bfirst[i] = -1;
+      if (!(j < nblk && needed(blk0 + j) && bfirst[i] >= 0 && bfirst[i] < a.num_blocks)) bfirst[i] = -1;
     }
     // the first three chunks' copies go out while the query is rotated (each
     // warp set up its staging ring's barriers before the dependency wait)
@@ -744,7 +955,7 @@ __global__ void __launch_bounds__(Roles<kWide>::kThreads, kWide ? 1 : kMinCtasOf
 #pragma unroll 4
     for (int i = 0; i < kTblPer; ++i) {
       const int j = tid + 32 * kLoadWarps * i;
-      const bool inside = j < nblk;
+      const bool inside = j < nblk && needed(blk0 + j);
       const int32_t p = inside ? __ldg(bt_row + blk0 + j) : -1;
       const bool okp = inside && p >= 0 && p < a.num_blocks;
       bad_blk |= inside && !okp;
@@ -846,8 +1057,10 @@ __global__ void __launch_bounds__(Roles<kWide>::kThreads, kWide ? 1 : kMinCtasOf
     const int mslot = mlive ? mseg : 0;
     const int mblk = seg_of<kWide>(warp, mslot);  // my factor segment's block within a chunk
     const uint32_t mnone = mkind == 2 ? 0xBC00BC00u : 0u;  // the factors of an absent segment (S_V = -1)
-    // the block holding position L-1, for the lanes holding S_V (-2: none)
-    const int blk_last = mkind == 2 ? (L - 1) / kBlockSize : -2;
+    // the blocks holding the ends of [qlo, qhi), for the lanes holding S_V
+    // (-2: none; without a window only the block of position L-1)
+    const int blk_hi = mkind == 2 ? (qhi - 1) / kBlockSize : -2;
+    const int blk_lo = mkind == 2 && (qlo & (kBlockSize - 1)) != 0 ? qlo / kBlockSize : -2;
     const uint32_t my_meta = smem_u32(&sm.meta[0][mkind][16 * mblk + mrow0]);
 #pragma unroll
     for (int i = 0; i < kNV; ++i)  // the deferred chunk, if it is one of the first three
@@ -918,12 +1131,14 @@ __global__ void __launch_bounds__(Roles<kWide>::kThreads, kWide ? 1 : kMinCtasOf
          // the sequence: only in the block holding position L-1)
         uint32_t m0 = seg_ok ? mr2.x : mnone, m1 = seg_ok ? mr2.y : mnone;
         const int blk = blk0 + kChunkBlocks * c + mblk;
-        if (blk == blk_last) {
-          const int nv = L - blk * kBlockSize - mrow0;  // my rows inside the sequence (may be <= 0 or > 4)
-          if (nv < 1) m0 = (m0 & 0xFFFF0000u) | 0xBC00u;
-          if (nv < 2) m0 = (m0 & 0x0000FFFFu) | 0xBC000000u;
-          if (nv < 3) m1 = (m1 & 0xFFFF0000u) | 0xBC00u;
-          if (nv < 4) m1 = (m1 & 0x0000FFFFu) | 0xBC000000u;
+        if (blk == blk_hi || blk == blk_lo) {
+          // my rows k with position p0 + k outside [qlo, qhi): k < nlo or k >= nhi
+          const int p0 = blk * kBlockSize + mrow0;
+          const int nlo = qlo - p0, nhi = qhi - p0;
+          if (0 < nlo || 0 >= nhi) m0 = (m0 & 0xFFFF0000u) | 0xBC00u;
+          if (1 < nlo || 1 >= nhi) m0 = (m0 & 0x0000FFFFu) | 0xBC000000u;
+          if (2 < nlo || 2 >= nhi) m1 = (m1 & 0xFFFF0000u) | 0xBC00u;
+          if (3 < nlo || 3 >= nhi) m1 = (m1 & 0x0000FFFFu) | 0xBC000000u;
         }
         if (mlive) sts64(my_meta + r.i * (4 * kChunkTokens * 2), m0, m1);
       }
@@ -1235,7 +1450,7 @@ __global__ void __launch_bounds__(Roles<kWide>::kThreads, kWide ? 1 : kMinCtasOf
     // With several splits, every thread writes its dim of the split's record
     // (o~[128], m, l per head) straight to the workspace; with one, the
     // normalised o~ goes to shared memory for the output rotation.
-    float* rec = a.partials + ((static_cast<int64_t>(b) * a.num_q_heads + h * G) * a.nsplit + split) * kPartialFloats;
+    float* rec = a.partials + ((static_cast<int64_t>(b) * a.num_q_heads + h * G) * a.nrec + split) * kPartialFloats;
     uint32_t oacc[8];
     tmem_ld8(my_acc, oacc);
     tmem_wait_ld();
@@ -1245,8 +1460,8 @@ __global__ void __launch_bounds__(Roles<kWide>::kThreads, kWide ? 1 : kMinCtasOf
       const float z = (sm.red[wg][gh][1] + sm.red[wg + 1][gh][1]) + (sm.red[wg + 2][gh][1] + sm.red[wg + 3][gh][1]);
       const float lsum = (sm.red[wg][gh][0] + sm.red[wg + 1][gh][0]) + (sm.red[wg + 2][gh][0] + sm.red[wg + 3][gh][0]);
       const float o = fmaf(__uint_as_float(oacc[g]), oscale, z);
-      if (a.nsplit > 1) {
-        float* rg = rec + static_cast<int64_t>(gh) * a.nsplit * kPartialFloats;
+      if (a.nrec > 1) {
+        float* rg = rec + static_cast<int64_t>(gh) * a.nrec * kPartialFloats;
         rg[d] = o;
         if (stok == gh) *reinterpret_cast<float2*>(rg + kHeadDim) = make_float2(mr[g], lsum);
       } else {
@@ -1264,8 +1479,8 @@ __global__ void __launch_bounds__(Roles<kWide>::kThreads, kWide ? 1 : kMinCtasOf
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "n"(kTmemCols));
   pdl_trigger();  // this CTA holds no tensor memory any more
 
-  // ---- 2. output rotation (one split), or ticket and merge ----------------------
-  if (a.nsplit == 1) {
+  // ---- 2. output rotation (one record), or ticket and merge ---------------------
+  if (a.nrec == 1) {
     // rotate back once (warp w owns heads w, w + 9, ...) and store; the CTA
     // barrier above published obuf
     for (int g = warp; g < G; g += kThreads / 32) {
@@ -1279,77 +1494,7 @@ __global__ void __launch_bounds__(Roles<kWide>::kThreads, kWide ? 1 : kMinCtasOf
     }
     return;
   }
-  {
-    // ticket: one acquire-release add by thread 0 after the CTA barrier above
-    // publishes every thread's record stores (they happen before the add)
-    // and, in the last CTA, makes every split's record visible to every
-    // thread's loads below (the barrier after the add)
-    if (tid == 0) {
-      int t;
-      asm volatile("atom.add.acq_rel.gpu.global.s32 %0, [%1], 1;"
-                   : "=r"(t)
-                   : "l"(a.tickets + b * a.num_kv_heads + h)
-                   : "memory");
-      sm.is_last = (t == a.nsplit - 1);
-    }
-    __syncthreads();
-    if (!sm.is_last) return;
-
-    // the last CTA of (b, h) merges the splits: warp g takes head g, lane l
-    // dims 4l .. 4l+3 of every split and, in lane s, (m, l) of split s; all
-    // loads of a batch of 16 splits are in flight at once, the weights go
-    // round by shuffles, and batches merge online (max, rescale, sum)
-    const int ns = a.nsplit;
-    const float* base = a.partials + (static_cast<int64_t>(b) * a.num_q_heads + h * G) * ns * kPartialFloats;
-    for (int g = warp; g < G; g += kThreads / 32) {
-      const float* hb = base + static_cast<int64_t>(g) * ns * kPartialFloats;
-      float M = -CUDART_INF_F, lsum = 0.0f;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int s0 = 0; s0 < ns; s0 += 16) {
-        float4 v[16];
-#pragma unroll
-        for (int u = 0; u < 16; ++u)
-          v[u] = s0 + u < ns ? __ldcg(reinterpret_cast<const float4*>(hb + static_cast<int64_t>(s0 + u) * kPartialFloats) + lane)
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
-        const float2 ml = lane < 16 && s0 + lane < ns
-                              ? __ldcg(reinterpret_cast<const float2*>(hb + static_cast<int64_t>(s0 + lane) * kPartialFloats + kHeadDim))
-                              : make_float2(0.f, 0.f);
-        const bool has = ml.y > 0.0f;  // (an empty split has l = 0)
-        float Mb = has ? ml.x : -CUDART_INF_F;
-#pragma unroll
-        for (int o = 16; o; o >>= 1) Mb = fmaxf(Mb, __shfl_xor_sync(0xffffffffu, Mb, o));
-        Mb = fmaxf(Mb, M);
-        const float f = M == -CUDART_INF_F ? 0.0f : ex2(M - Mb);
-        const float w = has ? ex2(ml.x - Mb) : 0.0f;  // weight of split s0 + lane
-        float lw = w * ml.y;
-#pragma unroll
-        for (int o = 16; o; o >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
-        lsum = fmaf(lsum, f, lw);
-        acc.x *= f;
-        acc.y *= f;
-        acc.z *= f;
-        acc.w *= f;
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const float wu = __shfl_sync(0xffffffffu, w, u);
-          acc.x = fmaf(wu, v[u].x, acc.x);
-          acc.y = fmaf(wu, v[u].y, acc.y);
-          acc.z = fmaf(wu, v[u].z, acc.z);
-          acc.w = fmaf(wu, v[u].w, acc.w);
-        }
-        M = Mb;
-      }
-      // normalise and rotate back once, in the layout the merge left (lane l
-      // holds dims 4l .. 4l+3), and store
-      const float inv = lsum > 0.0f ? 1.0f / lsum : 0.0f;
-      float x[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
-      fwht_warp_blocked(x, lane);
-      const int64_t o0 = (static_cast<int64_t>(b) * a.num_q_heads + h * G + g) * kHeadDim + 4 * lane;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) store_from_f32(a.out, a.out_dtype, o0 + k, x[k]);
-    }
-    if (tid == 0) a.tickets[b * a.num_kv_heads + h] = 0;  // ready for the next call
-  }
+  if (take_ticket(a, b, h, &sm.is_last)) merge_records<G, kThreads>(a, b, h);
 }
 
 template <int G, int KB, int VB, bool kWide>
@@ -1357,7 +1502,7 @@ cudaError_t launch_g(const DecodeArgs& a, cudaStream_t stream) {
   constexpr int kBytes = kSmemBytesOf<Fmt<KB, VB>::kSegBytes, kWide>;
   const cudaError_t e = ensure_smem_limit<decode_kernel<G, KB, VB, kWide>>(kBytes);
   if (e != cudaSuccess) return e;
-  const dim3 grid(a.nsplit, a.num_kv_heads, a.batch);
+  const dim3 grid(a.nsplit + (a.win != nullptr ? 1 : 0), a.num_kv_heads, a.batch);  // (+ the window's CTA)
   return launch_pdl(decode_kernel<G, KB, VB, kWide>, grid, dim3(Roles<kWide>::kThreads), kBytes, stream, a);
 }
 
@@ -1370,7 +1515,7 @@ cudaError_t launch_p(const DecodeArgs& a, cudaStream_t stream) {
     case 8:
       // a grid that the SMs hold at once, one CTA each: the wide role layout
       // (its chunks pass each role in about half the time)
-      if (static_cast<int64_t>(a.nsplit) * a.num_kv_heads * a.batch <= device_sm_count())
+      if (static_cast<int64_t>(a.nsplit + (a.win != nullptr ? 1 : 0)) * a.num_kv_heads * a.batch <= device_sm_count())
         return launch_g<8, KB, VB, true>(a, stream);
       return launch_g<8, KB, VB, false>(a, stream);
     default: return cudaErrorInvalidValue;

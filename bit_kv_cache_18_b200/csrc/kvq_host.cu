@@ -105,7 +105,7 @@ int device_sm_count() {
 // a sequence longer than cap x that many blocks is not supported.
 
 int plan_decode(int32_t batch, int32_t num_kv_heads, int32_t num_q_heads, int32_t max_seq_len,
-                int32_t bps_request, DecodePlan* plan) {
+                int32_t bps_request, DecodePlan* plan, int32_t extra_records) {
   if (batch < 0 || num_kv_heads <= 0 || num_q_heads <= 0 || max_seq_len < 0 || bps_request < 0)
     return KVQ_ERR_INVALID;
   const int64_t nb = (static_cast<int64_t>(max_seq_len) + kBlockSize - 1) / kBlockSize;
@@ -142,8 +142,9 @@ int plan_decode(int32_t batch, int32_t num_kv_heads, int32_t num_q_heads, int32_
   const int64_t nsplit = nb > 0 ? (nb + bps - 1) / bps : 1;
   plan->blocks_per_split = static_cast<int32_t>(bps);
   plan->nsplit = static_cast<int32_t>(nsplit);
+  plan->nrec = static_cast<int32_t>(nsplit + extra_records);
   plan->ticket_bytes = ((static_cast<size_t>(batch) * num_kv_heads * sizeof(int32_t)) + 255) / 256 * 256;
-  plan->partial_bytes = static_cast<size_t>(batch) * num_q_heads * nsplit * kPartialFloats * sizeof(float);
+  plan->partial_bytes = static_cast<size_t>(batch) * num_q_heads * plan->nrec * kPartialFloats * sizeof(float);
   plan->total_bytes = plan->ticket_bytes + plan->partial_bytes;
   return KVQ_OK;
 }
@@ -310,7 +311,8 @@ struct AppendRows {
 int decode_impl(const kvq_cache_desc* desc, const void* q, kvq_dtype q_dtype, int32_t batch, int32_t num_q_heads,
                 const int32_t* block_table, int32_t max_blocks_per_seq, const int32_t* seq_lens,
                 int32_t max_seq_len, float softmax_scale, void* out, kvq_dtype out_dtype, void* workspace,
-                size_t ws_bytes, int32_t blocks_per_split, void* stream, const AppendRows* app) {
+                size_t ws_bytes, int32_t blocks_per_split, void* stream, const AppendRows* app,
+                const kvq_window_desc* win = nullptr) {
   int rc = check_desc(desc);
   if (rc != KVQ_OK) return rc;
   if (batch < 0 || num_q_heads <= 0 || max_blocks_per_seq < 0 || max_seq_len < 0 ||
@@ -324,8 +326,10 @@ int decode_impl(const kvq_cache_desc* desc, const void* q, kvq_dtype q_dtype, in
   if (batch == 0) return KVQ_OK;
   if (!desc->pool || !q || !block_table || !seq_lens || !out) return KVQ_ERR_INVALID;
   if (!aligned16(desc->pool)) return KVQ_ERR_INVALID;
+  const bool use_win = win != nullptr && win->sink + win->recent > 0;
+  if (use_win && batch > win->num_seqs) return KVQ_ERR_INVALID;
   DecodePlan plan;
-  rc = plan_decode(batch, desc->num_kv_heads, num_q_heads, max_seq_len, blocks_per_split, &plan);
+  rc = plan_decode(batch, desc->num_kv_heads, num_q_heads, max_seq_len, blocks_per_split, &plan, use_win ? 1 : 0);
   if (rc != KVQ_OK) return rc;
   if (!workspace || !aligned16(workspace) || ws_bytes < plan.total_bytes) return KVQ_ERR_WORKSPACE;
   if (!std::isfinite(softmax_scale)) return KVQ_ERR_INVALID;
@@ -356,6 +360,10 @@ int decode_impl(const kvq_cache_desc* desc, const void* q, kvq_dtype q_dtype, in
   a.v_new = app ? static_cast<const uint8_t*>(app->v) : nullptr;
   a.new_bf16 = app && app->dtype == KVQ_BF16 ? 1 : 0;
   a.new_stride_bytes = app ? app->token_stride * 2 : 0;
+  a.win = use_win ? static_cast<const uint16_t*>(win->data) : nullptr;
+  a.win_sink = use_win ? win->sink : 0;
+  a.win_recent = use_win ? win->recent : 0;
+  a.nrec = plan.nrec;
   if (!a.status) return KVQ_ERR_CUDA;
   return launch_decode(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
@@ -387,6 +395,71 @@ int kvq_append_decode_attention(const kvq_cache_desc* desc, const void* k_new, c
   const AppendRows app{k_new, v_new, in_dtype, token_stride};
   return decode_impl(desc, q, q_dtype, batch, num_q_heads, block_table, max_blocks_per_seq, seq_lens, max_seq_len,
                      softmax_scale, out, out_dtype, workspace, ws_bytes, 0, stream, &app);
+}
+
+namespace {
+// The geometry of a window descriptor; with need_data, also its buffer.
+int check_window(const kvq_window_desc* w, bool need_data = true) {
+  if (!w || w->num_seqs < 0 || w->num_kv_heads <= 0 || w->sink < 0 || w->sink > kMaxWindowSink ||
+      w->recent < 0 || w->recent > kMaxWindowRecent)
+    return KVQ_ERR_INVALID;
+  if (need_data && w->num_seqs > 0 && w->sink + w->recent > 0 && (!w->data || !aligned16(w->data)))
+    return KVQ_ERR_INVALID;
+  return KVQ_OK;
+}
+}  // namespace
+
+size_t kvq_window_bytes(const kvq_window_desc* w) {
+  if (check_window(w, false) != KVQ_OK) return 0;
+  return static_cast<size_t>(w->num_seqs) * w->num_kv_heads * (w->sink + w->recent) * 2 * kHeadDim * 2;
+}
+
+int kvq_window_append(const kvq_window_desc* w, const void* k, const void* v, int64_t token_stride,
+                      const int32_t* seq_ids, const int32_t* positions, int32_t n_tokens, void* stream) {
+  int rc = check_window(w);
+  if (rc != KVQ_OK) return rc;
+  if (n_tokens < 0) return KVQ_ERR_INVALID;
+  if (n_tokens == 0 || w->sink + w->recent == 0 || w->num_seqs == 0) return KVQ_OK;
+  if (!k || !v || !seq_ids || !positions || !aligned16(k) || !aligned16(v)) return KVQ_ERR_INVALID;
+  if (token_stride < static_cast<int64_t>(w->num_kv_heads) * kHeadDim || token_stride % 8 != 0)
+    return KVQ_ERR_INVALID;
+  WindowAppendArgs a;
+  a.win = static_cast<uint16_t*>(w->data);
+  a.num_seqs = w->num_seqs;
+  a.num_kv_heads = w->num_kv_heads;
+  a.sink = w->sink;
+  a.recent = w->recent;
+  a.k = static_cast<const uint16_t*>(k);
+  a.v = static_cast<const uint16_t*>(v);
+  a.token_stride = token_stride;
+  a.seq_ids = seq_ids;
+  a.positions = positions;
+  a.n_tokens = n_tokens;
+  a.status = device_status_ptr();
+  if (!a.status) return KVQ_ERR_CUDA;
+  return launch_window_append(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+size_t kvq_decode_window_workspace_bytes(const kvq_cache_desc* desc, int32_t batch, int32_t num_q_heads,
+                                         int32_t max_seq_len) {
+  if (check_desc(desc) != KVQ_OK || num_q_heads <= 0 || num_q_heads % desc->num_kv_heads != 0) return 0;
+  DecodePlan plan;
+  if (plan_decode(batch, desc->num_kv_heads, num_q_heads, max_seq_len, 0, &plan, 1) != KVQ_OK) return 0;
+  return plan.total_bytes;
+}
+
+int kvq_decode_attention_window(const kvq_cache_desc* desc, const kvq_window_desc* w, const void* q,
+                                kvq_dtype q_dtype, int32_t batch, int32_t num_q_heads,
+                                const int32_t* block_table, int32_t max_blocks_per_seq,
+                                const int32_t* seq_lens, int32_t max_seq_len, float softmax_scale, void* out,
+                                kvq_dtype out_dtype, void* workspace, size_t ws_bytes, void* stream) {
+  int rc = check_desc(desc);
+  if (rc != KVQ_OK) return rc;
+  rc = check_window(w);
+  if (rc != KVQ_OK) return rc;
+  if (w->num_kv_heads != desc->num_kv_heads) return KVQ_ERR_INVALID;
+  return decode_impl(desc, q, q_dtype, batch, num_q_heads, block_table, max_blocks_per_seq, seq_lens, max_seq_len,
+                     softmax_scale, out, out_dtype, workspace, ws_bytes, 0, stream, nullptr, w);
 }
 
 int kvq_decode_attention(const kvq_cache_desc* desc, const void* q, kvq_dtype q_dtype, int32_t batch,

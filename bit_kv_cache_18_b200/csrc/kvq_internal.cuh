@@ -267,8 +267,29 @@ struct DecodeArgs {
   int32_t new_bf16;
   int64_t new_stride_bytes;
   int32_t k_bits, v_bits;  // preset
+  // optional bf16 window of sink and recent tokens: CTA x = nsplit of each
+  // (b, h) attends over it and hands in record nsplit (nrec = nsplit + 1)
+  const uint16_t* win;  // nullptr: no window (nrec = nsplit)
+  int32_t win_sink, win_recent;
+  int32_t nrec;  // records per (b, query head) in partials
 };
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+
+// Window append (kvq_window_append).
+struct WindowAppendArgs {
+  uint16_t* win;
+  int32_t num_seqs, num_kv_heads, sink, recent;
+  const uint16_t* k;
+  const uint16_t* v;
+  int64_t token_stride;  // elements
+  const int32_t* seq_ids;
+  const int32_t* positions;
+  int32_t n_tokens;
+  int* status;
+};
+cudaError_t launch_window_append(const WindowAppendArgs& a, cudaStream_t stream);
+constexpr int kMaxWindowSink = 64;
+constexpr int kMaxWindowRecent = 1024;
 
 // Failure-detection self-test (kvq_selftest_wait_timeout) and the time after
 // which a kernel's bounded wait gives up.
@@ -279,12 +300,14 @@ uint64_t wait_limit_ns();
 struct DecodePlan {
   int32_t blocks_per_split;
   int32_t nsplit;
+  int32_t nrec;          // records per (b, query head): nsplit + extra_records
   size_t ticket_bytes;   // rounded up to 256
   size_t partial_bytes;
   size_t total_bytes;
 };
 int plan_decode(int32_t batch, int32_t num_kv_heads, int32_t num_q_heads, int32_t max_seq_len,
-                int32_t blocks_per_split_request, DecodePlan* plan);
+                int32_t blocks_per_split_request, DecodePlan* plan,
+                int32_t extra_records = 0);
 
 int device_sm_count();
 int decode_ctas_per_sm();  // resident decode CTAs per SM on the current device

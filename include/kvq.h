@@ -262,6 +262,66 @@ int kvq_decode_attention_noalloc(const kvq_cache_desc* desc, const void* q, kvq_
                                  int32_t max_seq_len, float softmax_scale, void* out,
                                  kvq_dtype out_dtype, void* stream);
 
+/* ---- bf16 window of sink and recent tokens ------------------------------
+ * "Kompresja pamięci podręcznej KV to decyzja infrastrukturalna..."
+ * (encorp.ai), OSCAR section: the first ("sink") tokens and the most recent
+ * tokens of a sequence stay in BF16 while the history is compressed.  Here
+ * the history is the KVarN pool above, which keeps every position; the
+ * window holds the raw rows of the positions read unquantized: for a
+ * sequence of length L, positions t < sink and t >= L - recent.
+ *
+ * Window buffer (device memory the caller owns, 16-byte aligned): bf16
+ * [num_seqs][num_kv_heads][sink + recent][2 (K, V)][128]; row t holds sink
+ * position t (t < sink), row sink + t % recent holds recent position t.
+ * Limits: sink in [0, 64], recent in [0, 1024]. */
+typedef struct {
+  void* data;
+  int32_t num_seqs;
+  int32_t num_kv_heads;
+  int32_t sink;
+  int32_t recent;
+} kvq_window_desc;
+
+/* Bytes of the window buffer: num_seqs * num_kv_heads * (sink + recent) *
+ * 2 * 128 * 2; 0 for an invalid descriptor. */
+size_t kvq_window_bytes(const kvq_window_desc* w);
+
+/* Copy the raw K and V rows of n_tokens new tokens into the window: token n
+ * (bf16, element (n, h, i) of k and v at n*token_stride + h*128 + i, as in
+ * kvq_quantize_append: k and v 16-byte aligned, token_stride >=
+ * num_kv_heads*128 and a multiple of 8) of sequence seq_ids[n] at position positions[n] goes
+ * to its sink row when positions[n] < sink and to its ring row when
+ * recent > 0; a negative sequence id skips the token.  seq_ids and
+ * positions are device int32 arrays.  Call it for every appended token, as
+ * well as kvq_quantize_append (the pool keeps every position, so a token
+ * that leaves the recent window is read from the pool).  A sequence id >=
+ * num_seqs or a negative position is skipped and recorded as
+ * KVQ_ERR_OUT_OF_RANGE.  Asynchronous on the stream. */
+int kvq_window_append(const kvq_window_desc* w, const void* k, const void* v, int64_t token_stride,
+                      const int32_t* seq_ids, const int32_t* positions, int32_t n_tokens, void* stream);
+
+/* Workspace bytes of kvq_decode_attention_window (its split plan has one
+ * record more per head than kvq_decode_attention's: the window's). */
+size_t kvq_decode_window_workspace_bytes(const kvq_cache_desc* desc, int32_t batch, int32_t num_q_heads,
+                                         int32_t max_seq_len);
+
+/* kvq_decode_attention with the window's raw rows standing in at the window
+ * positions of every sequence (sequence b of the batch is window sequence
+ * b; w->num_kv_heads must equal the pool's): attention over positions
+ * 0 .. L-1 where t < sink and t >= L - recent read the window and every
+ * other position reads the pool, as kvq_decode_attention does.  One launch:
+ * the split CTAs skip the window positions of the pool, and one more CTA per
+ * (sequence, kv head) attends over the window rows (in fp32) and hands its
+ * partial (o, m, l), rotated into the cache's domain, to the same split-K
+ * merge.  Same arguments, workspace rules (sized by
+ * kvq_decode_window_workspace_bytes) and status rules as
+ * kvq_decode_attention; batch must not exceed w->num_seqs. */
+int kvq_decode_attention_window(const kvq_cache_desc* desc, const kvq_window_desc* w, const void* q,
+                                kvq_dtype q_dtype, int32_t batch, int32_t num_q_heads,
+                                const int32_t* block_table, int32_t max_blocks_per_seq,
+                                const int32_t* seq_lens, int32_t max_seq_len, float softmax_scale, void* out,
+                                kvq_dtype out_dtype, void* workspace, size_t ws_bytes, void* stream);
+
 /* Synchronise the stream, then read and clear the current device's status
  * word: KVQ_OK, or the first error that a kernel recorded since the last
  * read (KVQ_ERR_OUT_OF_RANGE, KVQ_ERR_DEVICE_TIMEOUT).  Returns

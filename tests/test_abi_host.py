@@ -202,3 +202,55 @@ def test_selftest_rejects_limits_out_of_range(kvq):
     L = kvq.lib()
     assert L.kvq_selftest_wait_timeout(0, None, None) == kvq.KVQ_ERR_INVALID
     assert L.kvq_selftest_wait_timeout(1000001, None, None) == kvq.KVQ_ERR_INVALID
+
+
+def test_window_argument_checks_need_no_device(kvq):
+    """The bf16 window of sink and recent tokens: buffer size, limits (sink
+    <= 64, recent <= 1024), row pointers and strides, the extra record of the
+    window decode's workspace, and the descriptor rules of the window decode;
+    all checked on the host before anything is launched."""
+    L = kvq.lib()
+    assert kvq.kvq_window_bytes(2, 8, 4, 128) == 2 * 8 * 132 * 2 * 128 * 2
+    assert kvq.kvq_window_bytes(3, 1, 64, 1024) == 3 * 1088 * 512
+    for bad in ((2, 8, 65, 0), (2, 8, 0, 1025), (2, 8, -1, 4), (2, 0, 4, 4), (-1, 8, 4, 4)):
+        assert kvq.kvq_window_bytes(*bad) == 0, bad
+    w = kvq.make_window(2, 2, 4, 16)
+    w.data = 0x10000
+    one = ctypes.c_void_p(0x4000)
+    k, v = ctypes.c_void_p(0x5000), ctypes.c_void_p(0x6000)
+
+    def append(win, kk, vv, stride, n):
+        return L.kvq_window_append(ctypes.byref(win), kk, vv, stride, one, one, n, None)
+
+    assert append(w, None, None, 256, 0) == kvq.KVQ_OK  # nothing to copy
+    assert append(w, None, v, 256, 1) == kvq.KVQ_ERR_INVALID
+    assert append(w, ctypes.c_void_p(0x5008), v, 256, 1) == kvq.KVQ_ERR_INVALID
+    assert append(w, k, v, 128, 1) == kvq.KVQ_ERR_INVALID  # a row is 2 heads x 128
+    assert append(w, k, v, 260, 1) == kvq.KVQ_ERR_INVALID  # not a multiple of 8
+    assert append(w, k, v, 256, -1) == kvq.KVQ_ERR_INVALID
+    bad = kvq.make_window(2, 2, 65, 16)
+    bad.data = 0x10000
+    assert append(bad, k, v, 256, 1) == kvq.KVQ_ERR_INVALID
+    nodata = kvq.make_window(2, 2, 4, 16)
+    assert append(nodata, k, v, 256, 1) == kvq.KVQ_ERR_INVALID
+    misaligned = kvq.make_window(2, 2, 4, 16)
+    misaligned.data = 0x10008
+    assert append(misaligned, k, v, 256, 1) == kvq.KVQ_ERR_INVALID
+    # the window decode's workspace holds one record more per query head
+    d = kvq.make_desc(1024, 8)
+    base = L.kvq_decode_workspace_bytes(ctypes.byref(d), 3, 64, 16384)
+    assert L.kvq_decode_window_workspace_bytes(ctypes.byref(d), 3, 64, 16384) == base + 3 * 64 * 132 * 4
+    # descriptor rules: kv heads must match the pool's, the batch must fit the window's sequences
+    d = kvq.make_desc(4, 2)
+    d.pool = 0x1000
+
+    def decode(win, batch, ws, ws_bytes):
+        return L.kvq_decode_attention_window(ctypes.byref(d), ctypes.byref(win), one, kvq.KVQ_BF16, batch, 16, one,
+                                             1, one, 16, 0.0, one, kvq.KVQ_F32, ws, ws_bytes, None)
+
+    w3 = kvq.make_window(2, 3, 4, 16)
+    w3.data = 0x10000
+    assert decode(w3, 1, None, 0) == kvq.KVQ_ERR_INVALID
+    assert decode(w, 3, None, 0) == kvq.KVQ_ERR_INVALID
+    assert decode(w, 1, None, 0) == kvq.KVQ_ERR_WORKSPACE
+    assert decode(bad, 1, None, 0) == kvq.KVQ_ERR_INVALID
