@@ -239,6 +239,8 @@ class QwenStep:
     hq = 64
     hkv = 8
     context = 16384
+    win_sink = 4
+    win_recent = 128
 
     def __init__(self, kvq, torch, dev, seed=0):
         self.kvq, self.torch, self.dev = kvq, torch, dev
@@ -254,8 +256,16 @@ class QwenStep:
         pool0 = kvq.new_pool(self.nblocks, self.hkv, device=dev)
         kvq.kvq_quantize_append(pool0, self.nblocks, self.hkv, k.reshape(T, -1), v.reshape(T, -1),
                                 torch.from_numpy(slots).to(dev))
+        # a bf16 window of the 4 sink and 128 most recent tokens, each layer its own
+        idx = np.concatenate([np.arange(self.win_sink), np.arange(T - self.win_recent, T)]).astype(np.int64)
+        ti = torch.from_numpy(idx).to(dev)
+        win0 = kvq.new_window(1, self.hkv, self.win_sink, self.win_recent, device=dev)
+        kvq.kvq_window_append(win0, self.win_sink, self.win_recent, k.reshape(T, -1)[ti].contiguous(),
+                              v.reshape(T, -1)[ti].contiguous(), torch.zeros(len(idx), dtype=torch.int32, device=dev),
+                              ti.to(torch.int32))
         torch.cuda.synchronize()
         del k, v
+        self.wins = [win0] + [win0.clone() for _ in range(self.layers - 1)]
         self.pools = [pool0] + [pool0.clone() for _ in range(self.layers - 1)]
         self.bt = torch.from_numpy(wl.block_table).to(dev)
         self.lens = torch.from_numpy(wl.seq_lens).to(dev)
@@ -276,6 +286,7 @@ class QwenStep:
         self.out = torch.empty((self.layers, self.batch, self.hq, 128), dtype=torch.bfloat16, device=dev)
         self.h_out = torch.empty(self.out.shape, dtype=torch.bfloat16).pin_memory()
         self.ws = kvq.new_workspace(self.nblocks, self.hkv, self.batch, self.hq, self.context, device=dev)
+        self.wws = kvq.new_window_workspace(self.nblocks, self.hkv, self.batch, self.hq, self.context, device=dev)
 
     @property
     def packed_bytes_per_decode(self):
@@ -297,6 +308,16 @@ class QwenStep:
             else:
                 kvq.kvq_append_decode_attention(self.pools[l], self.nblocks, self.hkv, self.new_k[l], self.new_v[l],
                                                 self.q[l], self.bt, self.lens, self.context, self.out[l], self.ws)
+
+    def step_window(self):
+        """The decode of every layer with its bf16 window of sink and recent
+        tokens (one launch per layer; the window's rows stand in for the
+        pool's at those positions)."""
+        kvq = self.kvq
+        for l in range(self.layers):
+            kvq.kvq_decode_attention_window(self.pools[l], self.nblocks, self.hkv, self.wins[l], self.win_sink,
+                                            self.win_recent, self.q[l], self.bt, self.lens, self.context, self.out[l],
+                                            self.wws)
 
     def tokens_per_step(self):
         return self.batch
@@ -704,6 +725,11 @@ def main():
     dms = time_replays(torch, g_dec, dec_reps) / (dec_reps * stepper.layers)
     achieved = stepper.packed_bytes_per_decode / (dms * 1e-3) / 1e9
     peak, peak_kind = measured_peaks()
+    # the same decode with a bf16 window of sink and recent tokens
+    g_win = graph_of(torch, stepper.step_window)
+    for _ in range(3):
+        g_win.replay()
+    wms = time_replays(torch, g_win, dec_reps) / (dec_reps * stepper.layers)
 
     # end to end: pinned host inputs in, outputs back, every step
     def h2d():
@@ -767,6 +793,9 @@ def main():
             "decode": {"us_per_layer": dms * 1e3, "effective_gbs": achieved,
                        "layer_tokens_per_s": stepper.batch / (dms * 1e-3),
                        "context_tokens_per_s": stepper.context * stepper.batch / (dms * 1e-3)},
+            "window": {"workload": "the decode graph with a bf16 window of 4 sink and 128 recent tokens per layer",
+                       "sink": stepper.win_sink, "recent": stepper.win_recent, "us_per_layer": wms * 1e3,
+                       "decode_us_per_layer": dms * 1e3},
             "quantize": {"workload": "prefill append 16 x 16384 tokens, 8 kv heads, bf16", "us": quant["us"],
                          "gbs": quant["gbs"], "bytes": quant["bytes"], "frac": quant["gbs"] / peak},
             "presets": presets,
@@ -784,7 +813,7 @@ def main():
             line["cpu_baseline_mt"] = cpu_mt
         print(json.dumps(line))
     if dist:
-        del g_step, g_dec
+        del g_step, g_dec, g_win
         dist.destroy_process_group()
     return 0
 

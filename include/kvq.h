@@ -296,7 +296,9 @@ size_t kvq_window_bytes(const kvq_window_desc* w);
  * well as kvq_quantize_append (the pool keeps every position, so a token
  * that leaves the recent window is read from the pool).  A sequence id >=
  * num_seqs or a negative position is skipped and recorded as
- * KVQ_ERR_OUT_OF_RANGE.  Asynchronous on the stream. */
+ * KVQ_ERR_OUT_OF_RANGE.  The tokens of one call must go to distinct rows
+ * (at most one position per ring row of a sequence; the order of writes to
+ * one row within a call is not defined).  Asynchronous on the stream. */
 int kvq_window_append(const kvq_window_desc* w, const void* k, const void* v, int64_t token_stride,
                       const int32_t* seq_ids, const int32_t* positions, int32_t n_tokens, void* stream);
 

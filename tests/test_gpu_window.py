@@ -20,8 +20,8 @@ def _torch():
     return torch
 
 
-def _oracle_pool(wl):
-    g = oracle.geom(num_blocks=wl.num_blocks, num_kv_heads=wl.hkv)
+def _oracle_pool(wl, preset=(4, 2)):
+    g = oracle.geom(num_blocks=wl.num_blocks, num_kv_heads=wl.hkv, k_bits=preset[0], v_bits=preset[1])
     pool = oracle.new_pool(g)
     k = wl.kv_rows(synth.TID_K, 0, wl.total_tokens)
     v = wl.kv_rows(synth.TID_V, 0, wl.total_tokens)
@@ -39,7 +39,7 @@ def _oracle_window(wl, k, v, sink, recent):
     return win
 
 
-def _gpu_decode_window(kvq, wl, pool_np, win_np, sink, recent, q_np, out_dtype="f32"):
+def _gpu_decode_window(kvq, wl, pool_np, win_np, sink, recent, q_np, out_dtype="f32", preset=(4, 2)):
     torch = _torch()
     pool = torch.from_numpy(pool_np).cuda()
     win = torch.from_numpy(win_np.view(np.int16)).cuda().view(torch.bfloat16)
@@ -49,8 +49,9 @@ def _gpu_decode_window(kvq, wl, pool_np, win_np, sink, recent, q_np, out_dtype="
     msl = max(int(wl.seq_lens.max()), 1)
     out = torch.empty((wl.batch, wl.hq, 128), dtype={"f32": torch.float32, "bf16": torch.bfloat16}[out_dtype],
                       device="cuda")
-    ws = kvq.new_window_workspace(wl.num_blocks, wl.hkv, wl.batch, wl.hq, msl)
-    kvq.kvq_decode_attention_window(pool, wl.num_blocks, wl.hkv, win, sink, recent, q, bt, sl, msl, out, ws)
+    ws = kvq.new_window_workspace(wl.num_blocks, wl.hkv, wl.batch, wl.hq, msl, preset=preset)
+    kvq.kvq_decode_attention_window(pool, wl.num_blocks, wl.hkv, win, sink, recent, q, bt, sl, msl, out, ws,
+                                    preset=preset)
     torch.cuda.synchronize()
     assert kvq.kvq_last_device_status() == 0
     return out.float().cpu().numpy().astype(np.float64)
@@ -89,6 +90,17 @@ def test_window_decode_group_sizes(kvq, cuda, G):
     q = wl.query()
     got = _gpu_decode_window(kvq, wl, pool, win, 4, 100, q)
     _check(wl, g, pool, win, 4, 100, q, got)
+
+
+@pytest.mark.parametrize("preset", [(4, 4), (2, 2), (8, 4)])
+def test_window_decode_presets(kvq, cuda, preset):
+    """The other presets: the same window CTA and masking over pools of other widths."""
+    wl = synth.Workload("wp", 3, 16, 2, 128, [900, 40, 2], 16, synth.BF16, 3, 10.0, 30.0, seed=90 + preset[0])
+    g, pool, k, v = _oracle_pool(wl, preset)
+    win = _oracle_window(wl, k, v, 4, 64)
+    q = wl.query()
+    got = _gpu_decode_window(kvq, wl, pool, win, 4, 64, q, preset=preset)
+    _check(wl, g, pool, win, 4, 64, q, got)
 
 
 def test_window_decode_bf16_output(kvq, cuda):
