@@ -640,19 +640,56 @@ __device__ __forceinline__ void merge_records(const DecodeArgs& a, int b, int h)
 // domain of every other record.  Window position i is sink row i for i <
 // nsink, else position rec_lo + i - nsink in ring row sink + t % recent.
 constexpr int kWinRowsMax = kMaxWindowSink + kMaxWindowRecent;
+constexpr int kWinInFlight = 8;  // rows a warp loads ahead
+// warps that walk the window rows: 8, or 16 in the wide layout
+template <int kThreads>
+constexpr int kWinWarpsOf = kThreads / 32 > 16 ? 16 : 8;
+template <int G, int kThreads>
+constexpr int kWindowSmemBytes = (kWinRowsMax * G + kWinWarpsOf<kThreads> * G * kHeadDim + 2 * G + 4) * 4;
+
+// Sum over the warp of G values per lane, G = 1, 2, 4 or 8: log2 G halving
+// exchanges (a lane keeps the half of its values that its lane bit selects
+// and adds the other lane's copy of that half), then plain butterflies over
+// the remaining lane bits.  Lane l returns the sum of value
+// (l >> (5 - log2 G)) & (G - 1).
 template <int G>
-constexpr int kWindowSmemBytes = (G * kHeadDim + G * kWinRowsMax + 2 * G * kHeadDim + 2 * G + 4) * 4;
+__device__ __forceinline__ float warp_sum_heads(float (&v)[G], int lane) {
+  constexpr int kLog = G == 8 ? 3 : G == 4 ? 2 : G == 2 ? 1 : 0;
+#pragma unroll
+  for (int st = 0; st < kLog; ++st) {
+    const int s = 16 >> st;
+    const int n = G >> (st + 1);
+    const bool up = (lane & s) != 0;
+#pragma unroll
+    for (int j = 0; j < n; ++j) {
+      const float send = up ? v[j] : v[j + n];
+      const float keep = up ? v[j + n] : v[j];
+      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, s);
+    }
+  }
+  float x = v[0];
+#pragma unroll
+  for (int s = 16 >> kLog; s >= 1; s >>= 1) x += __shfl_xor_sync(0xffffffffu, x, s);
+  return x;
+}
 
 template <int G, int kThreads>
 __device__ __forceinline__ void window_part(const DecodeArgs& a, uint8_t* smem) {
+  constexpr int kWinWarps = kWinWarpsOf<kThreads>;
+  static_assert(kThreads / 32 >= kWinWarps && kWinWarps >= G, "enough warps for the window's rows and heads");
   const int h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  float* qs = reinterpret_cast<float*>(smem);                     // [G][128]: q times the scale (log2 units)
-  float* sc = qs + G * kHeadDim;                                  // [G][kWinRowsMax]: s, then p
-  float* op = sc + G * kWinRowsMax;                               // [2][G][128]: halves of sum p v
-  float2* ml = reinterpret_cast<float2*>(op + 2 * G * kHeadDim);  // [G]: (m, l)
+  float* pw = reinterpret_cast<float*>(smem);                             // [kWinRowsMax][G]: s, then p
+  float* part = pw + kWinRowsMax * G;                                     // [kWinWarps][G][128]: sums of p v
+  float2* ml = reinterpret_cast<float2*>(part + kWinWarps * G * kHeadDim);  // [G]: (m, l)
   int* is_last = reinterpret_cast<int*>(ml + G);
+  const int wrows = a.win_sink + a.win_recent;
+  const uint16_t* wb = a.win + (static_cast<int64_t>(b) * a.num_kv_heads + h) * wrows * (2 * kHeadDim);
   pdl_trigger();  // this CTA holds no tensor memory
+  // L2 prefetch of this (b, h)'s window rows, before the dependency wait (a
+  // row written by the previous kernel is read after the wait, from L2, the
+  // point of coherence)
+  for (int r = tid; r < wrows; r += kThreads) prefetch_l2(wb + static_cast<int64_t>(r) * (2 * kHeadDim), 4 * kHeadDim);
   pdl_wait();
   // the length, cut as the split CTAs cut it (they record a bad one)
   int L = a.seq_lens[b];
@@ -662,53 +699,63 @@ __device__ __forceinline__ void window_part(const DecodeArgs& a, uint8_t* smem) 
   const int nsink = min(a.win_sink, L);
   const int rec_lo = a.win_recent > 0 ? max(L - a.win_recent, nsink) : L;
   const int nw = nsink + (L - rec_lo);  // <= sink + recent <= kWinRowsMax
-  const uint16_t* wb =
-      a.win + (static_cast<int64_t>(b) * a.num_kv_heads + h) * (a.win_sink + a.win_recent) * (2 * kHeadDim);
   auto row_of = [&](int i) { return i < nsink ? i : a.win_sink + (rec_lo + i - nsink) % a.win_recent; };
-  for (int i = tid; i < G * kHeadDim; i += kThreads)
-    qs[i] = load_as_f32(a.q, a.q_dtype, (static_cast<int64_t>(b) * a.num_q_heads + h * G) * kHeadDim + i) *
-            a.scale_log2;
-  __syncthreads();
-  // s: a thread per window position, all G heads (q from shared memory, the
-  // same address in every lane)
-  for (int i = tid; i < nw; i += kThreads) {
-    const uint4* kr = reinterpret_cast<const uint4*>(wb + static_cast<int64_t>(row_of(i)) * (2 * kHeadDim));
-    float acc[G];
+  if (warp < kWinWarps) {
+    // s: a warp per row (lane l: dims 4l .. 4l+3 of K and of every head's q)
+    float qr[G][4];
 #pragma unroll
-    for (int g = 0; g < G; ++g) acc[g] = 0.0f;
-#pragma unroll 2
-    for (int c = 0; c < kHeadDim / 8; ++c) {
-      const uint4 w = __ldg(kr + c);
-      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-      float kx[8];
+    for (int g = 0; g < G; ++g) {
+      const int64_t q0 = (static_cast<int64_t>(b) * a.num_q_heads + h * G + g) * kHeadDim + 4 * lane;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        kx[2 * e] = __uint_as_float(ww[e] << 16);
-        kx[2 * e + 1] = __uint_as_float(ww[e] & 0xFFFF0000u);
+      for (int k = 0; k < 4; ++k) qr[g][k] = load_as_f32(a.q, a.q_dtype, q0 + k) * a.scale_log2;
+    }
+    for (int i0 = warp; i0 < nw; i0 += kWinWarps * kWinInFlight) {
+      uint2 kr[kWinInFlight];
+#pragma unroll
+      for (int u = 0; u < kWinInFlight; ++u) {
+        const int i = i0 + u * kWinWarps;
+        kr[u] = i < nw ? __ldg(reinterpret_cast<const uint2*>(wb + static_cast<int64_t>(row_of(i)) * (2 * kHeadDim)) + lane)
+                       : make_uint2(0u, 0u);
       }
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float4 q0 = *reinterpret_cast<const float4*>(qs + g * kHeadDim + 8 * c);
-        const float4 q1 = *reinterpret_cast<const float4*>(qs + g * kHeadDim + 8 * c + 4);
-        acc[g] = fmaf(q0.x, kx[0], fmaf(q0.y, kx[1], fmaf(q0.z, kx[2], fmaf(q0.w, kx[3], acc[g]))));
-        acc[g] = fmaf(q1.x, kx[4], fmaf(q1.y, kx[5], fmaf(q1.z, kx[6], fmaf(q1.w, kx[7], acc[g]))));
+      for (int u = 0; u < kWinInFlight; ++u) {
+        const int i = i0 + u * kWinWarps;
+        if (i >= nw) break;  // (warp-uniform)
+        const float k0 = __uint_as_float(kr[u].x << 16), k1 = __uint_as_float(kr[u].x & 0xFFFF0000u);
+        const float k2 = __uint_as_float(kr[u].y << 16), k3 = __uint_as_float(kr[u].y & 0xFFFF0000u);
+        float d[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) d[g] = fmaf(qr[g][0], k0, fmaf(qr[g][1], k1, fmaf(qr[g][2], k2, qr[g][3] * k3)));
+        const float sum = warp_sum_heads<G>(d, lane);
+        constexpr int kShift = G == 8 ? 2 : G == 4 ? 3 : G == 2 ? 4 : 5;
+        if ((lane & ((1 << kShift) - 1)) == 0) pw[i * G + (lane >> kShift)] = sum;
       }
     }
-#pragma unroll
-    for (int g = 0; g < G; ++g) sc[g * kWinRowsMax + i] = acc[g];
   }
+  // the first rows of V go out now, under the barrier and the softmax below
+  uint2 vr[kWinInFlight];
+  auto load_v = [&](int i0) {
+#pragma unroll
+    for (int u = 0; u < kWinInFlight; ++u) {
+      const int i = i0 + u * kWinWarps;
+      vr[u] = i < nw ? __ldg(reinterpret_cast<const uint2*>(wb + static_cast<int64_t>(row_of(i)) * (2 * kHeadDim) +
+                                                            kHeadDim) + lane)
+                     : make_uint2(0u, 0u);
+    }
+  };
+  if (warp < kWinWarps) load_v(warp);
   __syncthreads();
   // per head (warp g): m, p = 2^(s - m) in place, l
-  for (int g = warp; g < G; g += kThreads / 32) {
-    float* sg = sc + g * kWinRowsMax;
+  if (warp < G) {
+    const int g = warp;
     float m = -CUDART_INF_F;
-    for (int i = lane; i < nw; i += 32) m = fmaxf(m, sg[i]);
+    for (int i = lane; i < nw; i += 32) m = fmaxf(m, pw[i * G + g]);
 #pragma unroll
     for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     float l = 0.0f;
     for (int i = lane; i < nw; i += 32) {
-      const float pv = ex2(sg[i] - m);
-      sg[i] = pv;
+      const float pv = ex2(pw[i * G + g] - m);
+      pw[i * G + g] = pv;
       l += pv;
     }
 #pragma unroll
@@ -716,27 +763,49 @@ __device__ __forceinline__ void window_part(const DecodeArgs& a, uint8_t* smem) 
     if (lane == 0) ml[g] = nw > 0 ? make_float2(m, l) : make_float2(0.0f, 0.0f);
   }
   __syncthreads();
-  // sum p v: thread (half, dim) for the first 256 threads, alternate positions
-  if (tid < 2 * kHeadDim) {
-    const int half = tid >> 7, d = tid & (kHeadDim - 1);
-    float acc[G];
+  if (warp < kWinWarps) {
+    // sum p v: a warp per row again (lane l: dims 4l .. 4l+3 of V), the G
+    // probabilities of a row read at one shared-memory address by every lane
+    float acc[G][4];
 #pragma unroll
-    for (int g = 0; g < G; ++g) acc[g] = 0.0f;
-    for (int i = half; i < nw; i += 2) {
-      const uint16_t vb = wb[static_cast<int64_t>(row_of(i)) * (2 * kHeadDim) + kHeadDim + d];
-      const float v = __uint_as_float(static_cast<uint32_t>(vb) << 16);
+    for (int g = 0; g < G; ++g) acc[g][0] = acc[g][1] = acc[g][2] = acc[g][3] = 0.0f;
+    for (int i0 = warp; i0 < nw; i0 += kWinWarps * kWinInFlight) {
+      if (i0 != warp) load_v(i0);
 #pragma unroll
-      for (int g = 0; g < G; ++g) acc[g] = fmaf(sc[g * kWinRowsMax + i], v, acc[g]);
+      for (int u = 0; u < kWinInFlight; ++u) {
+        const int i = i0 + u * kWinWarps;
+        if (i >= nw) break;
+        const float v0 = __uint_as_float(vr[u].x << 16), v1 = __uint_as_float(vr[u].x & 0xFFFF0000u);
+        const float v2 = __uint_as_float(vr[u].y << 16), v3 = __uint_as_float(vr[u].y & 0xFFFF0000u);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float pg = pw[i * G + g];
+          acc[g][0] = fmaf(pg, v0, acc[g][0]);
+          acc[g][1] = fmaf(pg, v1, acc[g][1]);
+          acc[g][2] = fmaf(pg, v2, acc[g][2]);
+          acc[g][3] = fmaf(pg, v3, acc[g][3]);
+        }
+      }
     }
 #pragma unroll
-    for (int g = 0; g < G; ++g) op[(half * G + g) * kHeadDim + d] = acc[g];
+    for (int g = 0; g < G; ++g)
+      *reinterpret_cast<float4*>(part + (warp * G + g) * kHeadDim + 4 * lane) =
+          make_float4(acc[g][0], acc[g][1], acc[g][2], acc[g][3]);
   }
   __syncthreads();
-  // rotate into the cache's domain and write record nsplit (warp g: dims 4 lane + k)
-  for (int g = warp; g < G; g += kThreads / 32) {
-    float x[4];
+  // o over the warps, rotated once into the cache's domain (R o; R = R^T),
+  // written as record nsplit (warp g: dims 4 lane + k)
+  if (warp < G) {
+    const int g = warp;
+    float x[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-    for (int k = 0; k < 4; ++k) x[k] = op[g * kHeadDim + 4 * lane + k] + op[(G + g) * kHeadDim + 4 * lane + k];
+    for (int w = 0; w < kWinWarps; ++w) {
+      const float4 t = *reinterpret_cast<const float4*>(part + (w * G + g) * kHeadDim + 4 * lane);
+      x[0] += t.x;
+      x[1] += t.y;
+      x[2] += t.z;
+      x[3] += t.w;
+    }
     fwht_warp_blocked(x, lane);
     float* rg = a.partials + ((static_cast<int64_t>(b) * a.num_q_heads + h * G + g) * a.nrec + a.nsplit) * kPartialFloats;
     *reinterpret_cast<float4*>(rg + 4 * lane) = make_float4(x[0], x[1], x[2], x[3]);
@@ -770,7 +839,7 @@ __global__ void __launch_bounds__(Roles<kWide>::kThreads, kWide ? 1 : kMinCtasOf
   const int lane = tid & 31;
   const bool is_loader = warp < kLoadWarps;
   const bool is_soft = warp >= kLoadWarps && warp < kMmaWarp;
-  static_assert(kWindowSmemBytes<G> <= kSmemBytesOf<kSeg, kWide>, "the window part fits the CTA's shared memory");
+  static_assert(kWindowSmemBytes<G, kThreads> <= kSmemBytesOf<kSeg, kWide>, "the window part fits the CTA's shared memory");
   if (a.win != nullptr && split == a.nsplit) {  // the window's CTA of (b, h)
     window_part<G, kThreads>(a, smem_raw);
     return;
