@@ -815,7 +815,9 @@ __device__ __forceinline__ void window_part(const DecodeArgs& a, uint8_t* smem) 
   if (take_ticket(a, b, h, is_last)) merge_records<G, kThreads>(a, b, h);
 }
 
-template <int G, int KB, int VB, bool kWide>
+// kWin: the instantiation that takes a bf16 window (a.win set); the others
+// carry no window code at all.
+template <int G, int KB, int VB, bool kWide, bool kWin>
 __global__ void __launch_bounds__(Roles<kWide>::kThreads, kWide ? 1 : kMinCtasOf<KB, VB>)
     decode_kernel(DecodeArgs a) {
   using F = Fmt<KB, VB>;
@@ -840,9 +842,11 @@ __global__ void __launch_bounds__(Roles<kWide>::kThreads, kWide ? 1 : kMinCtasOf
   const bool is_loader = warp < kLoadWarps;
   const bool is_soft = warp >= kLoadWarps && warp < kMmaWarp;
   static_assert(kWindowSmemBytes<G, kThreads> <= kSmemBytesOf<kSeg, kWide>, "the window part fits the CTA's shared memory");
-  if (a.win != nullptr && split == a.nsplit) {  // the window's CTA of (b, h)
-    window_part<G, kThreads>(a, smem_raw);
-    return;
+  if constexpr (kWin) {
+    if (split == a.nsplit) {  // the window's CTA of (b, h)
+      window_part<G, kThreads>(a, smem_raw);
+      return;
+    }
   }
 
   // tensor memory and barriers touch no global memory: set up before
@@ -967,7 +971,7 @@ __global__ void __launch_bounds__(Roles<kWide>::kThreads, kWide ? 1 : kMinCtasOf
   // window, its sink and recent positions; the split ends at the last block
   // that holds any
   int qlo = 0, qhi = L;
-  if (a.win != nullptr) {
+  if constexpr (kWin) {
     qlo = min(a.win_sink, L);
     qhi = a.win_recent > 0 ? max(L - a.win_recent, qlo) : L;
   }
@@ -1566,13 +1570,17 @@ __global__ void __launch_bounds__(Roles<kWide>::kThreads, kWide ? 1 : kMinCtasOf
   if (take_ticket(a, b, h, &sm.is_last)) merge_records<G, kThreads>(a, b, h);
 }
 
+template <int G, int KB, int VB, bool kWide, bool kWin>
+cudaError_t launch_gw(const DecodeArgs& a, cudaStream_t stream) {
+  constexpr int kBytes = kSmemBytesOf<Fmt<KB, VB>::kSegBytes, kWide>;
+  const cudaError_t e = ensure_smem_limit<decode_kernel<G, KB, VB, kWide, kWin>>(kBytes);
+  if (e != cudaSuccess) return e;
+  const dim3 grid(a.nsplit + (kWin ? 1 : 0), a.num_kv_heads, a.batch);  // (+ the window's CTA)
+  return launch_pdl(decode_kernel<G, KB, VB, kWide, kWin>, grid, dim3(Roles<kWide>::kThreads), kBytes, stream, a);
+}
 template <int G, int KB, int VB, bool kWide>
 cudaError_t launch_g(const DecodeArgs& a, cudaStream_t stream) {
-  constexpr int kBytes = kSmemBytesOf<Fmt<KB, VB>::kSegBytes, kWide>;
-  const cudaError_t e = ensure_smem_limit<decode_kernel<G, KB, VB, kWide>>(kBytes);
-  if (e != cudaSuccess) return e;
-  const dim3 grid(a.nsplit + (a.win != nullptr ? 1 : 0), a.num_kv_heads, a.batch);  // (+ the window's CTA)
-  return launch_pdl(decode_kernel<G, KB, VB, kWide>, grid, dim3(Roles<kWide>::kThreads), kBytes, stream, a);
+  return a.win != nullptr ? launch_gw<G, KB, VB, kWide, true>(a, stream) : launch_gw<G, KB, VB, kWide, false>(a, stream);
 }
 
 template <int KB, int VB>
@@ -1630,8 +1638,8 @@ int decode_ctas_per_sm() {
   if (cached[dev] > 0) return cached[dev];
   int n = 0;
   constexpr int kBytes = kSmemBytesOf<Fmt<4, 2>::kSegBytes>;
-  if (ensure_smem_limit<decode_kernel<8, 4, 2, false>>(kBytes) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<8, 4, 2, false>, Roles<false>::kThreads, kBytes) !=
+  if (ensure_smem_limit<decode_kernel<8, 4, 2, false, false>>(kBytes) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<8, 4, 2, false, false>, Roles<false>::kThreads, kBytes) !=
           cudaSuccess ||
       n < 1)
     n = 1;
