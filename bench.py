@@ -16,7 +16,7 @@ figure with pinned host copies inside the timed region; and the CPU oracle's
 throughput on a bounded sample.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kvq|reference]
-                    [--profile qwen3-32b-16k|batched|long|mixed|prefill-quantize]
+                    [--profile qwen3-32b-16k|qwen3-32b-16k-window|batched|long|mixed|prefill-quantize]
 
 --profile times the decode kernel alone on one workload (or, with
 prefill-quantize, the bulk write path on 3 x 16384 fresh tokens) and prints
@@ -55,8 +55,8 @@ BYTES_PER_TOKEN_HEAD = 104
 # does), with the SHA-256 of the kernel code it was taken on (decode_code_sha256:
 # comments stripped).  Reported as roofline.traffic only while the code still
 # has that hash.
-DECODE_TRAFFIC = {"sha256": "5126aea63648e26c2255b948131799c475636ebc37d1dde02cc94a122ab05bde",
-                  "bytes": 13761792}
+DECODE_TRAFFIC = {"sha256": "c4f33186e28d0459040e0ea253d5f85cc3abae1990a281bb1dbc0e466415e57e",
+                  "bytes": 13764352}
 
 
 def decode_code_sha256():
@@ -580,6 +580,7 @@ def host_threads() -> int:
 
 PROFILE_WORKLOADS = {
     "qwen3-32b-16k": lambda: synth.qwen3_32b_layer(0),
+    "qwen3-32b-16k-window": lambda: synth.qwen3_32b_layer(0),
     "batched": lambda: synth.batched(0),
     "long": lambda: synth.long_context(0),
     "mixed": lambda: synth.mixed_decode(0),
@@ -608,6 +609,24 @@ def profile_decode(args):
 
     def launch():
         kvq.kvq_decode_attention(pool, wl.num_blocks, wl.hkv, q, bt, lens, msl, out, ws)
+
+    if args.profile.endswith("-window"):
+        # the same layer with a bf16 window of 4 sink and 128 recent tokens,
+        # from the workload's own rows (one sequence: positions = rows)
+        sink, recent = QwenStep.win_sink, QwenStep.win_recent
+        T = wl.total_tokens
+        idx = np.concatenate([np.arange(sink), np.arange(T - recent, T)])
+        kw = torch.from_numpy(wl.kv_rows(synth.TID_K, 0, T)[idx].view(np.int16)).to(dev).view(torch.bfloat16)
+        vw = torch.from_numpy(wl.kv_rows(synth.TID_V, 0, T)[idx].view(np.int16)).to(dev).view(torch.bfloat16)
+        win = kvq.new_window(1, wl.hkv, sink, recent, device=dev)
+        kvq.kvq_window_append(win, sink, recent, kw.reshape(len(idx), -1), vw.reshape(len(idx), -1),
+                              torch.zeros(len(idx), dtype=torch.int32, device=dev),
+                              torch.from_numpy(idx.astype(np.int32)).to(dev))
+        wws = kvq.new_window_workspace(wl.num_blocks, wl.hkv, wl.batch, wl.hq, msl, device=dev)
+
+        def launch():  # noqa: F811
+            kvq.kvq_decode_attention_window(pool, wl.num_blocks, wl.hkv, win, sink, recent, q, bt, lens, msl, out,
+                                            wws)
 
     for _ in range(args.warmup):
         launch()
