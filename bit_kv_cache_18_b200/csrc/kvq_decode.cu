@@ -1396,6 +1396,8 @@ __global__ void __launch_bounds__(Roles<kWide>::kThreads, kWide ? 1 : kMinCtasOf
         }
       }
       const bool flag = valid && (dmax + e > kTrigger);
+      // (one vote over all softmax threads, the wide layout's two halves
+      // included: a move switches the O buffer that every head's PV runs into)
       const bool any = soft_vote_any<kSoftThreads>(flag);
       if (any) {
         // rare: move the running max of each head to the chunk's max of
