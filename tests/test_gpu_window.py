@@ -103,6 +103,30 @@ def test_window_decode_presets(kvq, cuda, preset):
     _check(wl, g, pool, win, 4, 64, q, got)
 
 
+def test_window_decode_f32_query(kvq, cuda):
+    """fp32 queries (the window CTA and the split CTAs read q in its own dtype)."""
+    torch = _torch()
+    wl = synth.Workload("wq", 2, 16, 2, 128, [700, 90], 16, synth.BF16, 3, 10.0, 30.0, seed=95)
+    g, pool_np, k, v = _oracle_pool(wl)
+    win_np = _oracle_window(wl, k, v, 4, 64)
+    q_np = synth.normal(95, synth.TID_Q, wl.batch * wl.hq * 128, synth.F32).reshape(wl.batch, wl.hq, 128)
+    pool = torch.from_numpy(pool_np).cuda()
+    win = torch.from_numpy(win_np.view(np.int16)).cuda().view(torch.bfloat16)
+    q = torch.from_numpy(np.ascontiguousarray(q_np, dtype=np.float32)).cuda()
+    bt = torch.from_numpy(wl.block_table).cuda()
+    sl = torch.from_numpy(wl.seq_lens).cuda()
+    msl = int(wl.seq_lens.max())
+    out = torch.empty((wl.batch, wl.hq, 128), dtype=torch.float32, device="cuda")
+    ws = kvq.new_window_workspace(wl.num_blocks, wl.hkv, wl.batch, wl.hq, msl)
+    kvq.kvq_decode_attention_window(pool, wl.num_blocks, wl.hkv, win, 4, 64, q, bt, sl, msl, out, ws)
+    torch.cuda.synchronize()
+    assert kvq.kvq_last_device_status() == 0
+    want = oracle.decode_attention_window(g, pool_np, win_np, 4, 64, q_np, synth.F32, wl.block_table, wl.seq_lens,
+                                          nthreads=8)
+    got = out.cpu().numpy().astype(np.float64)
+    assert np.max(np.abs(got - want)) <= helpers.ATTN_TOL
+
+
 def test_window_decode_bf16_output(kvq, cuda):
     wl = synth.Workload("wb", 3, 32, 4, 128, [5000, 64, 129], 16, synth.BF16, 3, 10.0, 30.0, seed=77)
     g, pool, k, v = _oracle_pool(wl)

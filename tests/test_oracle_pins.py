@@ -390,6 +390,22 @@ def test_window_decode_brute_force(orc, syn):
             assert np.array_equal(out, orc.decode_attention(g, pool, q, wl.dtype, wl.block_table, wl.seq_lens))
 
 
+def test_threaded_decode_is_the_single_threaded_one(orc, syn):
+    """The oracle's std::thread split over (sequence, kv head) pairs changes
+    nothing: every pair is computed by one thread in the same order."""
+    wl = syn.Workload("t", 3, 8, 2, 128, [50, 17, 33], 16, syn.BF16, 3, 10.0, 30.0, seed=9)
+    g, pool, _, _ = _build_pool(orc, syn, wl)
+    q = wl.query()
+    one = orc.decode_attention(g, pool, q, wl.dtype, wl.block_table, wl.seq_lens, nthreads=1)
+    for nt in (2, 4, 16):
+        assert np.array_equal(one, orc.decode_attention(g, pool, q, wl.dtype, wl.block_table, wl.seq_lens,
+                                                        nthreads=nt))
+    win = orc.new_window(wl.batch, wl.hkv, 3, 9)
+    assert np.array_equal(orc.decode_attention_window(g, pool, win, 3, 9, q, wl.dtype, wl.block_table, wl.seq_lens),
+                          orc.decode_attention_window(g, pool, win, 3, 9, q, wl.dtype, wl.block_table, wl.seq_lens,
+                                                      nthreads=5))
+
+
 def test_folded_form_equals_plain_form(orc, syn):
     wl = syn.Workload("t", 3, 16, 2, 128, [50, 17, 1], 16, syn.BF16, 3, 10.0, 30.0, seed=4, extra_blocks=2)
     g, pool, _, _ = _build_pool(orc, syn, wl)
